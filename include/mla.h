@@ -1,0 +1,189 @@
+/*
+ * mla.h - C ABI of the VideoMLA latent-window attention library (libmla.so, sm_100a).
+ *
+ * Source of the method: "VideoMLA: Low-Rank Latent KV Cache for Minute-Scale
+ * Autoregressive Video Diffusion" (paper text page), cited as [VideoMLA] with its section.
+ *
+ * The library keeps, per attention layer, a sliding window of the last W latent frames.
+ * Each cached token stores one head-shared content latent c_kv (d_latent scalars) and one
+ * head-shared decoupled 3D-RoPE key k_rope (d_rope scalars): 192 + 32 = 224 scalars instead
+ * of 2 x 12 x 128 = 3072 for a dense per-head K/V cache ([VideoMLA] §1, §3.1, §3.2).
+ * The current chunk's queries attend to the window plus the chunk itself through
+ * W_UK-absorbed scores q_c . c_kv + q_rope . k_rope, an online softmax, P . c_kv, and the
+ * W_UV / W_O up-projections folded into one output projection.
+ *
+ * Conventions shared by every call:
+ *  - Tensors are bf16, row-major, 16-byte aligned device pointers unless stated otherwise.
+ *  - Weights follow the nn.Linear layout [out_features, in_features] with head-major output
+ *    channels (channel c = head * dim + j).
+ *  - Hidden states are [batch, n_frames * F, hidden], F = frame_h * frame_w tokens per latent
+ *    frame, tokens of a frame in row-major (h, w) order ([VideoMLA] App. C.1, S = F H W).
+ *  - Positions are implicit: the i-th frame ever appended has temporal index t = i; a query
+ *    chunk gets the indices the next append will use.  Token k of a frame sits at
+ *    (h, w) = (k / frame_w, k % frame_w).
+ *  - Calls are stream-ordered and asynchronous: append and attention make no host sync.
+ *    `stream` is a cudaStream_t (NULL = legacy default stream).
+ *  - Errors: arguments are validated on the host before anything is launched; a failed check
+ *    returns MLA_ERR_INVALID_ARGUMENT / MLA_ERR_UNSUPPORTED / MLA_ERR_STATE and changes no
+ *    state.  Kernels never trap: a device-side wait that runs out of time sets the cache's
+ *    status word, which mla_cache_sync() returns as MLA_ERR_DEVICE_TIMEOUT.
+ *  - Threading: a cache may be used by one host thread and one stream at a time.
+ */
+#ifndef MLA_LATENT_WINDOW_H
+#define MLA_LATENT_WINDOW_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct mla_cache mla_cache; /* opaque */
+
+typedef enum {
+  MLA_OK = 0,
+  MLA_ERR_INVALID_ARGUMENT = 1, /* bad shape, pointer, alignment or size          */
+  MLA_ERR_UNSUPPORTED = 2,      /* valid for the method, not built into the kernels */
+  MLA_ERR_OUT_OF_MEMORY = 3,    /* cudaMalloc failed                                 */
+  MLA_ERR_CUDA = 4,             /* a CUDA runtime call failed                        */
+  MLA_ERR_DEVICE_TIMEOUT = 5,   /* a kernel's bounded wait ran out (status word)    */
+  MLA_ERR_STATE = 6             /* call not valid in the cache's current state      */
+} mla_status;
+
+/* The problem statement of one attention layer ([VideoMLA] §3, §4.1, App. D.1).
+ * Built kernels: d_latent == 192 and d_rope == 32; hidden a multiple of 128. */
+typedef struct {
+  int32_t hidden;           /* model width d (1536 for Wan-1.3B)                         */
+  int32_t n_heads;          /* n_h (12)                                                  */
+  int32_t d_head;           /* value width per head, W_O input per head (128)            */
+  int32_t d_nope;           /* content-key width per head (128 here; 96 in §4.1 default) */
+  int32_t d_latent;         /* d_c, shared content latent (192)                          */
+  int32_t d_rope;           /* d_h^rope, shared positional key (32)                      */
+  int32_t rope_t, rope_h, rope_w; /* channels per axis; each even, sum == d_rope        */
+  double rope_base;         /* RoPE base (10000); pair i of axis a turns at base^(-2i/d_a) */
+  int32_t frame_h, frame_w; /* latent-frame token grid (30 x 52 -> F = 1560)             */
+  int32_t window_frames;    /* W: cached latent frames kept in the ring (21)             */
+  int32_t max_chunk_frames; /* largest query chunk, in frames (3)                        */
+  int32_t batch;            /* B independent streams sharing the weights                 */
+  float softmax_scale;      /* 0 -> 1 / sqrt(d_nope + d_rope)                            */
+} mla_config;
+
+/* Device bf16 weights, nn.Linear layout [out, in]:
+ *  w_q  [n_heads*d_nope, hidden]    w_qr [n_heads*d_rope, hidden]
+ *  w_dkv[d_latent, hidden]          w_kr [d_rope, hidden]
+ *  w_uk [n_heads*d_nope, d_latent]  w_uv [n_heads*d_head, d_latent]
+ *  w_o  [hidden, n_heads*d_head]
+ * Read only during mla_cache_create; the caller keeps ownership. */
+typedef struct {
+  const void *w_q, *w_qr, *w_dkv, *w_kr, *w_uk, *w_uv, *w_o;
+} mla_weights;
+
+/* Validate a configuration on the host (no GPU needed).  MLA_OK, MLA_ERR_INVALID_ARGUMENT
+ * for values the method does not allow, MLA_ERR_UNSUPPORTED for values the kernels lack. */
+mla_status mla_config_check(const mla_config* cfg);
+
+/* Physical ring slot of (absolute frame index, token in frame): (frame mod W) * F + token
+ * ([VideoMLA] §1, App. D.4: fixed-size sliding window of W latent frames, oldest evicted).
+ * Host only.  MLA_ERR_INVALID_ARGUMENT for frame < 0 or token outside [0, F). */
+mla_status mla_ring_slot(const mla_config* cfg, int64_t frame, int32_t token, int64_t* slot);
+
+/* Bytes of the latent window itself: batch * W * F * (d_latent + d_rope) * 2 (bf16). */
+size_t mla_ring_bytes(const mla_config* cfg);
+
+/* Bytes of device memory mla_cache_create allocates for this configuration (ring with its
+ * chunk tail, absorbed weights, per-call scratch, status word).  0 for an invalid config. */
+size_t mla_cache_device_bytes(const mla_config* cfg);
+
+/* Create a cache on the current device.  Derives and owns the absorbed weights
+ *   W_Qabs[h] = W_UK[h]^T W_Q[h]   (hidden -> d_latent per head, queries)
+ *   W_OV[h]   = W_O[:, h] W_UV[h]  (d_latent per head -> hidden, outputs)
+ * ([VideoMLA] §3.3 reconstructs per-head K/V from the latent through W_UK/W_UV; folding them
+ * into the query and output projections is the standard MLA absorption), the RoPE tables and
+ * a zeroed ring.  Synchronises `stream` once before returning, so the caller may free the
+ * weights afterwards.  *out receives the handle (NULL on failure). */
+mla_status mla_cache_create(const mla_config* cfg, const mla_weights* w, void* stream,
+                            mla_cache** out);
+
+/* Append n_frames >= 1 whole latent frames x [batch, n_frames*F, hidden] to every stream's
+ * window: c_kv = x W_DKV^T and k_rope = RoPE3D(x W_KR^T) at the frames' own (t, h, w), written
+ * to ring slots (t mod W) * F + k ([VideoMLA] §3.1, §3.2).  When n_frames > W only the last W
+ * frames are computed (the others would be evicted within the call). */
+mla_status mla_cache_append(mla_cache* c, const void* x, int32_t n_frames, void* stream);
+
+/* Latent-window attention for one query chunk x_chunk [batch, n_frames*F, hidden],
+ * 1 <= n_frames <= max_chunk_frames, writing out [batch, n_frames*F, hidden].
+ * The chunk attends to the valid window frames plus all of its own tokens (chunk-causal,
+ * [VideoMLA] App. D.4).  The chunk's latents go to a scratch tail, not into the ring: call
+ * mla_cache_append with the final hidden states to make them part of the window.
+ * With an empty window (nothing appended yet) the chunk attends to itself alone. */
+mla_status mla_window_attention(mla_cache* c, const void* x_chunk, int32_t n_frames, void* out,
+                                void* stream);
+
+/* Free everything the cache owns (synchronises the device first).  NULL-safe. */
+void mla_cache_destroy(mla_cache* c);
+
+/* Frames appended so far and frames currently valid in the window (min(appended, W)). */
+mla_status mla_cache_state(const mla_cache* c, int64_t* frames_appended, int32_t* valid_frames);
+
+/* Synchronise `stream` and return the device status word: MLA_OK, or the error a kernel
+ * recorded (MLA_ERR_DEVICE_TIMEOUT).  Reading clears nothing. */
+mla_status mla_cache_sync(mla_cache* c, void* stream);
+
+/* Copy stream b's ring planes to host memory, in physical slot order: ckv_host receives
+ * W*F rows of d_latent bf16, krope_host W*F rows of d_rope bf16 (either may be NULL);
+ * *n_valid_rows = valid_frames * F.  Synchronous; diagnostic, not on the hot path. */
+mla_status mla_cache_read(const mla_cache* c, int32_t b, void* ckv_host, void* krope_host,
+                          int64_t* n_valid_rows);
+
+/* Device pointers of the cache's internal planes, for diagnostics and tests. */
+typedef struct {
+  void* ckv;          /* [batch][rows_per_stream][d_latent]; rows = (W + max_chunk)*F        */
+  void* krope;        /* [batch][rows_per_stream][d_rope]                                    */
+  void* qp;           /* [batch][max_chunk*F*n_heads][d_latent + d_rope]: absorbed, rotated,
+                         pre-scaled queries of the last attention call                      */
+  void* o_lat;        /* [batch][max_chunk*F][n_heads*d_latent]: normalised P . c_kv          */
+  void* w_qcat;       /* [(n_heads+1)*(d_latent+d_rope)][hidden]: per head W_Qabs|W_QR, then
+                         W_DKV|W_KR                                                          */
+  void* w_ov;         /* [hidden][n_heads*d_latent]                                          */
+  int64_t rows_per_stream;
+} mla_debug_buffers;
+mla_status mla_cache_debug_buffers(const mla_cache* c, mla_debug_buffers* out);
+
+/* Synchronous copy of the first min(bytes, size) bytes of an internal buffer to host memory;
+ * *size receives the buffer's full size in bytes (may be NULL).  Diagnostic only. */
+typedef enum {
+  MLA_BUFFER_QP = 0,     /* Qp of the last attention call    */
+  MLA_BUFFER_O_LAT = 1,  /* o_lat of the last attention call */
+  MLA_BUFFER_W_QCAT = 2, /* absorbed query + latent weights  */
+  MLA_BUFFER_W_OV = 3    /* absorbed output weights          */
+} mla_buffer;
+mla_status mla_cache_copy_buffer(const mla_cache* c, mla_buffer which, void* host_dst, size_t bytes,
+                                 size_t* size);
+
+/* Per-kernel device time.  With enable != 0 every later call records CUDA events around each
+ * kernel on its stream; mla_cache_profile_read synchronises those events, returns the sums
+ * since the last read and clears them. */
+typedef enum {
+  MLA_KERNEL_APPEND = 0,     /* fused down-projection + RoPE + ring write              */
+  MLA_KERNEL_QPROJ = 1,      /* absorbed query projection + RoPE + chunk latents       */
+  MLA_KERNEL_ATTENTION = 2,  /* latent-window attention (scores, softmax, P . c_kv)    */
+  MLA_KERNEL_OPROJ = 3,      /* absorbed output projection                             */
+  MLA_KERNEL_COUNT = 4
+} mla_kernel;
+typedef struct {
+  double ms[MLA_KERNEL_COUNT];
+  int64_t launches[MLA_KERNEL_COUNT];
+} mla_profile;
+mla_status mla_cache_profile_enable(mla_cache* c, int32_t enable);
+mla_status mla_cache_profile_read(mla_cache* c, mla_profile* out);
+
+/* Human-readable name of a status, and the last error message recorded on this thread. */
+const char* mla_status_string(mla_status s);
+const char* mla_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MLA_LATENT_WINDOW_H */

@@ -1,0 +1,280 @@
+"""ctypes binding of libmla.so: the C ABI of include/mla.h, same names, argument marshalling only.
+
+Every step of the attention path runs in the library's CUDA kernels; this module only turns
+torch tensors into device pointers and streams into cudaStream_t handles.  There is no fallback:
+if the shared library is missing or the device is not an sm_100 GPU, calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libmla.so")
+
+# mla_status values
+MLA_OK = 0
+MLA_ERR_INVALID_ARGUMENT = 1
+MLA_ERR_UNSUPPORTED = 2
+MLA_ERR_OUT_OF_MEMORY = 3
+MLA_ERR_CUDA = 4
+MLA_ERR_DEVICE_TIMEOUT = 5
+MLA_ERR_STATE = 6
+
+MLA_KERNEL_APPEND, MLA_KERNEL_QPROJ, MLA_KERNEL_ATTENTION, MLA_KERNEL_OPROJ = range(4)
+KERNEL_NAMES = ("append", "qproj", "attention", "oproj")
+
+EXPORTED = (
+    "mla_config_check", "mla_ring_slot", "mla_ring_bytes", "mla_cache_device_bytes",
+    "mla_cache_create", "mla_cache_append", "mla_window_attention", "mla_cache_destroy",
+    "mla_cache_state", "mla_cache_sync", "mla_cache_read", "mla_cache_debug_buffers", "mla_cache_copy_buffer",
+    "mla_cache_profile_enable", "mla_cache_profile_read", "mla_status_string", "mla_last_error",
+)
+
+
+class MLAError(RuntimeError):
+    def __init__(self, status: int, where: str, message: str):
+        super().__init__(f"{where}: {_status_name(status)}: {message}")
+        self.status = status
+
+
+class mla_config(ctypes.Structure):
+    _fields_ = [
+        ("hidden", ctypes.c_int32), ("n_heads", ctypes.c_int32), ("d_head", ctypes.c_int32),
+        ("d_nope", ctypes.c_int32), ("d_latent", ctypes.c_int32), ("d_rope", ctypes.c_int32),
+        ("rope_t", ctypes.c_int32), ("rope_h", ctypes.c_int32), ("rope_w", ctypes.c_int32),
+        ("rope_base", ctypes.c_double),
+        ("frame_h", ctypes.c_int32), ("frame_w", ctypes.c_int32),
+        ("window_frames", ctypes.c_int32), ("max_chunk_frames", ctypes.c_int32),
+        ("batch", ctypes.c_int32), ("softmax_scale", ctypes.c_float),
+    ]
+
+
+class mla_weights(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in ("w_q", "w_qr", "w_dkv", "w_kr", "w_uk", "w_uv", "w_o")]
+
+
+class mla_debug_buffers(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in ("ckv", "krope", "qp", "o_lat", "w_qcat", "w_ov")] + \
+        [("rows_per_stream", ctypes.c_int64)]
+
+
+class mla_profile(ctypes.Structure):
+    _fields_ = [("ms", ctypes.c_double * 4), ("launches", ctypes.c_int64 * 4)]
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libmla.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise ImportError(f"libmla.so not built at {path}: run mla_latent_kv_window_b200/build.py")
+    lib = ctypes.CDLL(path)
+    P, I32, I64, VP = ctypes.POINTER, ctypes.c_int32, ctypes.c_int64, ctypes.c_void_p
+    sig = {
+        "mla_config_check": (I32, [P(mla_config)]),
+        "mla_ring_slot": (I32, [P(mla_config), I64, I32, P(I64)]),
+        "mla_ring_bytes": (ctypes.c_size_t, [P(mla_config)]),
+        "mla_cache_device_bytes": (ctypes.c_size_t, [P(mla_config)]),
+        "mla_cache_create": (I32, [P(mla_config), P(mla_weights), VP, P(VP)]),
+        "mla_cache_append": (I32, [VP, VP, I32, VP]),
+        "mla_window_attention": (I32, [VP, VP, I32, VP, VP]),
+        "mla_cache_destroy": (None, [VP]),
+        "mla_cache_state": (I32, [VP, P(I64), P(I32)]),
+        "mla_cache_sync": (I32, [VP, VP]),
+        "mla_cache_read": (I32, [VP, I32, VP, VP, P(I64)]),
+        "mla_cache_debug_buffers": (I32, [VP, P(mla_debug_buffers)]),
+        "mla_cache_copy_buffer": (I32, [VP, I32, VP, ctypes.c_size_t, P(ctypes.c_size_t)]),
+        "mla_cache_profile_enable": (I32, [VP, I32]),
+        "mla_cache_profile_read": (I32, [VP, P(mla_profile)]),
+        "mla_status_string": (ctypes.c_char_p, [I32]),
+        "mla_last_error": (ctypes.c_char_p, []),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype, fn.argtypes = res, args
+    _lib = lib
+    return lib
+
+
+def _status_name(s: int) -> str:
+    try:
+        return load_library().mla_status_string(s).decode()
+    except Exception:  # pragma: no cover - only when the library itself is missing
+        return str(s)
+
+
+def _check(status: int, where: str) -> None:
+    if status != MLA_OK:
+        raise MLAError(status, where, load_library().mla_last_error().decode())
+
+
+def make_config(dims: dict, frame_h: int, frame_w: int, window_frames: int, max_chunk_frames: int,
+                batch: int = 1, softmax_scale: float = 0.0) -> mla_config:
+    return mla_config(
+        hidden=dims["hidden"], n_heads=dims["n_heads"], d_head=dims["d_head"], d_nope=dims["d_nope"],
+        d_latent=dims["d_latent"], d_rope=dims["d_rope"], rope_t=dims["rope_t"], rope_h=dims["rope_h"],
+        rope_w=dims["rope_w"], rope_base=float(dims["rope_base"]), frame_h=frame_h, frame_w=frame_w,
+        window_frames=window_frames, max_chunk_frames=max_chunk_frames, batch=batch,
+        softmax_scale=softmax_scale)
+
+
+# ---------------------------------------------------------------------------- C names, torch args
+def _stream_handle(stream) -> int:
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream)
+
+
+def _dev_ptr(t, name: str) -> int:
+    import torch
+    if not (t.is_cuda and t.dtype == torch.bfloat16 and t.is_contiguous()):
+        raise ValueError(f"{name} must be a contiguous bf16 CUDA tensor")
+    return int(t.data_ptr())
+
+
+def mla_config_check(cfg: mla_config) -> int:
+    return load_library().mla_config_check(ctypes.byref(cfg))
+
+
+def mla_ring_slot(cfg: mla_config, frame: int, token: int) -> int:
+    out = ctypes.c_int64()
+    _check(load_library().mla_ring_slot(ctypes.byref(cfg), frame, token, ctypes.byref(out)), "mla_ring_slot")
+    return out.value
+
+
+def mla_ring_bytes(cfg: mla_config) -> int:
+    return int(load_library().mla_ring_bytes(ctypes.byref(cfg)))
+
+
+def mla_cache_device_bytes(cfg: mla_config) -> int:
+    return int(load_library().mla_cache_device_bytes(ctypes.byref(cfg)))
+
+
+def mla_cache_create(cfg: mla_config, weights: dict, stream=None) -> int:
+    w = mla_weights(**{k: _dev_ptr(weights[k], k) for k in ("w_q", "w_qr", "w_dkv", "w_kr", "w_uk", "w_uv", "w_o")})
+    h = ctypes.c_void_p()
+    _check(load_library().mla_cache_create(ctypes.byref(cfg), ctypes.byref(w), _stream_handle(stream),
+                                           ctypes.byref(h)), "mla_cache_create")
+    return h.value
+
+
+def mla_cache_append(cache: int, x, n_frames: int, stream=None) -> None:
+    _check(load_library().mla_cache_append(cache, _dev_ptr(x, "x"), n_frames, _stream_handle(stream)),
+           "mla_cache_append")
+
+
+def mla_window_attention(cache: int, x_chunk, n_frames: int, out, stream=None) -> None:
+    _check(load_library().mla_window_attention(cache, _dev_ptr(x_chunk, "x_chunk"), n_frames,
+                                               _dev_ptr(out, "out"), _stream_handle(stream)),
+           "mla_window_attention")
+
+
+def mla_cache_destroy(cache: int) -> None:
+    load_library().mla_cache_destroy(cache)
+
+
+def mla_cache_state(cache: int):
+    fa, vf = ctypes.c_int64(), ctypes.c_int32()
+    _check(load_library().mla_cache_state(cache, ctypes.byref(fa), ctypes.byref(vf)), "mla_cache_state")
+    return fa.value, vf.value
+
+
+def mla_cache_sync(cache: int, stream=None) -> int:
+    return load_library().mla_cache_sync(cache, _stream_handle(stream))
+
+
+def mla_cache_read(cache: int, b: int, ckv_host=None, krope_host=None) -> int:
+    n = ctypes.c_int64()
+    _check(load_library().mla_cache_read(cache, b, None if ckv_host is None else ckv_host.data_ptr(),
+                                         None if krope_host is None else krope_host.data_ptr(),
+                                         ctypes.byref(n)), "mla_cache_read")
+    return n.value
+
+
+def mla_cache_debug_buffers(cache: int) -> mla_debug_buffers:
+    d = mla_debug_buffers()
+    _check(load_library().mla_cache_debug_buffers(cache, ctypes.byref(d)), "mla_cache_debug_buffers")
+    return d
+
+
+MLA_BUFFER_QP, MLA_BUFFER_O_LAT, MLA_BUFFER_W_QCAT, MLA_BUFFER_W_OV = range(4)
+
+
+def mla_cache_copy_buffer(cache: int, which: int, host_out) -> int:
+    """Copy the start of an internal buffer into the CPU tensor host_out; returns the buffer size."""
+    size = ctypes.c_size_t()
+    _check(load_library().mla_cache_copy_buffer(cache, which, host_out.data_ptr(),
+                                                host_out.numel() * host_out.element_size(),
+                                                ctypes.byref(size)), "mla_cache_copy_buffer")
+    return size.value
+
+
+def mla_cache_profile_enable(cache: int, enable: bool) -> None:
+    _check(load_library().mla_cache_profile_enable(cache, int(bool(enable))), "mla_cache_profile_enable")
+
+
+def mla_cache_profile_read(cache: int) -> dict:
+    p = mla_profile()
+    _check(load_library().mla_cache_profile_read(cache, ctypes.byref(p)), "mla_cache_profile_read")
+    return {KERNEL_NAMES[k]: (p.ms[k], p.launches[k]) for k in range(4)}
+
+
+# ---------------------------------------------------------------------------- convenience object
+class LatentWindowCache:
+    """One layer's latent window on the current CUDA device (owns the C handle)."""
+
+    def __init__(self, dims: dict, weights: dict, frame_h: int, frame_w: int, window_frames: int,
+                 max_chunk_frames: int, batch: int = 1, softmax_scale: float = 0.0, stream=None):
+        self.cfg = make_config(dims, frame_h, frame_w, window_frames, max_chunk_frames, batch, softmax_scale)
+        self.F = frame_h * frame_w
+        self.handle = mla_cache_create(self.cfg, weights, stream)
+
+    def append(self, x, stream=None) -> None:
+        n = x.shape[-2] // self.F
+        mla_cache_append(self.handle, x, n, stream)
+
+    def attention(self, x_chunk, out=None, stream=None):
+        import torch
+        if out is None:
+            out = torch.empty_like(x_chunk)
+        mla_window_attention(self.handle, x_chunk, x_chunk.shape[-2] // self.F, out, stream)
+        return out
+
+    def state(self):
+        return mla_cache_state(self.handle)
+
+    def sync(self, stream=None) -> None:
+        _check(mla_cache_sync(self.handle, stream), "mla_cache_sync")
+
+    def read_ring(self, b: int = 0):
+        """(ckv [W*F, 192], krope [W*F, 32]) of stream b in physical slot order, and the valid row count."""
+        import torch
+        W = self.cfg.window_frames
+        ckv = torch.empty(W * self.F, self.cfg.d_latent, dtype=torch.bfloat16)
+        kr = torch.empty(W * self.F, self.cfg.d_rope, dtype=torch.bfloat16)
+        n = mla_cache_read(self.handle, b, ckv, kr)
+        return ckv, kr, n
+
+    def copy_buffer(self, which: int, shape):
+        """Host copy (bf16 tensor of `shape`) of an internal buffer: MLA_BUFFER_QP, _O_LAT, _W_QCAT, _W_OV."""
+        import torch
+        out = torch.empty(shape, dtype=torch.bfloat16)
+        mla_cache_copy_buffer(self.handle, which, out)
+        return out
+
+    def close(self) -> None:
+        if getattr(self, "handle", None):
+            mla_cache_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

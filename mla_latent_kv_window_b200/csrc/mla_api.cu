@@ -1,0 +1,688 @@
+// mla_api.cu - the C ABI of libmla.so (declared in include/mla.h): host-side validation,
+// cache state, absorbed-weight derivation, tensor maps and kernel launches.
+//
+// Path of one attention call (VideoMLA paper page, §3.1-§3.3, App. D.4):
+//   1. tc_gemm<224, kEpiLatent>   x_chunk x [W_Qabs|W_QR per head ; W_DKV|W_KR]^T
+//        heads  -> Qp[(q,h)] = [W_UK[h]^T q_nope | RoPE3D(q_rope)] * scale * log2 e
+//        latent -> chunk tail rows (c_kv, RoPE3D k_rope)
+//   2. window_attn_kernel          o_lat[(q,h)] = softmax(Qp . [c_kv|k_rope]^T) c_kv
+//   3. tc_gemm<256, kEpiStore>    out = o_lat x W_OV^T,  W_OV[h] = W_O[:, h] W_UV[h]
+// An append is step 1's latent half written to ring slots (t mod W) * F + k.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "../../include/mla.h"
+#include "gemm_tc.cuh"
+#include "window_attn.cuh"
+
+namespace {
+
+using mla::EpiArgs;
+using mla::RopeBands;
+
+constexpr int kLatent = 192;
+constexpr int kRope = 32;
+constexpr int kQK = kLatent + kRope;  // 224
+
+// Pipeline depths of the launched kernel variants.
+constexpr int kProjStages = 4;      // 4 x 44 KB: one CTA per SM, deep enough for HBM latency
+constexpr int kOutStages = 4;
+constexpr int kAttnStages = 3;      // 3 KV tiles in flight (P kept in tensor memory)
+constexpr bool kAttnPInTmem = true;
+
+thread_local std::string g_last_error;
+
+mla_status fail(mla_status s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return s;
+}
+
+#define MLA_CUDA(call)                                                                \
+  do {                                                                                \
+    cudaError_t e_ = (call);                                                          \
+    if (e_ != cudaSuccess)                                                            \
+      return fail(e_ == cudaErrorMemoryAllocation ? MLA_ERR_OUT_OF_MEMORY : MLA_ERR_CUDA, \
+                  "%s failed: %s", #call, cudaGetErrorString(e_));                    \
+  } while (0)
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// ------------------------------------------------------------------------------ tensor maps
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 3-D bf16 map: (inner, rows, batch) with byte strides; box (box_inner, box_rows, 1).
+mla_status make_map(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows,
+                    uint64_t batch, uint64_t row_bytes, uint64_t batch_bytes, uint32_t box_inner,
+                    uint32_t box_rows, CUtensorMapSwizzle swz) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return fail(MLA_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+  cuuint64_t dims[3] = {inner, rows, batch};
+  cuuint64_t strides[2] = {row_bytes, batch_bytes};
+  cuuint32_t box[3] = {box_inner, box_rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    return fail(MLA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d): inner=%llu rows=%llu batch=%llu",
+                (int)r, (unsigned long long)inner, (unsigned long long)rows,
+                (unsigned long long)batch);
+  return MLA_OK;
+}
+
+// ------------------------------------------------------------------------------ kernels
+// Create-time derivation of the absorbed weights (fp32 accumulation, one bf16 rounding).
+// Wqcat rows, per head h: [h*224, h*224+192) = W_UK[h]^T W_Q[h], [h*224+192, h*224+224) = W_QR[h];
+// then [n_h*224, n_h*224+192) = W_DKV and [n_h*224+192, (n_h+1)*224) = W_KR.
+__global__ void build_wqcat_kernel(const __nv_bfloat16* __restrict__ w_q,
+                                   const __nv_bfloat16* __restrict__ w_qr,
+                                   const __nv_bfloat16* __restrict__ w_dkv,
+                                   const __nv_bfloat16* __restrict__ w_kr,
+                                   const __nv_bfloat16* __restrict__ w_uk,
+                                   __nv_bfloat16* __restrict__ wqcat, int hidden, int n_heads,
+                                   int d_nope) {
+  const int k = blockIdx.x * blockDim.x + threadIdx.x;
+  const int rowq = blockIdx.y;  // 0 .. (n_heads+1)*224 - 1
+  if (k >= hidden) return;
+  const int h = rowq / kQK;
+  const int c = rowq % kQK;
+  float acc = 0.f;
+  if (h < n_heads) {
+    if (c < kLatent) {
+      for (int j = 0; j < d_nope; ++j) {
+        const int r = h * d_nope + j;
+        acc += __bfloat162float(w_uk[(size_t)r * kLatent + c]) *
+               __bfloat162float(w_q[(size_t)r * hidden + k]);
+      }
+    } else {
+      acc = __bfloat162float(w_qr[(size_t)(h * kRope + c - kLatent) * hidden + k]);
+    }
+  } else {
+    acc = c < kLatent ? __bfloat162float(w_dkv[(size_t)c * hidden + k])
+                      : __bfloat162float(w_kr[(size_t)(c - kLatent) * hidden + k]);
+  }
+  wqcat[(size_t)rowq * hidden + k] = __float2bfloat16_rn(acc);
+}
+
+// W_OV[o][h*192 + c] = sum_j W_O[o][h*d_head + j] * W_UV[h*d_head + j][c].
+__global__ void build_wov_kernel(const __nv_bfloat16* __restrict__ w_o,
+                                 const __nv_bfloat16* __restrict__ w_uv,
+                                 __nv_bfloat16* __restrict__ wov, int hidden, int n_heads,
+                                 int d_head) {
+  const int col = blockIdx.x * blockDim.x + threadIdx.x;  // h*192 + c
+  const int o = blockIdx.y;
+  if (col >= n_heads * kLatent) return;
+  const int h = col / kLatent;
+  const int c = col % kLatent;
+  const int in_o = n_heads * d_head;
+  float acc = 0.f;
+  for (int j = 0; j < d_head; ++j) {
+    const int r = h * d_head + j;
+    acc += __bfloat162float(w_o[(size_t)o * in_o + r]) *
+           __bfloat162float(w_uv[(size_t)r * kLatent + c]);
+  }
+  wov[(size_t)o * (n_heads * kLatent) + col] = __float2bfloat16_rn(acc);
+}
+
+template <typename K>
+mla_status set_smem(K kernel, int bytes) {
+  MLA_CUDA(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
+  return MLA_OK;
+}
+
+}  // namespace
+
+// ------------------------------------------------------------------------------ the cache
+struct mla_cache {
+  mla_config cfg;
+  int F = 0;
+  int64_t rows_per_stream = 0;     // (W + max_chunk) * F
+  int64_t max_q_tokens = 0;        // max_chunk * F
+  int64_t frames_appended = 0;
+  float softmax_scale = 0.f;
+  RopeBands rope{};
+  int device = 0;
+
+  __nv_bfloat16* ckv = nullptr;
+  __nv_bfloat16* krope = nullptr;
+  __nv_bfloat16* qp = nullptr;
+  __nv_bfloat16* o_lat = nullptr;
+  __nv_bfloat16* wqcat = nullptr;
+  __nv_bfloat16* wov = nullptr;
+  int* status = nullptr;
+
+  CUtensorMap map_wqcat{};         // B operand of the projections: box 64 x 224
+  CUtensorMap map_wov{};           // B operand of the output projection: box 64 x out_bn
+  int out_bn = 256;
+
+  bool profiling = false;
+  struct Rec {
+    int kind;
+    cudaEvent_t a, b;
+  };
+  std::vector<Rec> pending;
+  std::vector<cudaEvent_t> pool;
+  double prof_ms[MLA_KERNEL_COUNT] = {0, 0, 0, 0};
+  int64_t prof_n[MLA_KERNEL_COUNT] = {0, 0, 0, 0};
+};
+
+namespace {
+
+cudaEvent_t take_event(mla_cache* c) {
+  if (!c->pool.empty()) {
+    cudaEvent_t e = c->pool.back();
+    c->pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+  return e;
+}
+
+struct ProfScope {
+  mla_cache* c;
+  int kind;
+  cudaStream_t s;
+  cudaEvent_t a = nullptr;
+  ProfScope(mla_cache* c_, int k, cudaStream_t s_) : c(c_), kind(k), s(s_) {
+    if (c->profiling && (a = take_event(c)) != nullptr) cudaEventRecord(a, s);
+  }
+  ~ProfScope() {
+    if (!a) return;
+    cudaEvent_t b = take_event(c);
+    if (!b) {
+      c->pool.push_back(a);
+      return;
+    }
+    cudaEventRecord(b, s);
+    c->pending.push_back({kind, a, b});
+  }
+};
+
+mla_status check_launch(const char* what) {
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(MLA_ERR_CUDA, "%s launch failed: %s", what, cudaGetErrorString(e));
+  return MLA_OK;
+}
+
+RopeBands make_bands(const mla_config& cfg) {
+  RopeBands rb{};
+  int p = 0;
+  const int dims[3] = {cfg.rope_t, cfg.rope_h, cfg.rope_w};
+  for (int a = 0; a < 3; ++a)
+    for (int i = 0; i < dims[a] / 2; ++i, ++p) {
+      rb.axis[p] = a;
+      rb.freq[p] = std::pow(cfg.rope_base, -2.0 * i / dims[a]);
+    }
+  return rb;
+}
+
+// Launch the latent/query projection GEMM over `rows` rows of x per stream.
+mla_status launch_latent_gemm(mla_cache* c, const void* x, int64_t rows, int64_t x_batch_rows,
+                              int grid_y, int latent_y, int b_row0, int ring_mode, int64_t t0,
+                              int64_t base_row, cudaStream_t st) {
+  const mla_config& cfg = c->cfg;
+  CUtensorMap map_x;
+  mla_status s = make_map(&map_x, x, cfg.hidden, rows, cfg.batch, (uint64_t)cfg.hidden * 2,
+                          (uint64_t)x_batch_rows * cfg.hidden * 2, 64, 128,
+                          CU_TENSOR_MAP_SWIZZLE_128B);
+  if (s != MLA_OK) return s;
+  EpiArgs ep{};
+  ep.ckv = c->ckv;
+  ep.krope = c->krope;
+  ep.rows_per_stream = c->rows_per_stream;
+  ep.qp = c->qp;
+  ep.qp_rows_per_stream = c->max_q_tokens * cfg.n_heads;
+  ep.latent_y = latent_y;
+  ep.n_heads = cfg.n_heads;
+  ep.ring_mode = ring_mode;
+  ep.t0 = t0;
+  ep.window_frames = cfg.window_frames;
+  ep.tokens_per_frame = c->F;
+  ep.frame_w = cfg.frame_w;
+  ep.base_row = base_row;
+  ep.q_scale = c->softmax_scale * 1.4426950408889634f;
+  ep.rope = c->rope;
+  using Sm = mla::GemmSmem<kQK, kProjStages>;
+  dim3 grid((unsigned)((rows + 127) / 128), (unsigned)grid_y, (unsigned)cfg.batch);
+  mla::tc_gemm_kernel<kQK, kProjStages, mla::kEpiLatent>
+      <<<grid, mla::kGemmThreads, Sm::kBytes, st>>>(map_x, c->map_wqcat, (int)rows, cfg.hidden,
+                                                   b_row0, ep, c->status);
+  return check_launch("latent projection");
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* mla_status_string(mla_status s) {
+  switch (s) {
+    case MLA_OK: return "MLA_OK";
+    case MLA_ERR_INVALID_ARGUMENT: return "MLA_ERR_INVALID_ARGUMENT";
+    case MLA_ERR_UNSUPPORTED: return "MLA_ERR_UNSUPPORTED";
+    case MLA_ERR_OUT_OF_MEMORY: return "MLA_ERR_OUT_OF_MEMORY";
+    case MLA_ERR_CUDA: return "MLA_ERR_CUDA";
+    case MLA_ERR_DEVICE_TIMEOUT: return "MLA_ERR_DEVICE_TIMEOUT";
+    case MLA_ERR_STATE: return "MLA_ERR_STATE";
+  }
+  return "MLA_ERR_UNKNOWN";
+}
+
+const char* mla_last_error(void) { return g_last_error.c_str(); }
+
+mla_status mla_config_check(const mla_config* cfg) {
+  if (!cfg) return fail(MLA_ERR_INVALID_ARGUMENT, "config is NULL");
+  const mla_config& c = *cfg;
+  if (c.hidden <= 0 || c.n_heads <= 0 || c.d_head <= 0 || c.d_nope <= 0 || c.d_latent <= 0 ||
+      c.d_rope < 0)
+    return fail(MLA_ERR_INVALID_ARGUMENT, "dimensions must be positive");
+  if (c.rope_t < 0 || c.rope_h < 0 || c.rope_w < 0 || (c.rope_t | c.rope_h | c.rope_w) & 1)
+    return fail(MLA_ERR_INVALID_ARGUMENT, "RoPE axis widths must be even and non-negative");
+  if (c.rope_t + c.rope_h + c.rope_w != c.d_rope)
+    return fail(MLA_ERR_INVALID_ARGUMENT, "rope_t + rope_h + rope_w must equal d_rope");
+  if (!(c.rope_base > 0.0) || !std::isfinite(c.rope_base))
+    return fail(MLA_ERR_INVALID_ARGUMENT, "rope_base must be positive and finite");
+  if (c.frame_h <= 0 || c.frame_w <= 0 || c.window_frames <= 0 || c.max_chunk_frames <= 0 ||
+      c.batch <= 0)
+    return fail(MLA_ERR_INVALID_ARGUMENT, "frame grid, window, chunk and batch must be >= 1");
+  if (!(c.softmax_scale >= 0.f) || !std::isfinite(c.softmax_scale))
+    return fail(MLA_ERR_INVALID_ARGUMENT, "softmax_scale must be finite and >= 0");
+  const int64_t F = (int64_t)c.frame_h * c.frame_w;
+  const int64_t rows = (int64_t)(c.window_frames + (int64_t)c.max_chunk_frames) * F;
+  if (rows > (int64_t)1 << 30 || (int64_t)c.max_chunk_frames * F * c.n_heads > (int64_t)1 << 30)
+    return fail(MLA_ERR_INVALID_ARGUMENT, "window or chunk too large (row index overflow)");
+  if ((int64_t)c.batch * rows * kQK > ((int64_t)1 << 40))
+    return fail(MLA_ERR_INVALID_ARGUMENT, "cache too large");
+  if (c.d_latent != kLatent || c.d_rope != kRope)
+    return fail(MLA_ERR_UNSUPPORTED, "kernels are built for d_latent = 192 and d_rope = 32");
+  if (c.hidden % 128 != 0)
+    return fail(MLA_ERR_UNSUPPORTED, "hidden must be a multiple of 128");
+  if (c.batch > 65535 || (c.n_heads + 1) > 65535)
+    return fail(MLA_ERR_UNSUPPORTED, "batch and heads must fit a grid dimension");
+  return MLA_OK;
+}
+
+mla_status mla_ring_slot(const mla_config* cfg, int64_t frame, int32_t token, int64_t* slot) {
+  if (!cfg || !slot) return fail(MLA_ERR_INVALID_ARGUMENT, "NULL argument");
+  if (cfg->window_frames <= 0 || cfg->frame_h <= 0 || cfg->frame_w <= 0)
+    return fail(MLA_ERR_INVALID_ARGUMENT, "window and frame grid must be >= 1");
+  const int64_t F = (int64_t)cfg->frame_h * cfg->frame_w;
+  if (frame < 0 || token < 0 || token >= F)
+    return fail(MLA_ERR_INVALID_ARGUMENT, "frame must be >= 0 and token in [0, F)");
+  *slot = (frame % cfg->window_frames) * F + token;
+  return MLA_OK;
+}
+
+size_t mla_ring_bytes(const mla_config* cfg) {
+  if (!cfg || cfg->batch <= 0 || cfg->window_frames <= 0 || cfg->frame_h <= 0 ||
+      cfg->frame_w <= 0 || cfg->d_latent <= 0 || cfg->d_rope < 0)
+    return 0;
+  return (size_t)cfg->batch * cfg->window_frames * cfg->frame_h * cfg->frame_w *
+         (size_t)(cfg->d_latent + cfg->d_rope) * 2;
+}
+
+size_t mla_cache_device_bytes(const mla_config* cfg) {
+  if (mla_config_check(cfg) != MLA_OK) return 0;
+  const mla_config& c = *cfg;
+  const size_t F = (size_t)c.frame_h * c.frame_w;
+  const size_t rows = (size_t)(c.window_frames + c.max_chunk_frames) * F;
+  const size_t q = (size_t)c.max_chunk_frames * F;
+  size_t b = 0;
+  b += (size_t)c.batch * rows * kQK * 2;                   // ckv + krope (ring + chunk tail)
+  b += (size_t)c.batch * q * c.n_heads * kQK * 2;          // Qp
+  b += (size_t)c.batch * q * c.n_heads * kLatent * 2;      // o_lat
+  b += (size_t)(c.n_heads + 1) * kQK * c.hidden * 2;       // Wqcat
+  b += (size_t)c.hidden * c.n_heads * kLatent * 2;         // W_OV
+  b += 256;                                                // status word
+  return b;
+}
+
+void mla_cache_destroy(mla_cache* c) {
+  if (!c) return;
+  cudaDeviceSynchronize();
+  for (auto& r : c->pending) {
+    cudaEventDestroy(r.a);
+    cudaEventDestroy(r.b);
+  }
+  for (auto e : c->pool) cudaEventDestroy(e);
+  cudaFree(c->ckv);
+  cudaFree(c->krope);
+  cudaFree(c->qp);
+  cudaFree(c->o_lat);
+  cudaFree(c->wqcat);
+  cudaFree(c->wov);
+  cudaFree(c->status);
+  delete c;
+}
+
+mla_status mla_cache_create(const mla_config* cfg, const mla_weights* w, void* stream,
+                            mla_cache** out) {
+  if (!out) return fail(MLA_ERR_INVALID_ARGUMENT, "out is NULL");
+  *out = nullptr;
+  mla_status s = mla_config_check(cfg);
+  if (s != MLA_OK) return s;
+  if (!w || !w->w_q || !w->w_qr || !w->w_dkv || !w->w_kr || !w->w_uk || !w->w_uv || !w->w_o)
+    return fail(MLA_ERR_INVALID_ARGUMENT, "a weight pointer is NULL");
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+
+  mla_cache* c = new mla_cache();
+  c->cfg = *cfg;
+  c->F = cfg->frame_h * cfg->frame_w;
+  c->rows_per_stream = (int64_t)(cfg->window_frames + cfg->max_chunk_frames) * c->F;
+  c->max_q_tokens = (int64_t)cfg->max_chunk_frames * c->F;
+  c->softmax_scale = cfg->softmax_scale > 0.f
+                         ? cfg->softmax_scale
+                         : (float)(1.0 / std::sqrt((double)(cfg->d_nope + cfg->d_rope)));
+  c->rope = make_bands(*cfg);
+  c->out_bn = cfg->hidden % 256 == 0 ? 256 : 128;
+  cudaGetDevice(&c->device);
+
+  auto cleanup = [&](mla_status r) {
+    mla_cache_destroy(c);
+    return r;
+  };
+#define MLA_TRY(call)                                                                \
+  do {                                                                               \
+    cudaError_t e_ = (call);                                                         \
+    if (e_ != cudaSuccess)                                                           \
+      return cleanup(fail(e_ == cudaErrorMemoryAllocation ? MLA_ERR_OUT_OF_MEMORY : MLA_ERR_CUDA, \
+                          "%s failed: %s", #call, cudaGetErrorString(e_)));          \
+  } while (0)
+
+  const mla_config& k = *cfg;
+  const size_t ring_rows = (size_t)k.batch * c->rows_per_stream;
+  const size_t q_rows = (size_t)k.batch * c->max_q_tokens;
+  MLA_TRY(cudaMalloc(&c->ckv, ring_rows * kLatent * 2));
+  MLA_TRY(cudaMalloc(&c->krope, ring_rows * kRope * 2));
+  MLA_TRY(cudaMalloc(&c->qp, q_rows * k.n_heads * kQK * 2));
+  MLA_TRY(cudaMalloc(&c->o_lat, q_rows * k.n_heads * kLatent * 2));
+  MLA_TRY(cudaMalloc(&c->wqcat, (size_t)(k.n_heads + 1) * kQK * k.hidden * 2));
+  MLA_TRY(cudaMalloc(&c->wov, (size_t)k.hidden * k.n_heads * kLatent * 2));
+  MLA_TRY(cudaMalloc(&c->status, 256));
+  MLA_TRY(cudaMemsetAsync(c->ckv, 0, ring_rows * kLatent * 2, st));
+  MLA_TRY(cudaMemsetAsync(c->krope, 0, ring_rows * kRope * 2, st));
+  MLA_TRY(cudaMemsetAsync(c->qp, 0, q_rows * k.n_heads * kQK * 2, st));
+  MLA_TRY(cudaMemsetAsync(c->o_lat, 0, q_rows * k.n_heads * kLatent * 2, st));
+  MLA_TRY(cudaMemsetAsync(c->status, 0, 256, st));
+
+  {
+    dim3 g((k.hidden + 255) / 256, (k.n_heads + 1) * kQK);
+    build_wqcat_kernel<<<g, 256, 0, st>>>(
+        (const __nv_bfloat16*)w->w_q, (const __nv_bfloat16*)w->w_qr,
+        (const __nv_bfloat16*)w->w_dkv, (const __nv_bfloat16*)w->w_kr,
+        (const __nv_bfloat16*)w->w_uk, c->wqcat, k.hidden, k.n_heads, k.d_nope);
+    MLA_TRY(cudaGetLastError());
+    dim3 g2((k.n_heads * kLatent + 255) / 256, k.hidden);
+    build_wov_kernel<<<g2, 256, 0, st>>>((const __nv_bfloat16*)w->w_o,
+                                         (const __nv_bfloat16*)w->w_uv, c->wov, k.hidden,
+                                         k.n_heads, k.d_head);
+    MLA_TRY(cudaGetLastError());
+  }
+  s = make_map(&c->map_wqcat, c->wqcat, k.hidden, (uint64_t)(k.n_heads + 1) * kQK, 1,
+               (uint64_t)k.hidden * 2, (uint64_t)(k.n_heads + 1) * kQK * k.hidden * 2, 64, kQK,
+               CU_TENSOR_MAP_SWIZZLE_128B);
+  if (s != MLA_OK) return cleanup(s);
+  s = make_map(&c->map_wov, c->wov, (uint64_t)k.n_heads * kLatent, k.hidden, 1,
+               (uint64_t)k.n_heads * kLatent * 2, (uint64_t)k.hidden * k.n_heads * kLatent * 2,
+               64, c->out_bn, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (s != MLA_OK) return cleanup(s);
+
+  static std::once_flag attr_once;
+  static mla_status attr_status = MLA_OK;
+  std::call_once(attr_once, [] {
+    mla_status r = set_smem(mla::tc_gemm_kernel<kQK, kProjStages, mla::kEpiLatent>,
+                            mla::GemmSmem<kQK, kProjStages>::kBytes);
+    if (r == MLA_OK)
+      r = set_smem(mla::tc_gemm_kernel<256, kOutStages, mla::kEpiStore>,
+                   mla::GemmSmem<256, kOutStages>::kBytes);
+    if (r == MLA_OK)
+      r = set_smem(mla::tc_gemm_kernel<128, kOutStages, mla::kEpiStore>,
+                   mla::GemmSmem<128, kOutStages>::kBytes);
+    if (r == MLA_OK)
+      r = set_smem(mla::window_attn_kernel<kAttnStages, kAttnPInTmem>,
+                   mla::AttnSmem<kAttnStages, kAttnPInTmem>::kBytes);
+    attr_status = r;
+  });
+  if (attr_status != MLA_OK) return cleanup(attr_status);
+
+  MLA_TRY(cudaStreamSynchronize(st));
+#undef MLA_TRY
+  *out = c;
+  return MLA_OK;
+}
+
+mla_status mla_cache_append(mla_cache* c, const void* x, int32_t n_frames, void* stream) {
+  if (!c || !x) return fail(MLA_ERR_INVALID_ARGUMENT, "NULL argument");
+  if (n_frames < 1) return fail(MLA_ERR_INVALID_ARGUMENT, "n_frames must be >= 1");
+  if (!aligned16(x)) return fail(MLA_ERR_INVALID_ARGUMENT, "x must be 16-byte aligned");
+  if ((int64_t)n_frames * c->F > ((int64_t)1 << 30))
+    return fail(MLA_ERR_INVALID_ARGUMENT, "too many frames in one append");
+  const mla_config& cfg = c->cfg;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int skip = n_frames > cfg.window_frames ? n_frames - cfg.window_frames : 0;
+  const int64_t rows = (int64_t)(n_frames - skip) * c->F;
+  const void* x0 = static_cast<const __nv_bfloat16*>(x) + (int64_t)skip * c->F * cfg.hidden;
+  mla_status s;
+  {
+    ProfScope p(c, MLA_KERNEL_APPEND, st);
+    s = launch_latent_gemm(c, x0, rows, (int64_t)n_frames * c->F, 1, 0, cfg.n_heads * kQK, 1,
+                           c->frames_appended + skip, 0, st);
+  }
+  if (s != MLA_OK) return s;
+  c->frames_appended += n_frames;
+  return MLA_OK;
+}
+
+mla_status mla_window_attention(mla_cache* c, const void* x_chunk, int32_t n_frames, void* out,
+                                void* stream) {
+  if (!c || !x_chunk || !out) return fail(MLA_ERR_INVALID_ARGUMENT, "NULL argument");
+  const mla_config& cfg = c->cfg;
+  if (n_frames < 1 || n_frames > cfg.max_chunk_frames)
+    return fail(MLA_ERR_INVALID_ARGUMENT, "n_frames must be in [1, max_chunk_frames=%d]",
+                cfg.max_chunk_frames);
+  if (!aligned16(x_chunk) || !aligned16(out))
+    return fail(MLA_ERR_INVALID_ARGUMENT, "x_chunk and out must be 16-byte aligned");
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t nq = (int64_t)n_frames * c->F;
+  const int64_t valid = c->frames_appended < cfg.window_frames ? c->frames_appended
+                                                               : cfg.window_frames;
+  const int64_t base_row = valid * c->F;
+  const int64_t n_keys = base_row + nq;
+  mla_status s;
+
+  // 1. absorbed queries + chunk latents (one GEMM over [heads | latent] column blocks)
+  {
+    ProfScope p(c, MLA_KERNEL_QPROJ, st);
+    s = launch_latent_gemm(c, x_chunk, nq, nq, cfg.n_heads + 1, cfg.n_heads, 0, 0,
+                           c->frames_appended, base_row, st);
+  }
+  if (s != MLA_OK) return s;
+
+  // 2. window attention over [0, n_keys) of every stream
+  {
+    const int64_t R = nq * cfg.n_heads;
+    const uint64_t qp_rows = (uint64_t)c->max_q_tokens * cfg.n_heads;
+    CUtensorMap mqc, mqr, mkc, mkr;
+    if ((s = make_map(&mqc, c->qp, kQK, R, cfg.batch, kQK * 2, qp_rows * kQK * 2, 64, 128,
+                      CU_TENSOR_MAP_SWIZZLE_128B)) != MLA_OK)
+      return s;
+    if ((s = make_map(&mqr, c->qp, kQK, R, cfg.batch, kQK * 2, qp_rows * kQK * 2, 32, 128,
+                      CU_TENSOR_MAP_SWIZZLE_64B)) != MLA_OK)
+      return s;
+    if ((s = make_map(&mkc, c->ckv, kLatent, n_keys, cfg.batch, kLatent * 2,
+                      (uint64_t)c->rows_per_stream * kLatent * 2, 64, 128,
+                      CU_TENSOR_MAP_SWIZZLE_128B)) != MLA_OK)
+      return s;
+    if ((s = make_map(&mkr, c->krope, kRope, n_keys, cfg.batch, kRope * 2,
+                      (uint64_t)c->rows_per_stream * kRope * 2, 32, 128,
+                      CU_TENSOR_MAP_SWIZZLE_64B)) != MLA_OK)
+      return s;
+    mla::AttnArgs a{};
+    a.rows = (int32_t)R;
+    a.n_keys = (int32_t)n_keys;
+    a.o_lat = c->o_lat;
+    a.o_lat_batch_stride = (int64_t)c->max_q_tokens * cfg.n_heads * kLatent;
+    using Sm = mla::AttnSmem<kAttnStages, kAttnPInTmem>;
+    dim3 grid((unsigned)((R + 127) / 128), (unsigned)cfg.batch);
+    ProfScope p(c, MLA_KERNEL_ATTENTION, st);
+    mla::window_attn_kernel<kAttnStages, kAttnPInTmem>
+        <<<grid, mla::kAttnThreads, Sm::kBytes, st>>>(mqc, mqr, mkc, mkr, a, c->status);
+    if ((s = check_launch("window attention")) != MLA_OK) return s;
+  }
+
+  // 3. output projection out = o_lat W_OV^T
+  {
+    CUtensorMap ma;
+    const uint64_t kin = (uint64_t)cfg.n_heads * kLatent;
+    if ((s = make_map(&ma, c->o_lat, kin, nq, cfg.batch, kin * 2,
+                      (uint64_t)c->max_q_tokens * kin * 2, 64, 128,
+                      CU_TENSOR_MAP_SWIZZLE_128B)) != MLA_OK)
+      return s;
+    EpiArgs ep{};
+    ep.out = static_cast<__nv_bfloat16*>(out);
+    ep.out_batch_stride = nq * cfg.hidden;
+    ep.ld_out = cfg.hidden;
+    ProfScope p(c, MLA_KERNEL_OPROJ, st);
+    dim3 grid((unsigned)((nq + 127) / 128), (unsigned)(cfg.hidden / c->out_bn),
+              (unsigned)cfg.batch);
+    if (c->out_bn == 256) {
+      mla::tc_gemm_kernel<256, kOutStages, mla::kEpiStore>
+          <<<grid, mla::kGemmThreads, mla::GemmSmem<256, kOutStages>::kBytes, st>>>(
+              ma, c->map_wov, (int)nq, (int)kin, 0, ep, c->status);
+    } else {
+      mla::tc_gemm_kernel<128, kOutStages, mla::kEpiStore>
+          <<<grid, mla::kGemmThreads, mla::GemmSmem<128, kOutStages>::kBytes, st>>>(
+              ma, c->map_wov, (int)nq, (int)kin, 0, ep, c->status);
+    }
+    if ((s = check_launch("output projection")) != MLA_OK) return s;
+  }
+  return MLA_OK;
+}
+
+mla_status mla_cache_state(const mla_cache* c, int64_t* frames_appended, int32_t* valid) {
+  if (!c) return fail(MLA_ERR_INVALID_ARGUMENT, "NULL cache");
+  if (frames_appended) *frames_appended = c->frames_appended;
+  if (valid)
+    *valid = (int32_t)(c->frames_appended < c->cfg.window_frames ? c->frames_appended
+                                                                 : c->cfg.window_frames);
+  return MLA_OK;
+}
+
+mla_status mla_cache_sync(mla_cache* c, void* stream) {
+  if (!c) return fail(MLA_ERR_INVALID_ARGUMENT, "NULL cache");
+  MLA_CUDA(cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)));
+  int word = 0;
+  MLA_CUDA(cudaMemcpy(&word, c->status, sizeof(int), cudaMemcpyDeviceToHost));
+  if (word != 0) return fail((mla_status)word, "a kernel recorded device status %d", word);
+  return MLA_OK;
+}
+
+mla_status mla_cache_read(const mla_cache* c, int32_t b, void* ckv_host, void* krope_host,
+                          int64_t* n_valid_rows) {
+  if (!c) return fail(MLA_ERR_INVALID_ARGUMENT, "NULL cache");
+  if (b < 0 || b >= c->cfg.batch) return fail(MLA_ERR_INVALID_ARGUMENT, "stream index out of range");
+  const int64_t ring = (int64_t)c->cfg.window_frames * c->F;
+  if (ckv_host)
+    MLA_CUDA(cudaMemcpy(ckv_host, c->ckv + (int64_t)b * c->rows_per_stream * kLatent,
+                        ring * kLatent * 2, cudaMemcpyDeviceToHost));
+  if (krope_host)
+    MLA_CUDA(cudaMemcpy(krope_host, c->krope + (int64_t)b * c->rows_per_stream * kRope,
+                        ring * kRope * 2, cudaMemcpyDeviceToHost));
+  if (n_valid_rows) {
+    const int64_t v = c->frames_appended < c->cfg.window_frames ? c->frames_appended
+                                                                : c->cfg.window_frames;
+    *n_valid_rows = v * c->F;
+  }
+  return MLA_OK;
+}
+
+mla_status mla_cache_debug_buffers(const mla_cache* c, mla_debug_buffers* out) {
+  if (!c || !out) return fail(MLA_ERR_INVALID_ARGUMENT, "NULL argument");
+  out->ckv = c->ckv;
+  out->krope = c->krope;
+  out->qp = c->qp;
+  out->o_lat = c->o_lat;
+  out->w_qcat = c->wqcat;
+  out->w_ov = c->wov;
+  out->rows_per_stream = c->rows_per_stream;
+  return MLA_OK;
+}
+
+mla_status mla_cache_copy_buffer(const mla_cache* c, mla_buffer which, void* host_dst,
+                                 size_t bytes, size_t* size) {
+  if (!c) return fail(MLA_ERR_INVALID_ARGUMENT, "NULL cache");
+  const mla_config& k = c->cfg;
+  const size_t q_rows = (size_t)k.batch * c->max_q_tokens * k.n_heads;
+  const void* src = nullptr;
+  size_t total = 0;
+  switch (which) {
+    case MLA_BUFFER_QP: src = c->qp; total = q_rows * kQK * 2; break;
+    case MLA_BUFFER_O_LAT: src = c->o_lat; total = q_rows * kLatent * 2; break;
+    case MLA_BUFFER_W_QCAT: src = c->wqcat; total = (size_t)(k.n_heads + 1) * kQK * k.hidden * 2; break;
+    case MLA_BUFFER_W_OV: src = c->wov; total = (size_t)k.hidden * k.n_heads * kLatent * 2; break;
+    default: return fail(MLA_ERR_INVALID_ARGUMENT, "unknown buffer %d", (int)which);
+  }
+  if (size) *size = total;
+  if (host_dst && bytes)
+    MLA_CUDA(cudaMemcpy(host_dst, src, bytes < total ? bytes : total, cudaMemcpyDeviceToHost));
+  return MLA_OK;
+}
+
+mla_status mla_cache_profile_enable(mla_cache* c, int32_t enable) {
+  if (!c) return fail(MLA_ERR_INVALID_ARGUMENT, "NULL cache");
+  c->profiling = enable != 0;
+  return MLA_OK;
+}
+
+mla_status mla_cache_profile_read(mla_cache* c, mla_profile* out) {
+  if (!c || !out) return fail(MLA_ERR_INVALID_ARGUMENT, "NULL argument");
+  for (auto& r : c->pending) {
+    MLA_CUDA(cudaEventSynchronize(r.b));
+    float ms = 0.f;
+    MLA_CUDA(cudaEventElapsedTime(&ms, r.a, r.b));
+    c->prof_ms[r.kind] += ms;
+    c->prof_n[r.kind] += 1;
+    c->pool.push_back(r.a);
+    c->pool.push_back(r.b);
+  }
+  c->pending.clear();
+  for (int k = 0; k < MLA_KERNEL_COUNT; ++k) {
+    out->ms[k] = c->prof_ms[k];
+    out->launches[k] = c->prof_n[k];
+    c->prof_ms[k] = 0;
+    c->prof_n[k] = 0;
+  }
+  return MLA_OK;
+}
+
+}  // extern "C"

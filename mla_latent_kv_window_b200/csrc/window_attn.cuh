@@ -1,0 +1,328 @@
+// window_attn.cuh - latent-window attention on tcgen05 (sm_100a).
+//
+// Rows r = (query token, head) of the absorbed, rotated, pre-scaled queries Qp[r] (224 =
+// 192 latent + 32 RoPE channels) attend to every key j of the window plus the chunk:
+//
+//   s_j = Qp[r] . [c_kv_j | k_rope_j]          (log2-domain scores: Qp carries scale*log2 e)
+//   o_lat[r] = sum_j 2^(s_j - m) c_kv_j / sum_j 2^(s_j - m)
+//
+// This is the W_UK-absorbed form of the VideoMLA paper page's §3.3 attention: per-head keys
+// k_h = [c W_UK[h]^T | k_R] and values v_h = c W_UV[h]^T are never built; all heads read the
+// same head-shared latent tile, which makes the contraction an MQA-shaped dense GEMM.
+//
+// One CTA owns 128 rows.  Warp roles (192 threads):
+//   warp 0      TMA producer: the Q tile once, then 128-key tiles of c_kv (3 x 64-column
+//               128B-swizzled boxes) and k_rope (one 32-column 64B-swizzled box) into a
+//               KV_STAGES-deep ring.  Keys past n_keys are zero-filled by the tensor map.
+//   warp 1      TMEM allocator + single-thread MMA issuer:
+//                 S_j  = Q K_j^T     M=128 N=128 K=224 (14 k-steps; both operands K-major)
+//                 O   += P_j C_j     M=128 N=192 K=128 (8 k-steps; C_j is the SAME smem tile
+//                                    read MN-major, P_j from shared or tensor memory)
+//               S is double-buffered in TMEM so S_{j+1} runs while softmax works on S_j.
+//   warps 2..5  softmax: one row per thread, tcgen05.ld of its S row, running max with lazy
+//               rescaling (O is rescaled in TMEM only when the max grows by > 2^8), ex2,
+//               P_j as bf16 into shared memory (P_IN_TMEM = false) or tensor memory (true);
+//               finally O / l -> bf16 -> o_lat, staged for coalesced 384-byte row stores.
+//
+// TMEM columns: S0 [0,128), S1 [128,256), O [256,448), P [448,512) (P_IN_TMEM only).
+#pragma once
+
+#include "ptx.cuh"
+
+namespace mla {
+
+constexpr int kAttnThreads = 192;
+constexpr int kTileKeys = 128;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units: lazy O rescale when max grows > 2^8
+
+template <int KV_STAGES, bool P_IN_TMEM>
+struct AttnSmem {
+  static constexpr int kAtomC = 128 * 128;           // 128 rows x 64 bf16 (SW128)
+  static constexpr int kAtomR = 128 * 64;            // 128 rows x 32 bf16 (SW64)
+  static constexpr int kTileBytes = 3 * kAtomC + kAtomR;   // 57344: one Q or KV tile
+  static constexpr int kQ = 0;
+  static constexpr int kKV = kTileBytes;
+  static constexpr int kP = kKV + KV_STAGES * kTileBytes;
+  static constexpr int kPBytes = P_IN_TMEM ? 0 : 2 * kAtomC;
+  static constexpr int kBar = kP + kPBytes;
+  static constexpr int kBytes = kBar + 256 + 1024;
+  static_assert(kBytes <= 232448, "attention tile does not fit in shared memory");
+};
+
+struct AttnArgs {
+  int32_t rows;       // R = n_q * n_heads valid rows per stream
+  int32_t n_keys;     // keys per stream (window + chunk)
+  __nv_bfloat16* o_lat;
+  int64_t o_lat_batch_stride;  // elements
+};
+
+template <int KV_STAGES, bool P_IN_TMEM>
+__global__ void __launch_bounds__(kAttnThreads, 1)
+    window_attn_kernel(const __grid_constant__ CUtensorMap map_qc,
+                       const __grid_constant__ CUtensorMap map_qr,
+                       const __grid_constant__ CUtensorMap map_kc,
+                       const __grid_constant__ CUtensorMap map_kr, AttnArgs args, int* status) {
+  using L = AttnSmem<KV_STAGES, P_IN_TMEM>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
+  uint64_t* q_full = bars;
+  uint64_t* kv_full = bars + 1;                  // [KV_STAGES]
+  uint64_t* kv_empty = kv_full + KV_STAGES;      // [KV_STAGES]
+  uint64_t* s_full = kv_empty + KV_STAGES;       // [2]
+  uint64_t* s_free = s_full + 2;                 // [2]
+  uint64_t* p_full = s_free + 2;
+  uint64_t* pv_done = p_full + 1;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(pv_done + 1);
+
+  const uint32_t warp = warp_id();
+  const uint32_t lane = lane_id();
+  const int m0 = blockIdx.x * 128;
+  const int z = blockIdx.y;
+  const int n_keys = args.n_keys;
+  const int nt = (n_keys + kTileKeys - 1) / kTileKeys;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int s = 0; s < KV_STAGES; ++s) {
+      mbar_init(&kv_full[s], 1);
+      mbar_init(&kv_empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&s_full[s], 1);
+      mbar_init(&s_free[s], 128);
+    }
+    mbar_init(p_full, 128);
+    mbar_init(pv_done, 1);
+    fence_mbar_init();
+    tma_prefetch(&map_qc);
+    tma_prefetch(&map_qr);
+    tma_prefetch(&map_kc);
+    tma_prefetch(&map_kr);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  const uint32_t tmem_o = tmem + 256;
+  const uint32_t tmem_p = tmem + 448;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      const uint64_t keep = l2_policy_evict_last();    // keys are re-read by every row tile
+      const uint64_t once = l2_policy_evict_first();   // the Q tile is read once
+      uint8_t* q = smem + L::kQ;
+      mbar_arrive_expect_tx(q_full, L::kTileBytes);
+      for (int a = 0; a < 3; ++a)
+        tma_load_3d_hint(q + a * L::kAtomC, &map_qc, q_full, a * 64, m0, z, once);
+      tma_load_3d_hint(q + 3 * L::kAtomC, &map_qr, q_full, 192, m0, z, once);
+      int issued = 0;
+      for (int j = 0; j < nt; ++j) {
+        const int st = j % KV_STAGES;
+        const uint32_t round = j / KV_STAGES;
+        if (!mbar_wait(&kv_empty[st], (round & 1u) ^ 1u, status)) break;
+        uint8_t* kv = smem + L::kKV + st * L::kTileBytes;
+        mbar_arrive_expect_tx(&kv_full[st], L::kTileBytes);
+        for (int a = 0; a < 3; ++a)
+          tma_load_3d_hint(kv + a * L::kAtomC, &map_kc, &kv_full[st], a * 64, j * kTileKeys, z,
+                           keep);
+        tma_load_3d_hint(kv + 3 * L::kAtomC, &map_kr, &kv_full[st], 0, j * kTileKeys, z, keep);
+        issued = j + 1;
+      }
+      // Drain: never leave the CTA with a copy still landing in its shared memory.
+      for (int j = issued > KV_STAGES ? issued - KV_STAGES : 0; j < issued; ++j)
+        mbar_wait(&kv_full[j % KV_STAGES], (uint32_t)(j / KV_STAGES) & 1u, status);
+      mbar_wait(q_full, 0, status);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = idesc_bf16_f32(128, kTileKeys, false);
+      constexpr uint32_t idesc_o = idesc_bf16_f32(128, 192, true);
+      const uint32_t q_base = smem_u32(smem + L::kQ);
+      bool ok = mbar_wait(q_full, 0, status);
+      for (int j = 0; ok && j <= nt; ++j) {
+        if (j < nt) {
+          const int st = j % KV_STAGES;
+          const int sb = j & 1;
+          if (!mbar_wait(&kv_full[st], (uint32_t)(j / KV_STAGES) & 1u, status)) break;
+          if (j >= 2 && !mbar_wait(&s_free[sb], (uint32_t)((j >> 1) - 1) & 1u, status)) break;
+          tc_fence_after();
+          const uint32_t kv_base = smem_u32(smem + L::kKV + st * L::kTileBytes);
+#pragma unroll
+          for (int kk = 0; kk < 14; ++kk) {
+            uint64_t da, db;
+            if (kk < 12) {
+              const uint32_t off = (kk >> 2) * L::kAtomC + (kk & 3) * 32;
+              da = smem_desc(q_base + off, 16, 1024, kSwizzle128B);
+              db = smem_desc(kv_base + off, 16, 1024, kSwizzle128B);
+            } else {
+              const uint32_t off = 3 * L::kAtomC + (kk - 12) * 32;
+              da = smem_desc(q_base + off, 16, 512, kSwizzle64B);
+              db = smem_desc(kv_base + off, 16, 512, kSwizzle64B);
+            }
+            umma_ss(tmem + sb * kTileKeys, da, db, idesc_s, kk > 0 ? 1u : 0u);
+          }
+          tc_commit(&s_full[sb]);
+        }
+        if (j >= 1) {
+          const int jj = j - 1;
+          const int st = jj % KV_STAGES;
+          if (!mbar_wait(p_full, (uint32_t)jj & 1u, status)) break;
+          tc_fence_after();
+          const uint32_t c_base = smem_u32(smem + L::kKV + st * L::kTileBytes);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            // C_j read MN-major: 16 keys per step = two 8-row core groups of 1 KB; the three
+            // 64-column atoms are 16 KB apart (leading byte offset).
+            const uint64_t db = smem_desc(c_base + kk * 2048, L::kAtomC, 1024, kSwizzle128B);
+            const uint32_t acc = (jj > 0 || kk > 0) ? 1u : 0u;
+            if constexpr (P_IN_TMEM) {
+              umma_ts(tmem_o, tmem_p + kk * 8, db, idesc_o, acc);
+            } else {
+              const uint32_t p_base = smem_u32(smem + L::kP);
+              const uint64_t da = smem_desc(p_base + (kk >> 2) * L::kAtomC + (kk & 3) * 32, 16,
+                                            1024, kSwizzle128B);
+              umma_ss(tmem_o, da, db, idesc_o, acc);
+            }
+          }
+          tc_commit(pv_done);
+          tc_commit(&kv_empty[st]);
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------------ softmax warps
+    const uint32_t sub = warp & 3u;
+    const int row = sub * 32 + lane;
+    const uint32_t lane_off = (sub * 32u) << 16;
+    float m_used = -INFINITY;
+    float l_sum = 0.f;
+    bool ok = true;
+    for (int j = 0; j < nt; ++j) {
+      const int sb = j & 1;
+      if (!mbar_wait(&s_full[sb], (uint32_t)(j >> 1) & 1u, status)) { ok = false; break; }
+      tc_fence_after();
+      float s[kTileKeys];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        tmem_ld32(tmem + lane_off + sb * kTileKeys + c * 32, reinterpret_cast<uint32_t*>(s) + c * 32);
+      }
+      tmem_ld_wait();
+      tc_fence_before();
+      mbar_arrive(&s_free[sb]);
+
+      const int valid = n_keys - j * kTileKeys;   // keys of this tile that exist
+      if (valid < kTileKeys) {
+#pragma unroll
+        for (int i = 0; i < kTileKeys; ++i)
+          if (i >= valid) s[i] = -INFINITY;
+      }
+      float mx = s[0];
+#pragma unroll
+      for (int i = 1; i < kTileKeys; ++i) mx = fmaxf(mx, s[i]);
+      float alpha = 1.f;
+      bool rescale = false;
+      if (j == 0) {
+        m_used = mx;
+      } else if (mx > m_used + kRescaleThreshold) {
+        alpha = ex2_approx(m_used - mx);
+        m_used = mx;
+        rescale = true;
+        l_sum *= alpha;
+      }
+      float tile_sum = 0.f;
+      uint32_t pk[kTileKeys / 2];
+#pragma unroll
+      for (int i = 0; i < kTileKeys / 2; ++i) {
+        const float p0 = ex2_approx(s[2 * i] - m_used);
+        const float p1 = ex2_approx(s[2 * i + 1] - m_used);
+        pk[i] = pack_bf16x2(p0, p1);
+        tile_sum += p0 + p1;
+      }
+      l_sum += tile_sum;
+
+      // P buffer and O become free once PV_{j-1} has completed.
+      if (j >= 1 && !mbar_wait(pv_done, (uint32_t)(j - 1) & 1u, status)) { ok = false; break; }
+      tc_fence_after();
+      if (__any_sync(0xffffffffu, rescale)) {
+#pragma unroll 1
+        for (int c = 0; c < 6; ++c) {
+          uint32_t o[32];
+          tmem_ld32(tmem_o + lane_off + c * 32, o);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          tmem_st32(tmem_o + lane_off + c * 32, o);
+        }
+        tmem_st_wait();
+      }
+      if constexpr (P_IN_TMEM) {
+        tmem_st32(tmem_p + lane_off, pk);
+        tmem_st32(tmem_p + lane_off + 32, pk + 32);
+        tmem_st_wait();
+      } else {
+        uint8_t* p_row = smem + L::kP + row * 128;
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {   // 16-byte chunk c = keys 8c..8c+7
+          const int atom = c >> 3;
+          const int phys = (c & 7) ^ (row & 7);
+          *reinterpret_cast<uint4*>(p_row + atom * L::kAtomC + phys * 16) =
+              make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+        }
+        fence_proxy_async_smem();
+      }
+      tc_fence_before();
+      mbar_arrive(p_full);
+    }
+
+    // ---------------------------------------------------------------- epilogue: O / l
+    if (ok && mbar_wait(pv_done, (uint32_t)(nt - 1) & 1u, status)) {
+      tc_fence_after();
+      const float inv_l = 1.f / l_sum;
+      // Stage in the (now idle) first KV stage: 128 rows x (384 + 16) bytes.
+      constexpr int kStride = 400;
+      uint8_t* st_row = smem + L::kKV + row * kStride;
+#pragma unroll 1
+      for (int c = 0; c < 6; ++c) {
+        uint32_t o[32];
+        tmem_ld32(tmem_o + lane_off + c * 32, o);
+        tmem_ld_wait();
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          reinterpret_cast<uint4*>(st_row + c * 64)[q] = make_uint4(
+              pack_bf16x2(__uint_as_float(o[8 * q + 0]) * inv_l, __uint_as_float(o[8 * q + 1]) * inv_l),
+              pack_bf16x2(__uint_as_float(o[8 * q + 2]) * inv_l, __uint_as_float(o[8 * q + 3]) * inv_l),
+              pack_bf16x2(__uint_as_float(o[8 * q + 4]) * inv_l, __uint_as_float(o[8 * q + 5]) * inv_l),
+              pack_bf16x2(__uint_as_float(o[8 * q + 6]) * inv_l, __uint_as_float(o[8 * q + 7]) * inv_l));
+        }
+      }
+      __syncwarp();
+      __nv_bfloat16* out = args.o_lat + z * args.o_lat_batch_stride;
+      for (int rr = 0; rr < 32; ++rr) {
+        const int trow = sub * 32 + rr;
+        const int gr = m0 + trow;
+        if (gr >= args.rows) break;
+        if (lane < 24) {
+          reinterpret_cast<uint4*>(out + (int64_t)gr * 192)[lane] =
+              reinterpret_cast<const uint4*>(smem + L::kKV + trow * kStride)[lane];
+        }
+      }
+    }
+    tc_fence_before();
+  }
+
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace mla

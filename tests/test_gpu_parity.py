@@ -1,0 +1,236 @@
+"""GPU parity: the CUDA path through the C ABI against the fp64 oracle, on identical seeded inputs.
+
+Bar (bf16 inputs, fp32 accumulation): relative L2 error <= 1e-2 and max-abs error <= 3e-2 x RMS of
+the oracle output, for the layer output and the intermediates (ring contents, absorbed queries,
+latent-space attention output); ring slot placement exact.  Small cases compare every element;
+the full-size workloads compare seeded samples of query rows, which the oracle computes exactly.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import mla_synth
+from oracle import ring_slot, rope3d
+from tests.harness import Pair, assert_close, dims_of, errors
+
+pytestmark = pytest.mark.gpu
+
+LOG2E = 1.0 / math.log(2.0)
+
+
+def small(frame_h=4, frame_w=6, window=2, fill=2, q=1, batch=1, seed=0, scale=False):
+    return mla_synth.Workload("small", frame_h=frame_h, frame_w=frame_w, window_frames=window,
+                              fill_frames=fill, query_frames=q, batch=batch, seed=seed, stream_scale=scale)
+
+
+def check_ring(pair: Pair, what: str):
+    """Every valid frame f sits at slots (f mod W) F + k with the oracle's c_kv and k_rope."""
+    W, F = pair.w.window_frames, pair.F
+    for b, orc in enumerate(pair.oracles):
+        ckv, kr, n_valid = pair.gpu.read_ring(b)
+        contents = orc.cache_contents()
+        assert n_valid == len(contents) * F
+        for f, c, r in contents:
+            s0 = ring_slot(f, 0, W, F)
+            assert s0 == pair.gpu_slot(f, 0)
+            assert_close(ckv[s0:s0 + F], c, f"{what}: c_kv of frame {f} (stream {b})")
+            assert_close(kr[s0:s0 + F], r, f"{what}: k_rope of frame {f} (stream {b})")
+
+
+def oracle_qp(pair: Pair, x_chunk, b: int):
+    """Absorbed, rotated, pre-scaled queries in the GPU's row order (q, h), at absolute positions."""
+    orc = pair.oracles[b]
+    d = pair.dims
+    ctx = orc.keys_and_queries(x_chunk, positions="absolute")
+    rows = []
+    for h in range(d["n_heads"]):
+        dn, dr = d["d_nope"], d["d_rope"]
+        q_nope = ctx["x"] @ orc.W["w_q"][h * dn:(h + 1) * dn].T
+        q_abs = q_nope @ orc.W["w_uk"][h * dn:(h + 1) * dn]
+        q_rope = rope3d(ctx["x"] @ orc.W["w_qr"][h * dr:(h + 1) * dr].T, ctx["t_q"], ctx["h_q"], ctx["w_q"],
+                        d["rope_t"], d["rope_h"], d["rope_w"], d["rope_base"])
+        rows.append(np.concatenate([q_abs, q_rope], axis=1) * orc.scale * LOG2E)
+    return np.stack(rows, axis=1).reshape(-1, 224)
+
+
+def _slot(self, f, k):
+    from mla_latent_kv_window_b200 import mla_ring_slot
+    return mla_ring_slot(self.gpu.cfg, f, k)
+
+
+Pair.gpu_slot = _slot
+
+
+def full_check(pair: Pair, x_chunk, what: str, intermediates: bool = True):
+    out = pair.attention(x_chunk)
+    nq = x_chunk.shape[1]
+    for b, orc in enumerate(pair.oracles):
+        ref, parts = orc.attention(x_chunk[b], return_parts=True)
+        assert_close(out[b], ref, f"{what}: out (stream {b})")
+        if intermediates:
+            qp = pair.gpu.copy_buffer(0, (pair.w.batch, pair.gpu.cfg.max_chunk_frames * pair.F * 12, 224))
+            assert_close(qp[b, :nq * 12], oracle_qp(pair, x_chunk[b], b), f"{what}: Qp (stream {b})")
+            ol = pair.gpu.copy_buffer(1, (pair.w.batch, pair.gpu.cfg.max_chunk_frames * pair.F * 12, 192))
+            assert_close(ol[b, :nq * 12], parts["Pc"].reshape(-1, 192), f"{what}: o_lat (stream {b})")
+    pair.check_status()
+    return out
+
+
+# ---------------------------------------------------------------------------- small, every element
+def test_tiny_layer_full():
+    w = mla_synth.WORKLOADS["tiny"]
+    p = Pair(w)
+    p.append(p.hidden(w.fill_frames, mla_synth.fill_seed(w, 0)))
+    check_ring(p, "tiny")
+    full_check(p, p.hidden(w.query_frames, mla_synth.chunk_seed(w, 0, 0)), "tiny")
+
+
+def test_ring_wrap_and_bulk_append():
+    w = small(window=3, q=2, seed=11)
+    p = Pair(w, max_chunk_frames=2)
+    seed = 500
+    for n in (2, 2, 5, 1):          # wraps twice; the 5-frame append is larger than the window
+        p.append(p.hidden(n, seed))
+        seed += 1
+        check_ring(p, f"after append of {n}")
+    assert p.gpu.state() == (10, 3)
+    full_check(p, p.hidden(2, seed), "wrapped window, 2-frame chunk")
+
+
+def test_empty_window_attends_to_chunk_only():
+    w = small(window=3, q=1, seed=12)
+    p = Pair(w)
+    assert p.gpu.state() == (0, 0)
+    full_check(p, p.hidden(1, 900), "empty window")
+
+
+def test_partial_window():
+    w = small(window=3, q=2, seed=13)
+    p = Pair(w, max_chunk_frames=2)
+    p.append(p.hidden(1, 901))
+    full_check(p, p.hidden(2, 902), "one of three frames valid")
+    p.append(p.hidden(1, 903))
+    full_check(p, p.hidden(1, 904), "two of three frames valid")
+
+
+def test_multi_tile_ragged():
+    # F = 200: 1000 keys = 7 full 128-key tiles + 104; R = 400 tokens x 12 heads = 37.5 row tiles.
+    w = small(frame_h=10, frame_w=20, window=3, fill=4, q=2, seed=14)
+    p = Pair(w, max_chunk_frames=2)
+    p.append(p.hidden(4, 905))
+    check_ring(p, "ragged")
+    full_check(p, p.hidden(2, 906), "ragged multi-tile")
+
+
+def test_batched_streams_with_scales():
+    w = small(frame_h=6, frame_w=7, window=2, fill=3, q=1, batch=3, seed=15, scale=True)
+    p = Pair(w)
+    p.append(p.hidden(3, 907))
+    check_ring(p, "batched")
+    full_check(p, p.hidden(1, 908), "batched streams")
+
+
+def test_repeated_calls_same_cache():
+    # Several denoising steps over one window, then the chunk is appended (the rollout pattern).
+    w = small(window=2, q=1, seed=16)
+    p = Pair(w)
+    p.append(p.hidden(2, 909))
+    for s in range(3):
+        full_check(p, p.hidden(1, 910 + s), f"step {s}", intermediates=False)
+    x = p.hidden(1, 913)
+    full_check(p, x, "last step", intermediates=False)
+    p.append(x)
+    check_ring(p, "after chunk append")
+    full_check(p, p.hidden(1, 914), "next chunk")
+
+
+def test_invalid_calls_change_nothing():
+    from mla_latent_kv_window_b200 import MLAError
+    w = small(window=2, q=1, seed=17)
+    p = Pair(w)
+    p.append(p.hidden(2, 915))
+    with pytest.raises(MLAError):
+        p.gpu.attention(p.hidden(2, 916).cuda())          # 2 frames > max_chunk_frames = 1
+    with pytest.raises(ValueError):
+        p.gpu.attention(p.hidden(1, 917).cuda().float())  # wrong dtype, rejected in marshalling
+    assert p.gpu.state() == (2, 2)
+    full_check(p, p.hidden(1, 918), "after rejected calls", intermediates=False)
+
+
+# ---------------------------------------------------------------------------- full-size, sampled rows
+def sampled_check(pair: Pair, x_chunk, what: str, n_rows: int, seed: int):
+    out = pair.attention(x_chunk)
+    nq = x_chunk.shape[1]
+    rng = np.random.default_rng(seed)
+    worst = (0.0, 0.0)
+    for b, orc in enumerate(pair.oracles):
+        rows = np.sort(rng.choice(nq, size=min(n_rows, nq), replace=False))
+        ref = orc.attention(x_chunk[b], rows=rows)
+        rel, mx = assert_close(out[b][rows], ref, f"{what}: out rows (stream {b})")
+        worst = (max(worst[0], rel), max(worst[1], mx))
+        assert torch.isfinite(out[b].float()).all()
+    pair.check_status()
+    return worst
+
+
+def test_wan_w21_q1_full_size():
+    w = mla_synth.WORKLOADS["wan_w21_q1"]
+    p = Pair(w)
+    p.append(p.hidden(w.fill_frames, mla_synth.fill_seed(w, 0)))
+    # ring parity on a few frames (all 21 would be 32760 rows; sample 3)
+    ckv, kr, n = p.gpu.read_ring(0)
+    contents = p.oracles[0].cache_contents()
+    for f, c, r in (contents[0], contents[10], contents[-1]):
+        s0 = ring_slot(f, 0, w.window_frames, w.F)
+        assert_close(ckv[s0:s0 + w.F], c, f"c_kv frame {f}")
+        assert_close(kr[s0:s0 + w.F], r, f"k_rope frame {f}")
+    sampled_check(p, p.hidden(1, mla_synth.chunk_seed(w, 0, 0)), "21-frame window", 96, 1)
+
+
+def test_wan_b4_w21_q3_full_size():
+    w = mla_synth.WORKLOADS["wan_b4_w21_q3"]
+    p = Pair(w)
+    p.append(p.hidden(w.fill_frames, mla_synth.fill_seed(w, 0)))
+    sampled_check(p, p.hidden(3, mla_synth.chunk_seed(w, 0, 0)), "B=4 streams", 48, 3)
+
+
+def test_wan_w63_q1_full_size():
+    w = mla_synth.WORKLOADS["wan_w63_q1"]
+    p = Pair(w)
+    p.append(p.hidden(w.fill_frames, mla_synth.fill_seed(w, 0)))
+    sampled_check(p, p.hidden(1, mla_synth.chunk_seed(w, 0, 0)), "63-frame window", 48, 4)
+
+
+def test_wan_30_layers_4_steps_wrapped():
+    # 30 independent layers; each: append 24 frames (the ring wraps once, frames 3..23 stay), four
+    # denoising steps with a fresh 3-frame chunk over the same window, then the step-4 chunk is
+    # appended.  The oracle checks sampled rows of layers 0 and 29 (steps 0 and 3); every layer's
+    # output must be finite and its status word clean.
+    w = mla_synth.WORKLOADS["wan_30l_w21_q3_wrap"]
+    checked = {0: (0, 3), 29: (0, 3)}
+    for layer in range(w.layers):
+        p = Pair(w, layer=layer)
+        oracle_on = layer in checked
+        p.append(p.hidden(w.fill_frames, mla_synth.fill_seed(w, layer)), oracle=oracle_on)
+        assert p.gpu.state() == (24, 21)
+        x = None
+        for step in range(w.steps):
+            x = p.hidden(w.query_frames, mla_synth.chunk_seed(w, layer, step))
+            if oracle_on and step in checked[layer]:
+                sampled_check(p, x, f"layer {layer} step {step}", 32, 100 * layer + step)
+            else:
+                out = p.attention(x)
+                assert torch.isfinite(out.float()).all()
+        p.append(x, oracle=oracle_on)
+        assert p.gpu.state() == (27, 21)
+        if oracle_on:
+            ckv, kr, _ = p.gpu.read_ring(0)
+            f, c, r = p.oracles[0].cache_contents()[-1]
+            assert f == 26
+            s0 = ring_slot(f, 0, w.window_frames, w.F)
+            assert_close(ckv[s0:s0 + w.F], c, "appended chunk c_kv")
+            assert_close(kr[s0:s0 + w.F], r, "appended chunk k_rope")
+        p.check_status()
+        p.gpu.close()

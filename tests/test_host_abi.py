@@ -1,0 +1,93 @@
+"""Host side of the C ABI, without a GPU: the library loads, exports every symbol that
+include/mla.h declares, validates configurations, maps ring slots exactly like the oracle's
+definition, and reproduces the cache accounting printed on the VideoMLA paper page."""
+import ctypes
+import json
+import os
+import re
+
+import pytest
+
+import mla_synth
+from mla_latent_kv_window_b200 import binding as B
+from oracle import cache_scalars, dense_scalars_per_token, ring_slot
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def cfg(**over):
+    d = dict(mla_synth.DIMS_WAN13B)
+    kw = dict(frame_h=30, frame_w=52, window_frames=21, max_chunk_frames=3, batch=1)
+    kw.update({k: over.pop(k) for k in list(over) if k in kw})
+    d.update(over)
+    return B.make_config(d, **kw)
+
+
+def test_library_exports_every_declared_symbol():
+    lib = B.load_library()
+    header = open(os.path.join(ROOT, "include", "mla.h")).read()
+    declared = set(re.findall(r"^\s*(?:const\s+)?[\w\s\*]*?\b(mla_\w+)\s*\(", header, re.M))
+    assert {"mla_cache_create", "mla_cache_append", "mla_window_attention", "mla_cache_destroy"} <= declared
+    for name in sorted(declared):
+        assert hasattr(lib, name), f"{name} declared in include/mla.h but not exported"
+    assert set(B.EXPORTED) == declared
+
+
+def test_config_check():
+    assert B.mla_config_check(cfg()) == B.MLA_OK
+    bad = [
+        dict(rope_t=7, rope_h=13),                 # odd axis widths
+        dict(rope_t=10),                           # widths do not sum to d_rope
+        dict(window_frames=0), dict(max_chunk_frames=0), dict(batch=0), dict(frame_h=0),
+        dict(hidden=0), dict(n_heads=-1), dict(rope_base=-1.0),
+    ]
+    for over in bad:
+        assert B.mla_config_check(cfg(**over)) == B.MLA_ERR_INVALID_ARGUMENT, over
+    assert B.mla_config_check(cfg(d_latent=128)) == B.MLA_ERR_UNSUPPORTED
+    assert b"d_latent" in B.load_library().mla_last_error()
+    assert B.mla_config_check(cfg(hidden=1600)) == B.MLA_ERR_UNSUPPORTED
+    # the paper's default (6,5,5)-pair split is valid
+    assert B.mla_config_check(cfg(rope_t=12, rope_h=10, rope_w=10)) == B.MLA_OK
+
+
+def test_ring_slot_matches_oracle_exactly():
+    for W, fh, fw in ((21, 30, 52), (2, 4, 6), (63, 30, 52), (1, 1, 1), (5, 3, 7)):
+        c = cfg(window_frames=W, frame_h=fh, frame_w=fw)
+        F = fh * fw
+        for f in list(range(0, 3 * W + 2)) + [10**6 + 7, 2**40 + 3]:
+            for k in sorted({0, min(1, F - 1), F // 2, F - 1}):
+                assert B.mla_ring_slot(c, f, k) == ring_slot(f, k, W, F)
+    with pytest.raises(B.MLAError):
+        B.mla_ring_slot(cfg(), -1, 0)
+    with pytest.raises(B.MLAError):
+        B.mla_ring_slot(cfg(), 0, 1560)
+
+
+def test_ring_bytes_reproduce_printed_accounting():
+    g = json.load(open(os.path.join(ROOT, "tests", "golden", "accounting.json")))
+    d = g["dims"]
+    per_layer = B.mla_ring_bytes(cfg())
+    assert per_layer == 21 * 1560 * 224 * 2
+    dense_bytes = cache_scalars(d["layers"], d["window_frames"], d["tokens_per_frame"],
+                                dense_scalars_per_token(d["n_heads"], d["d_head"])) * 2
+    assert round(dense_bytes / 1e9, 1) == g["dense_cache_gb_bf16"]["value"]
+    assert round(dense_bytes / (d["layers"] * per_layer), 1) == g["reduction_factor"]["value"]
+    assert B.mla_ring_bytes(cfg(batch=4)) == 4 * per_layer
+    assert B.mla_cache_device_bytes(cfg()) > per_layer
+    assert B.mla_cache_device_bytes(cfg(d_latent=128)) == 0
+
+
+def test_calls_validate_before_any_device_work():
+    lib = B.load_library()
+    c = cfg()
+    out = ctypes.c_void_p(1234)
+    assert lib.mla_cache_create(ctypes.byref(c), None, None, ctypes.byref(out)) == B.MLA_ERR_INVALID_ARGUMENT
+    assert out.value is None
+    bad = cfg(window_frames=0)
+    w = B.mla_weights()
+    assert lib.mla_cache_create(ctypes.byref(bad), ctypes.byref(w), None, ctypes.byref(out)) == B.MLA_ERR_INVALID_ARGUMENT
+    assert lib.mla_cache_append(None, None, 1, None) == B.MLA_ERR_INVALID_ARGUMENT
+    assert lib.mla_window_attention(None, None, 1, None, None) == B.MLA_ERR_INVALID_ARGUMENT
+    assert lib.mla_cache_sync(None, None) == B.MLA_ERR_INVALID_ARGUMENT
+    lib.mla_cache_destroy(None)  # NULL-safe
+    assert lib.mla_status_string(5) == b"MLA_ERR_DEVICE_TIMEOUT"
