@@ -1,0 +1,469 @@
+#!/usr/bin/env python
+"""Benchmark of the VideoMLA latent-window attention hot path on B200.
+
+One step = one rollout step of one attention layer at the Wan-1.3B geometry (hidden 1536,
+12 heads, latent 192 + RoPE 32, 30 x 52 = 1560 tokens per latent frame, 21-frame window):
+the 1560-token query frame attends to the window plus itself through the C ABI
+(mla_window_attention: query projection, window attention, output projection), then the frame
+is appended to the window (mla_cache_append: fused down-projection + RoPE + ring write).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Multi-GPU: one process per GPU under torchrun; every rank runs its own independent replicas
+(no collective on the data path), the device time is the maximum over ranks and `value` is the
+query tokens of all ranks divided by it (weak scaling).  Prints one JSON line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "latent-window attention query tokens/s and TFLOP/s (% of bf16 peak) per layer"
+UNIT = "query tokens/s"
+WORKLOAD = "wan_w21_q1"
+FLOP_PER_QHK = 832          # 2*(192+32) for scores + 2*192 for P.c_kv, per (query, head, key)
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+L2_BYTES = 126 * 1024 * 1024
+
+
+def parse_args(argv=None):
+    p = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=1000)
+    p.add_argument("--warmup", type=int, default=20)
+    p.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    p.add_argument("--layers-cycle", type=int, default=12,
+                   help="independent layer caches cycled so the step's inputs are not L2-resident")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cpu-rows", type=int, default=1560, help="query tokens in the oracle's timed sample")
+    p.add_argument("--ncu-case", choices=("attention", "append", "steps"), default=None,
+                   help="minimal launch sequence for an ncu capture (prints no benchmark line): "
+                        "'attention' = fill + 2 steps, 'append' = 2 x 21-frame fill, 'steps' = warmup + K steps")
+    return p.parse_args(argv)
+
+
+def run_ncu_case(args, local):
+    """Short, fixed launch sequences for profiling under ncu (small device footprint)."""
+    import torch
+
+    import mla_synth
+    from mla_latent_kv_window_b200 import build
+    from mla_latent_kv_window_b200 import binding as B
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    build.build()
+    w = mla_synth.WORKLOADS[WORKLOAD]
+    dims = dict(w.dims)
+    F, W, hidden = w.F, w.window_frames, dims["hidden"]
+    nq = w.query_frames * F
+    n_layers = 1 if args.ncu_case != "steps" else 2
+    caches = []
+    for layer in range(n_layers):
+        wts = {k: v.to(dev) for k, v in mla_synth.make_weights(dims, mla_synth.weight_seed(w, layer)).items()}
+        caches.append(B.LatentWindowCache(dims, wts, w.frame_h, w.frame_w, W, w.query_frames))
+    x_fill = mla_synth.make_hidden(1, W * F, hidden, mla_synth.fill_seed(w, 0)).to(dev)
+    x = mla_synth.make_hidden(1, nq, hidden, mla_synth.chunk_seed(w, 0, 0)).to(dev)
+    out = torch.empty_like(x)
+    for c in caches:
+        c.append(x_fill)
+    if args.ncu_case == "append":
+        caches[0].append(x_fill)
+    else:
+        n = 2 if args.ncu_case == "attention" else args.warmup + args.steps
+        for s in range(n):
+            c = caches[s % n_layers]
+            c.attention(x, out)
+            c.append(x)
+    torch.cuda.synchronize()
+    ok = all(B.mla_cache_sync(c.handle) == 0 for c in caches)
+    print(json.dumps({"ncu_case": args.ncu_case, "device_status_ok": ok}))
+    return 0 if ok else 1
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(path))
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in ("ptx.cuh", "gemm_tc.cuh", "window_attn.cuh", "mla_api.cu"):
+        h.update(open(os.path.join(ROOT, "mla_latent_kv_window_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(kernel: str):
+    """DRAM bytes per launch from a committed ncu summary, if taken on the current kernel source."""
+    try:
+        d = json.load(open(os.path.join(ROOT, "profiles", "traffic.json")))
+        e = d[kernel]
+        if e.get("source_hash") == kernel_source_hash():
+            return float(e["bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples, kept only for the timed window."""
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.lines = []
+        self.t0 = self.t1 = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            threading.Thread(target=self._read, daemon=True).start()
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line.strip()))
+
+    def mark(self, which: str):
+        if which == "start":
+            self.t0 = time.time()
+        else:
+            self.t1 = time.time()
+
+    def stop(self) -> dict:
+        time.sleep(0.15)
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+        rows = []
+        for t, line in self.lines:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            rows.append((t, parts))
+        inside = [r for t, r in rows if self.t0 is not None and self.t0 - 0.05 <= t <= (self.t1 or t) + 0.05]
+        use = inside or [r for _, r in rows]
+        sm = [float(r[1]) for r in use if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in use if r[2].replace(".", "").isdigit()]
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        reasons = sorted({n for r in use for n, v in zip(names, r[5:9]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(use), "samples_in_timed_region": len(inside)}
+
+
+# ---------------------------------------------------------------------------- our arm
+def run_ours(args, rank, local, world):
+    import torch
+
+    import mla_synth
+    from mla_latent_kv_window_b200 import build, replicas
+    from mla_latent_kv_window_b200 import binding as B
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    distributed = replicas.init("nccl")
+    if rank == 0:
+        build.build()
+    replicas.barrier()
+    B.load_library()
+
+    w = mla_synth.WORKLOADS[WORKLOAD]
+    dims = dict(w.dims)
+    F, W = w.F, w.window_frames
+    hidden = dims["hidden"]
+    nq = w.query_frames * F
+    n_keys = W * F + nq
+    R = nq * dims["n_heads"]
+    L = args.layers_cycle
+    hbm_peak, tf_peak, peak_kind = peaks()
+
+    # Independent layer caches (distinct weights), each filled with a 21-frame window.
+    caches = []
+    for layer in range(L):
+        wts = {k: v.to(dev) for k, v in mla_synth.make_weights(dims, mla_synth.weight_seed(w, layer) + 1000 * rank).items()}
+        c = B.LatentWindowCache(dims, wts, w.frame_h, w.frame_w, W, w.query_frames)
+        x_fill = mla_synth.make_hidden(1, w.fill_frames * F, hidden, mla_synth.fill_seed(w, layer) + 1000 * rank).to(dev)
+        c.append(x_fill)
+        caches.append(c)
+        del x_fill
+    chunks = [mla_synth.make_hidden(1, nq, hidden, mla_synth.chunk_seed(w, 0, s) + 1000 * rank).to(dev) for s in range(4)]
+    out = torch.empty(1, nq, hidden, dtype=torch.bfloat16, device=dev)
+    torch.cuda.synchronize()
+    per_cache_bytes = B.mla_cache_device_bytes(caches[0].cfg)
+    stream = torch.cuda.current_stream()
+
+    def step(s):
+        c = caches[s % L]
+        x = chunks[s % 4]
+        B.mla_window_attention(c.handle, x, w.query_frames, out, stream)
+        B.mla_cache_append(c.handle, x, w.query_frames, stream)
+
+    # ---- append roofline: the 21-frame fill, L2 flushed before each launch
+    fill_cache = B.LatentWindowCache(dims, {k: v.to(dev) for k, v in mla_synth.make_weights(dims, 7).items()},
+                                     w.frame_h, w.frame_w, W, w.query_frames)
+    x_fill = mla_synth.make_hidden(1, W * F, hidden, 99).to(dev)
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+    B.mla_cache_profile_enable(fill_cache.handle, True)
+    for _ in range(3):
+        fill_cache.append(x_fill)
+    torch.cuda.synchronize()
+    B.mla_cache_profile_read(fill_cache.handle)
+    reps = 20
+    for _ in range(reps):
+        flush.fill_(1.0)
+        fill_cache.append(x_fill)
+    torch.cuda.synchronize()
+    ap = B.mla_cache_profile_read(fill_cache.handle)["append"]
+    append_ms = ap[0] / max(ap[1], 1)
+    append_bytes = W * F * (hidden * 2 + 224 * 2) + 224 * hidden * 2
+    fill_cache.close()
+    del flush, x_fill
+
+    # ---- main timed loop
+    for c in caches:
+        B.mla_cache_profile_enable(c.handle, True)
+    for s in range(args.warmup):
+        step(s)
+    torch.cuda.synchronize()
+    for c in caches:
+        B.mla_cache_profile_read(c.handle)
+    gpu_uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    clocks = ClockSampler(gpu_uuid if gpu_uuid.startswith("GPU-") else f"GPU-{gpu_uuid}")
+    clocks.start()
+    replicas.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks.mark("start")
+    e0.record(stream)
+    for s in range(args.steps):
+        step(args.warmup + s)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    clocks.mark("stop")
+    replicas.barrier()
+    clk = clocks.stop()
+    ms_local = e0.elapsed_time(e1)
+    ms = replicas.max_over_ranks(ms_local, dev)
+    prof = {k: [0.0, 0] for k in B.KERNEL_NAMES}
+    for c in caches:
+        for k, (t, n) in B.mla_cache_profile_read(c.handle).items():
+            prof[k][0] += t
+            prof[k][1] += n
+    launches = sum(n for _, n in prof.values())
+    attn_ms = prof["attention"][0] / max(prof["attention"][1], 1)
+    attn_ms = replicas.max_over_ranks(attn_ms, dev)
+
+    tokens = world * nq * args.steps
+    value = tokens / (ms / 1e3)
+    attn_flop = FLOP_PER_QHK * R * n_keys
+    attn_tflops = attn_flop / (attn_ms / 1e3) / 1e12
+    step_tflops = attn_flop * args.steps / (ms_local / 1e3) / 1e12
+
+    # ---- end to end through the public API with host buffers (pinned), copies inside the region
+    for c in caches:
+        B.mla_cache_profile_enable(c.handle, False)
+    x_host = [ch.cpu().pin_memory() for ch in chunks]
+    out_host = torch.empty(1, nq, hidden, dtype=torch.bfloat16).pin_memory()
+    x_dev = torch.empty(1, nq, hidden, dtype=torch.bfloat16, device=dev)
+    e2e_steps = max(1, min(args.steps, 400))
+
+    def e2e_step(s):
+        c = caches[s % L]
+        x_dev.copy_(x_host[s % 4], non_blocking=True)
+        B.mla_window_attention(c.handle, x_dev, w.query_frames, out, stream)
+        B.mla_cache_append(c.handle, x_dev, w.query_frames, stream)
+        out_host.copy_(out, non_blocking=True)
+
+    for s in range(min(args.warmup, 5)):
+        e2e_step(s)
+    torch.cuda.synchronize()
+    replicas.barrier()
+    e2 = torch.cuda.Event(enable_timing=True)
+    e3 = torch.cuda.Event(enable_timing=True)
+    e2.record(stream)
+    for s in range(e2e_steps):
+        e2e_step(s)
+    e3.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = replicas.max_over_ranks(e2.elapsed_time(e3), dev)
+    e2e_value = world * nq * e2e_steps / (e2e_ms / 1e3)
+
+    status_ok = all(B.mla_cache_sync(c.handle) == 0 for c in caches)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, args.cpu_rows)
+    replicas.barrier()
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 5),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic: seeded N(0,1) hidden states, N(0,1/fan_in) weights (no checkpoint)",
+            "config": {
+                "workload": f"{WORKLOAD}: Wan-1.3B-shaped layer, 21-frame latent window (32,760 cached tokens) "
+                            f"+ one 1,560-token query frame",
+                "hidden": hidden, "n_heads": dims["n_heads"], "d_latent": 192, "d_rope": 32, "d_nope": dims["d_nope"],
+                "tokens_per_frame": F, "window_frames": W, "query_tokens": nq, "keys": n_keys, "batch": 1,
+                "step": "mla_window_attention (Q-proj + latent-window attention + out-proj) then a 1-frame mla_cache_append",
+                "l2": f"inputs larger than L2: {L} independent layer caches cycled "
+                      f"({L * per_cache_bytes / 2**20:.0f} MB > 126 MB)",
+                "parallelism": f"replicas x{world} (no data-path collective)",
+            },
+            "attention_tflops": round(attn_tflops, 1),
+            "pct_bf16_peak": round(100 * attn_tflops / tf_peak, 1),
+            "step_attention_tflops": round(step_tflops, 1),
+            "kernel_ms_per_launch": {k: round(t / max(n, 1), 5) for k, (t, n) in prof.items()},
+            "roofline": {
+                "kernel": "window_attn_kernel", "bound": "tensor", "achieved": round(attn_tflops, 1),
+                "peak": tf_peak, "unit": "TFLOP/s", "frac": round(attn_tflops / tf_peak, 4),
+                "traffic": measured_traffic("window_attn_kernel"),
+                "peak_source": f"{peak_kind} bf16 (burst)",
+                "algorithmic": f"{FLOP_PER_QHK} flop per (query, head, key) x {R} rows x {n_keys} keys "
+                               f"= {attn_flop / 1e9:.1f} GFLOP per launch",
+            },
+            "append_roofline": {
+                "kernel": "tc_gemm_kernel<224,latent> (21-frame fill, L2 flushed)", "bound": "hbm",
+                "achieved": round(append_bytes / (append_ms / 1e3) / 1e9, 1), "peak": hbm_peak, "unit": "GB/s",
+                "frac": round(append_bytes / (append_ms / 1e3) / 1e9 / hbm_peak, 4),
+                "ms_per_launch": round(append_ms, 5), "traffic": measured_traffic("append_fill"),
+                "algorithmic": f"{W * F} tokens x (3072 B in + 448 B out) + 688,128 B weights = {append_bytes / 1e6:.1f} MB",
+                "peak_source": f"{peak_kind} HBM copy",
+            },
+            "e2e": {"value": round(e2e_value, 1), "unit": UNIT, "h2d_bytes_per_step": nq * hidden * 2,
+                    "d2h_bytes_per_step": nq * hidden * 2, "steps": e2e_steps},
+            "gpu_launches": int(launches),
+            "device_status_ok": status_ok,
+            "clocks": clk,
+        }
+        if cpu is not None:
+            line["cpu_baseline"] = cpu
+        print(json.dumps(line), flush=True)
+    for c in caches:
+        c.close()
+    replicas.shutdown()
+
+
+# ---------------------------------------------------------------------------- the oracle on CPU
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def _oracle_layer(w, rank=0):
+    import mla_synth
+    from oracle import OracleLayer
+    dims = dict(w.dims)
+    dims.update(frame_h=w.frame_h, frame_w=w.frame_w, window_frames=w.window_frames)
+    orc = OracleLayer(dims, mla_synth.make_weights(dict(w.dims), mla_synth.weight_seed(w, 0) + 1000 * rank))
+    orc.append(mla_synth.make_hidden(1, w.fill_frames * w.F, dims["hidden"], mla_synth.fill_seed(w, 0) + 1000 * rank)[0])
+    return orc
+
+
+def cpu_baseline(w, rows: int) -> dict:
+    """The fp64 oracle, as it stands, on a bounded sample of one step: `rows` query tokens, all
+    heads, all 34,320 keys (window filled beforehand, not timed)."""
+    import numpy as np
+
+    import mla_synth
+    orc = _oracle_layer(w)
+    x = mla_synth.make_hidden(1, w.query_frames * w.F, w.dim("hidden"), mla_synth.chunk_seed(w, 0, 0))[0]
+    sel = np.linspace(0, x.shape[0] - 1, rows).astype(np.int64)
+    t0 = time.perf_counter()
+    orc.attention(x, rows=sel)
+    dt = time.perf_counter() - t0
+    return {"value": round(rows / dt, 3), "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+            "seconds": round(dt, 2),
+            "sample": f"{rows} of {x.shape[0]} query tokens of one step (12 heads, {w.window_frames * w.F + x.shape[0]} keys, "
+                      f"float64 NumPy, per-head K/V materialised)"}
+
+
+def run_reference(args, rank, world):
+    """The oracle timed on the host cores as the reference arm (rank 0 only)."""
+    if rank != 0:
+        return
+    import numpy as np
+
+    import mla_synth
+    w = mla_synth.WORKLOADS[WORKLOAD]
+    orc = _oracle_layer(w)
+    nq = w.query_frames * w.F
+    chunks = [mla_synth.make_hidden(1, nq, w.dim("hidden"), mla_synth.chunk_seed(w, 0, s))[0] for s in range(4)]
+    rows_per_step = 8
+    heads = list(range(w.dim("n_heads")))
+    # One step: append the previous chunk (window slides by one frame) and attend a bounded sample of
+    # query rows of one head over the whole window + chunk.  Token-equivalents: rows * heads_used / 12.
+    def step(s):
+        x = chunks[s % 4]
+        sel = np.arange(s * 37, s * 37 + rows_per_step * 97, 97) % nq
+        orc.attention(x, rows=sel, heads=[heads[s % len(heads)]])
+        orc.append(x)
+
+    for s in range(args.warmup):
+        step(s)
+    t0 = time.perf_counter()
+    for s in range(args.steps):
+        step(args.warmup + s)
+    dt = time.perf_counter() - t0
+    tok = args.steps * rows_per_step / len(heads)
+    value = tok / dt
+    cores = blas_threads()
+    sample = (f"per step: 1-frame append + {rows_per_step} query rows x 1 of 12 heads over all "
+              f"{w.window_frames * w.F + nq} keys (float64 NumPy oracle); value counts rows*heads/12 token-equivalents")
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * dt / max(args.steps, 1), 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"{WORKLOAD}: Wan-1.3B-shaped layer, 21-frame latent window + one 1,560-token query frame"},
+        "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    from mla_latent_kv_window_b200.replicas import env_rank
+    rank, local, world = env_rank()
+    if args.gpus != world and world > 1:
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE {world}", file=sys.stderr)
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+    if args.ncu_case:
+        return run_ncu_case(args, local)
+    return run_ours(args, rank, local, world)
+
+
+if __name__ == "__main__":
+    sys.exit(main() or 0)

@@ -12,6 +12,12 @@
  * W_UK-absorbed scores q_c . c_kv + q_rope . k_rope, an online softmax, P . c_kv, and the
  * W_UV / W_O up-projections folded into one output projection.
  *
+ * Precision: the caller's hidden states, weights and outputs are bf16.  The cached latent
+ * (c_kv, k_rope), the absorbed queries, the softmax weights P, the latent-space output and the
+ * folded output weight are 16-bit fp16 internally (the paper sizes the cache as bf16/fp16; fp16
+ * keeps three more mantissa bits for the same 448 bytes per token), saturating at +-65504; every
+ * product accumulates in fp32.
+ *
  * Conventions shared by every call:
  *  - Tensors are bf16, row-major, 16-byte aligned device pointers unless stated otherwise.
  *  - Weights follow the nn.Linear layout [out_features, in_features] with head-major output
@@ -131,21 +137,21 @@ mla_status mla_cache_state(const mla_cache* c, int64_t* frames_appended, int32_t
 mla_status mla_cache_sync(mla_cache* c, void* stream);
 
 /* Copy stream b's ring planes to host memory, in physical slot order: ckv_host receives
- * W*F rows of d_latent bf16, krope_host W*F rows of d_rope bf16 (either may be NULL);
+ * W*F rows of d_latent fp16, krope_host W*F rows of d_rope fp16 (either may be NULL);
  * *n_valid_rows = valid_frames * F.  Synchronous; diagnostic, not on the hot path. */
 mla_status mla_cache_read(const mla_cache* c, int32_t b, void* ckv_host, void* krope_host,
                           int64_t* n_valid_rows);
 
 /* Device pointers of the cache's internal planes, for diagnostics and tests. */
 typedef struct {
-  void* ckv;          /* [batch][rows_per_stream][d_latent]; rows = (W + max_chunk)*F        */
-  void* krope;        /* [batch][rows_per_stream][d_rope]                                    */
-  void* qp;           /* [batch][max_chunk*F*n_heads][d_latent + d_rope]: absorbed, rotated,
-                         pre-scaled queries of the last attention call                      */
-  void* o_lat;        /* [batch][max_chunk*F][n_heads*d_latent]: normalised P . c_kv          */
-  void* w_qcat;       /* [(n_heads+1)*(d_latent+d_rope)][hidden]: per head W_Qabs|W_QR, then
-                         W_DKV|W_KR                                                          */
-  void* w_ov;         /* [hidden][n_heads*d_latent]                                          */
+  void* ckv;          /* fp16 [batch][rows_per_stream][d_latent]; rows = (W + max_chunk)*F   */
+  void* krope;        /* fp16 [batch][rows_per_stream][d_rope]                               */
+  void* qp;           /* fp16 [batch][max_chunk*F*n_heads][d_latent + d_rope]: absorbed,
+                         rotated queries of the last attention call, times scale * log2(e)   */
+  void* o_lat;        /* fp16 [batch][max_chunk*F][n_heads*d_latent]: normalised P . c_kv     */
+  void* w_qcat;       /* bf16 [(n_heads+1)*(d_latent+d_rope)][hidden]: per head W_Qabs|W_QR,
+                         then W_DKV|W_KR                                                     */
+  void* w_ov;         /* fp16 [hidden][n_heads*d_latent]                                     */
   int64_t rows_per_stream;
 } mla_debug_buffers;
 mla_status mla_cache_debug_buffers(const mla_cache* c, mla_debug_buffers* out);
@@ -153,10 +159,10 @@ mla_status mla_cache_debug_buffers(const mla_cache* c, mla_debug_buffers* out);
 /* Synchronous copy of the first min(bytes, size) bytes of an internal buffer to host memory;
  * *size receives the buffer's full size in bytes (may be NULL).  Diagnostic only. */
 typedef enum {
-  MLA_BUFFER_QP = 0,     /* Qp of the last attention call    */
-  MLA_BUFFER_O_LAT = 1,  /* o_lat of the last attention call */
-  MLA_BUFFER_W_QCAT = 2, /* absorbed query + latent weights  */
-  MLA_BUFFER_W_OV = 3    /* absorbed output weights          */
+  MLA_BUFFER_QP = 0,     /* Qp of the last attention call (fp16)   */
+  MLA_BUFFER_O_LAT = 1,  /* o_lat of the last attention call (fp16) */
+  MLA_BUFFER_W_QCAT = 2, /* absorbed query + latent weights (bf16)  */
+  MLA_BUFFER_W_OV = 3    /* absorbed output weights (fp16)          */
 } mla_buffer;
 mla_status mla_cache_copy_buffer(const mla_cache* c, mla_buffer which, void* host_dst, size_t bytes,
                                  size_t* size);

@@ -253,18 +253,19 @@ class LatentWindowCache:
         _check(mla_cache_sync(self.handle, stream), "mla_cache_sync")
 
     def read_ring(self, b: int = 0):
-        """(ckv [W*F, 192], krope [W*F, 32]) of stream b in physical slot order, and the valid row count."""
+        """(ckv [W*F, 192], krope [W*F, 32]) fp16 of stream b in physical slot order, and the valid row count."""
         import torch
         W = self.cfg.window_frames
-        ckv = torch.empty(W * self.F, self.cfg.d_latent, dtype=torch.bfloat16)
-        kr = torch.empty(W * self.F, self.cfg.d_rope, dtype=torch.bfloat16)
+        ckv = torch.empty(W * self.F, self.cfg.d_latent, dtype=torch.float16)
+        kr = torch.empty(W * self.F, self.cfg.d_rope, dtype=torch.float16)
         n = mla_cache_read(self.handle, b, ckv, kr)
         return ckv, kr, n
 
     def copy_buffer(self, which: int, shape):
-        """Host copy (bf16 tensor of `shape`) of an internal buffer: MLA_BUFFER_QP, _O_LAT, _W_QCAT, _W_OV."""
+        """Host copy (tensor of `shape`) of an internal buffer: MLA_BUFFER_QP, _O_LAT, _W_OV (fp16)
+        or MLA_BUFFER_W_QCAT (bf16)."""
         import torch
-        out = torch.empty(shape, dtype=torch.bfloat16)
+        out = torch.empty(shape, dtype=torch.bfloat16 if which == MLA_BUFFER_W_QCAT else torch.float16)
         mla_cache_copy_buffer(self.handle, which, out)
         return out
 

@@ -1,18 +1,26 @@
 // gemm_tc.cuh - tcgen05 GEMM for the projections of the latent-window attention path.
 //
-//   D[m, n] = sum_k A[z][m, k] * B[n, k]          (A: [batch][M][K], B: [N][K], both K-major bf16)
+//   D[m, n] = sum_k A[z][m, k] * B[n, k]    (A: [batch][M][K], B: [N][K], K-major, both bf16 or
+//                                            both fp16, fp32 accumulation)
 //
 // One CTA computes a 128 x BN tile with fp32 accumulation in tensor memory:
-//   warp 0      TMA producer: A and B k-blocks of 64 into a STAGES-deep shared-memory ring
+//   warp 0      TMA producer of A k-blocks (64 wide) into an A_STAGES-deep ring
+//   warp 6      TMA producer of B k-blocks into a B_STAGES-deep ring
 //   warp 1      TMEM allocator + single-thread tcgen05.mma issuer (M=128, N=BN, K=16 steps)
 //   warps 2..5  epilogue: tcgen05.ld of the accumulator (one row per thread), fused row
 //               transform, staged through shared memory for coalesced 16-byte row stores.
+// A (hidden states, streamed once from HBM) and B (weights, shared by every CTA and
+// L2-resident) have separate rings so that A can run far ahead of the short-latency B loads;
+// each CTA starts its k-loop at a rotated block so the CTAs do not all hit the same weight
+// block at once.
 //
 // Epilogues (kEpi):
 //   kEpiStore   bf16 store of the tile into out[z][m][n]                (output projection)
-//   kEpiLatent  columns 0..191 -> c_kv, 192..223 -> RoPE3D -> k_rope, written to ring slots
-//               (t mod W)*F + k, or to the chunk tail; for blockIdx.y below latent_y the tile is
-//               one head's absorbed query [W_UK^T q_nope | RoPE3D(q_rope)] * scale -> Qp.
+//   kEpiLatent  columns 0..191 -> c_kv, 192..223 -> RoPE3D -> k_rope, written as fp16 to ring
+//               slots (t mod W)*F + k, or to the chunk tail; for blockIdx.y below latent_y the
+//               tile is one head's absorbed query [W_UK^T q_nope | RoPE3D(q_rope)] * scale ->
+//               Qp (fp16).  The latent path is 16-bit like the paper's cache; fp16 keeps three
+//               more mantissa bits than bf16 for the same bytes.
 //
 // The latent epilogue is the fused "append" of the VideoMLA paper page: c_kv = x W_DKV^T and
 // the decoupled positional key k_R = RoPE3D(x W_KR^T) (§3.1, §3.2), one head-shared copy per
@@ -25,7 +33,7 @@ namespace mla {
 
 constexpr int kEpiStore = 0;
 constexpr int kEpiLatent = 1;
-constexpr int kGemmThreads = 192;
+constexpr int kGemmThreads = 224;
 
 // Rotary bands of the d_rope = 32 positional channels: pair p rotates by pos[axis[p]] * freq[p].
 struct RopeBands {
@@ -39,10 +47,10 @@ struct EpiArgs {
   int64_t out_batch_stride;  // elements
   int32_t ld_out;            // elements per output row
   // kEpiLatent
-  __nv_bfloat16* ckv;        // [batch][rows_per_stream][192]
-  __nv_bfloat16* krope;      // [batch][rows_per_stream][32]
+  __half* ckv;               // [batch][rows_per_stream][192] fp16
+  __half* krope;             // [batch][rows_per_stream][32]  fp16
   int64_t rows_per_stream;
-  __nv_bfloat16* qp;         // [batch][qp_rows_per_stream][224]
+  __half* qp;                // [batch][qp_rows_per_stream][224] fp16
   int64_t qp_rows_per_stream;
   int32_t latent_y;          // blockIdx.y >= latent_y -> latent tile, else query head blockIdx.y
   int32_t n_heads;
@@ -56,15 +64,16 @@ struct EpiArgs {
   RopeBands rope;
 };
 
-template <int BN, int STAGES>
+template <int BN, int A_STAGES, int B_STAGES>
 struct GemmSmem {
   static constexpr int kABytes = 128 * 64 * 2;
   static constexpr int kBBytes = BN * 64 * 2;
-  static constexpr int kStageBytes = kABytes + kBBytes;
-  static constexpr int kBarOffset = STAGES * kStageBytes;
-  static constexpr int kBytes = kBarOffset + 256 + 1024;  // barriers + alignment slack
+  static constexpr int kBOffset = A_STAGES * kABytes;
+  static constexpr int kBarOffset = kBOffset + B_STAGES * kBBytes;
+  static constexpr int kBytes = kBarOffset + 512 + 1024;  // barriers + alignment slack
   static_assert(kABytes % 1024 == 0 && kBBytes % 1024 == 0, "stage atoms must stay 1 KB aligned");
-  static_assert(STAGES * kStageBytes >= 128 * (BN * 2 + 16), "staging must fit in the ring");
+  static_assert(kBarOffset >= 128 * (BN * 2 + 16), "staging must fit in the rings");
+  static_assert(kBytes <= 232448, "GEMM tile does not fit in shared memory");
 };
 
 __device__ __forceinline__ void rope_rotate32(float* v, int64_t t, int h, int w,
@@ -83,19 +92,21 @@ __device__ __forceinline__ void rope_rotate32(float* v, int64_t t, int h, int w,
   }
 }
 
-template <int BN, int STAGES, int kEpi>
+template <int BN, int A_STAGES, int B_STAGES, int kEpi, bool kF16In>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
                    const __grid_constant__ CUtensorMap map_b, int32_t M, int32_t K,
                    int32_t b_row0, EpiArgs ep, int* status) {
-  using L = GemmSmem<BN, STAGES>;
+  using L = GemmSmem<BN, A_STAGES, B_STAGES>;
   static_assert(kEpi != kEpiLatent || BN == 224, "the latent epilogue owns 192 + 32 columns");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kBarOffset);
-  uint64_t* empty = full + STAGES;
-  uint64_t* acc_full = empty + STAGES;
+  uint64_t* a_full = reinterpret_cast<uint64_t*>(smem + L::kBarOffset);
+  uint64_t* a_empty = a_full + A_STAGES;
+  uint64_t* b_full = a_empty + A_STAGES;
+  uint64_t* b_empty = b_full + B_STAGES;
+  uint64_t* acc_full = b_empty + B_STAGES;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(acc_full + 1);
 
   const uint32_t warp = warp_id();
@@ -104,12 +115,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const int y = blockIdx.y;
   const int z = blockIdx.z;
   const int num_kb = K / 64;
+  const int kb_rot = (int)((blockIdx.x * 7u + blockIdx.y * 3u + blockIdx.z) % (unsigned)num_kb);
   constexpr uint32_t kTmemCols = BN <= 128 ? 128 : 256;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
+    for (int s = 0; s < A_STAGES; ++s) {
+      mbar_init(&a_full[s], 1);
+      mbar_init(&a_empty[s], 1);
+    }
+    for (int s = 0; s < B_STAGES; ++s) {
+      mbar_init(&b_full[s], 1);
+      mbar_init(&b_empty[s], 1);
     }
     mbar_init(acc_full, 1);
     fence_mbar_init();
@@ -125,38 +141,51 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
 
-  if (warp == 0) {
+  if (warp == 0 || warp == 6) {
+    // ------------------------------------------------------------------ TMA producers
     if (lane == 0) {
+      const bool is_a = warp == 0;
+      const int stages = is_a ? A_STAGES : B_STAGES;
+      uint64_t* full = is_a ? a_full : b_full;
+      uint64_t* empty = is_a ? a_empty : b_empty;
+      const uint32_t bytes = is_a ? L::kABytes : L::kBBytes;
+      const uint64_t policy = is_a ? l2_policy_evict_first() : l2_policy_evict_last();
+      int issued = 0;
       for (int kb = 0; kb < num_kb; ++kb) {
-        const int s = kb % STAGES;
-        const uint32_t round = kb / STAGES;
-        if (!mbar_wait(&empty[s], (round & 1u) ^ 1u, status)) break;
-        uint8_t* sa = smem + s * L::kStageBytes;
-        mbar_arrive_expect_tx(&full[s], L::kStageBytes);
-        tma_load_3d(sa, &map_a, &full[s], kb * 64, m0, z);
-        tma_load_3d(sa + L::kABytes, &map_b, &full[s], kb * 64, b_row0 + y * BN, 0);
+        const int s = kb % stages;
+        if (!mbar_wait(&empty[s], ((uint32_t)(kb / stages) & 1u) ^ 1u, status)) break;
+        const int kx = ((kb + kb_rot) % num_kb) * 64;
+        mbar_arrive_expect_tx(&full[s], bytes);
+        if (is_a)
+          tma_load_3d_hint(smem + s * L::kABytes, &map_a, &full[s], kx, m0, z, policy);
+        else
+          tma_load_3d_hint(smem + L::kBOffset + s * L::kBBytes, &map_b, &full[s], kx,
+                           b_row0 + y * BN, 0, policy);
+        issued = kb + 1;
       }
+      // Drain: never leave the CTA with a copy still landing in its shared memory.
+      for (int kb = issued > stages ? issued - stages : 0; kb < issued; ++kb)
+        mbar_wait(&full[kb % stages], (uint32_t)(kb / stages) & 1u, status);
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(128, BN, false);
-      bool ok = true;
-      for (int kb = 0; kb < num_kb && ok; ++kb) {
-        const int s = kb % STAGES;
-        if (!mbar_wait(&full[s], (uint32_t)(kb / STAGES) & 1u, status)) {
-          ok = false;
-          break;
-        }
+      constexpr uint32_t idesc = idesc_f32acc(128, BN, false, kF16In);
+      for (int kb = 0; kb < num_kb; ++kb) {
+        const int sa = kb % A_STAGES;
+        const int sb = kb % B_STAGES;
+        if (!mbar_wait(&a_full[sa], (uint32_t)(kb / A_STAGES) & 1u, status)) break;
+        if (!mbar_wait(&b_full[sb], (uint32_t)(kb / B_STAGES) & 1u, status)) break;
         tc_fence_after();
-        const uint32_t sa = smem_u32(smem + s * L::kStageBytes);
-        const uint32_t sb = sa + L::kABytes;
+        const uint32_t a_addr = smem_u32(smem + sa * L::kABytes);
+        const uint32_t b_addr = smem_u32(smem + L::kBOffset + sb * L::kBBytes);
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-          const uint64_t da = smem_desc(sa + k * 32, 16, 1024, kSwizzle128B);
-          const uint64_t db = smem_desc(sb + k * 32, 16, 1024, kSwizzle128B);
+          const uint64_t da = smem_desc(a_addr + k * 32, 16, 1024, kSwizzle128B);
+          const uint64_t db = smem_desc(b_addr + k * 32, 16, 1024, kSwizzle128B);
           umma_ss(tmem, da, db, idesc, (kb | k) != 0 ? 1u : 0u);
         }
-        tc_commit(&empty[s]);
+        tc_commit(&a_empty[sa]);
+        tc_commit(&b_empty[sb]);
       }
       tc_commit(acc_full);
     }
@@ -202,10 +231,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         uint4* dst = reinterpret_cast<uint4*>(stage_row + c * 64);
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          dst[q] = make_uint4(pack_bf16x2(v[8 * q + 0], v[8 * q + 1]),
-                              pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
-                              pack_bf16x2(v[8 * q + 4], v[8 * q + 5]),
-                              pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
+          if constexpr (kEpi == kEpiLatent) {
+            dst[q] = make_uint4(pack_f16x2(v[8 * q + 0], v[8 * q + 1]),
+                                pack_f16x2(v[8 * q + 2], v[8 * q + 3]),
+                                pack_f16x2(v[8 * q + 4], v[8 * q + 5]),
+                                pack_f16x2(v[8 * q + 6], v[8 * q + 7]));
+          } else {
+            dst[q] = make_uint4(pack_bf16x2(v[8 * q + 0], v[8 * q + 1]),
+                                pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
+                                pack_bf16x2(v[8 * q + 4], v[8 * q + 5]),
+                                pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
+          }
         }
       }
     }

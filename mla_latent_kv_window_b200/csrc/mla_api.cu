@@ -32,9 +32,11 @@ constexpr int kLatent = 192;
 constexpr int kRope = 32;
 constexpr int kQK = kLatent + kRope;  // 224
 
-// Pipeline depths of the launched kernel variants.
-constexpr int kProjStages = 4;      // 4 x 44 KB: one CTA per SM, deep enough for HBM latency
-constexpr int kOutStages = 4;
+// Pipeline depths of the launched kernel variants (A = activations, B = weights).
+constexpr int kProjAStages = 8;     // 8 x 16 KB of hidden states in flight per SM (HBM latency)
+constexpr int kProjBStages = 3;     // 3 x 28 KB of L2-resident weights
+constexpr int kOutAStages = 6;
+constexpr int kOutBStages = 3;
 constexpr int kAttnStages = 3;      // 3 KV tiles in flight (P kept in tensor memory)
 constexpr bool kAttnPInTmem = true;
 
@@ -80,17 +82,19 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 3-D bf16 map: (inner, rows, batch) with byte strides; box (box_inner, box_rows, 1).
+// 3-D 16-bit map (bf16, or fp16 when f16): (inner, rows, batch) with byte strides; box
+// (box_inner, box_rows, 1).
 mla_status make_map(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows,
                     uint64_t batch, uint64_t row_bytes, uint64_t batch_bytes, uint32_t box_inner,
-                    uint32_t box_rows, CUtensorMapSwizzle swz) {
+                    uint32_t box_rows, CUtensorMapSwizzle swz, bool f16 = false) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return fail(MLA_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
   cuuint64_t dims[3] = {inner, rows, batch};
   cuuint64_t strides[2] = {row_bytes, batch_bytes};
   cuuint32_t box[3] = {box_inner, box_rows, 1};
   cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+  CUresult r = enc(map, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                   const_cast<void*>(base), dims,
                    strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS)
@@ -134,10 +138,11 @@ __global__ void build_wqcat_kernel(const __nv_bfloat16* __restrict__ w_q,
   wqcat[(size_t)rowq * hidden + k] = __float2bfloat16_rn(acc);
 }
 
-// W_OV[o][h*192 + c] = sum_j W_O[o][h*d_head + j] * W_UV[h*d_head + j][c].
+// W_OV[o][h*192 + c] = sum_j W_O[o][h*d_head + j] * W_UV[h*d_head + j][c], stored fp16 (it
+// multiplies the fp16 o_lat).
 __global__ void build_wov_kernel(const __nv_bfloat16* __restrict__ w_o,
                                  const __nv_bfloat16* __restrict__ w_uv,
-                                 __nv_bfloat16* __restrict__ wov, int hidden, int n_heads,
+                                 __half* __restrict__ wov, int hidden, int n_heads,
                                  int d_head) {
   const int col = blockIdx.x * blockDim.x + threadIdx.x;  // h*192 + c
   const int o = blockIdx.y;
@@ -151,7 +156,7 @@ __global__ void build_wov_kernel(const __nv_bfloat16* __restrict__ w_o,
     acc += __bfloat162float(w_o[(size_t)o * in_o + r]) *
            __bfloat162float(w_uv[(size_t)r * kLatent + c]);
   }
-  wov[(size_t)o * (n_heads * kLatent) + col] = __float2bfloat16_rn(acc);
+  wov[(size_t)o * (n_heads * kLatent) + col] = __float2half_rn(acc);
 }
 
 template <typename K>
@@ -173,12 +178,12 @@ struct mla_cache {
   RopeBands rope{};
   int device = 0;
 
-  __nv_bfloat16* ckv = nullptr;
-  __nv_bfloat16* krope = nullptr;
-  __nv_bfloat16* qp = nullptr;
-  __nv_bfloat16* o_lat = nullptr;
-  __nv_bfloat16* wqcat = nullptr;
-  __nv_bfloat16* wov = nullptr;
+  __half* ckv = nullptr;           // fp16 latent planes (ring + chunk tail)
+  __half* krope = nullptr;
+  __half* qp = nullptr;            // fp16 absorbed queries
+  __half* o_lat = nullptr;         // fp16 P . c_kv
+  __nv_bfloat16* wqcat = nullptr;  // bf16: multiplies the caller's bf16 hidden states
+  __half* wov = nullptr;           // fp16: multiplies o_lat
   int* status = nullptr;
 
   CUtensorMap map_wqcat{};         // B operand of the projections: box 64 x 224
@@ -273,9 +278,9 @@ mla_status launch_latent_gemm(mla_cache* c, const void* x, int64_t rows, int64_t
   ep.base_row = base_row;
   ep.q_scale = c->softmax_scale * 1.4426950408889634f;
   ep.rope = c->rope;
-  using Sm = mla::GemmSmem<kQK, kProjStages>;
+  using Sm = mla::GemmSmem<kQK, kProjAStages, kProjBStages>;
   dim3 grid((unsigned)((rows + 127) / 128), (unsigned)grid_y, (unsigned)cfg.batch);
-  mla::tc_gemm_kernel<kQK, kProjStages, mla::kEpiLatent>
+  mla::tc_gemm_kernel<kQK, kProjAStages, kProjBStages, mla::kEpiLatent, false>
       <<<grid, mla::kGemmThreads, Sm::kBytes, st>>>(map_x, c->map_wqcat, (int)rows, cfg.hidden,
                                                    b_row0, ep, c->status);
   return check_launch("latent projection");
@@ -454,20 +459,20 @@ mla_status mla_cache_create(const mla_config* cfg, const mla_weights* w, void* s
   if (s != MLA_OK) return cleanup(s);
   s = make_map(&c->map_wov, c->wov, (uint64_t)k.n_heads * kLatent, k.hidden, 1,
                (uint64_t)k.n_heads * kLatent * 2, (uint64_t)k.hidden * k.n_heads * kLatent * 2,
-               64, c->out_bn, CU_TENSOR_MAP_SWIZZLE_128B);
+               64, c->out_bn, CU_TENSOR_MAP_SWIZZLE_128B, true);
   if (s != MLA_OK) return cleanup(s);
 
   static std::once_flag attr_once;
   static mla_status attr_status = MLA_OK;
   std::call_once(attr_once, [] {
-    mla_status r = set_smem(mla::tc_gemm_kernel<kQK, kProjStages, mla::kEpiLatent>,
-                            mla::GemmSmem<kQK, kProjStages>::kBytes);
+    mla_status r = set_smem(mla::tc_gemm_kernel<kQK, kProjAStages, kProjBStages, mla::kEpiLatent, false>,
+                            mla::GemmSmem<kQK, kProjAStages, kProjBStages>::kBytes);
     if (r == MLA_OK)
-      r = set_smem(mla::tc_gemm_kernel<256, kOutStages, mla::kEpiStore>,
-                   mla::GemmSmem<256, kOutStages>::kBytes);
+      r = set_smem(mla::tc_gemm_kernel<256, kOutAStages, kOutBStages, mla::kEpiStore, true>,
+                   mla::GemmSmem<256, kOutAStages, kOutBStages>::kBytes);
     if (r == MLA_OK)
-      r = set_smem(mla::tc_gemm_kernel<128, kOutStages, mla::kEpiStore>,
-                   mla::GemmSmem<128, kOutStages>::kBytes);
+      r = set_smem(mla::tc_gemm_kernel<128, kOutAStages, kOutBStages, mla::kEpiStore, true>,
+                   mla::GemmSmem<128, kOutAStages, kOutBStages>::kBytes);
     if (r == MLA_OK)
       r = set_smem(mla::window_attn_kernel<kAttnStages, kAttnPInTmem>,
                    mla::AttnSmem<kAttnStages, kAttnPInTmem>::kBytes);
@@ -534,18 +539,18 @@ mla_status mla_window_attention(mla_cache* c, const void* x_chunk, int32_t n_fra
     const uint64_t qp_rows = (uint64_t)c->max_q_tokens * cfg.n_heads;
     CUtensorMap mqc, mqr, mkc, mkr;
     if ((s = make_map(&mqc, c->qp, kQK, R, cfg.batch, kQK * 2, qp_rows * kQK * 2, 64, 128,
-                      CU_TENSOR_MAP_SWIZZLE_128B)) != MLA_OK)
+                      CU_TENSOR_MAP_SWIZZLE_128B, true)) != MLA_OK)
       return s;
     if ((s = make_map(&mqr, c->qp, kQK, R, cfg.batch, kQK * 2, qp_rows * kQK * 2, 32, 128,
-                      CU_TENSOR_MAP_SWIZZLE_64B)) != MLA_OK)
+                      CU_TENSOR_MAP_SWIZZLE_64B, true)) != MLA_OK)
       return s;
     if ((s = make_map(&mkc, c->ckv, kLatent, n_keys, cfg.batch, kLatent * 2,
                       (uint64_t)c->rows_per_stream * kLatent * 2, 64, 128,
-                      CU_TENSOR_MAP_SWIZZLE_128B)) != MLA_OK)
+                      CU_TENSOR_MAP_SWIZZLE_128B, true)) != MLA_OK)
       return s;
     if ((s = make_map(&mkr, c->krope, kRope, n_keys, cfg.batch, kRope * 2,
                       (uint64_t)c->rows_per_stream * kRope * 2, 32, 128,
-                      CU_TENSOR_MAP_SWIZZLE_64B)) != MLA_OK)
+                      CU_TENSOR_MAP_SWIZZLE_64B, true)) != MLA_OK)
       return s;
     mla::AttnArgs a{};
     a.rows = (int32_t)R;
@@ -566,7 +571,7 @@ mla_status mla_window_attention(mla_cache* c, const void* x_chunk, int32_t n_fra
     const uint64_t kin = (uint64_t)cfg.n_heads * kLatent;
     if ((s = make_map(&ma, c->o_lat, kin, nq, cfg.batch, kin * 2,
                       (uint64_t)c->max_q_tokens * kin * 2, 64, 128,
-                      CU_TENSOR_MAP_SWIZZLE_128B)) != MLA_OK)
+                      CU_TENSOR_MAP_SWIZZLE_128B, true)) != MLA_OK)
       return s;
     EpiArgs ep{};
     ep.out = static_cast<__nv_bfloat16*>(out);
@@ -576,12 +581,12 @@ mla_status mla_window_attention(mla_cache* c, const void* x_chunk, int32_t n_fra
     dim3 grid((unsigned)((nq + 127) / 128), (unsigned)(cfg.hidden / c->out_bn),
               (unsigned)cfg.batch);
     if (c->out_bn == 256) {
-      mla::tc_gemm_kernel<256, kOutStages, mla::kEpiStore>
-          <<<grid, mla::kGemmThreads, mla::GemmSmem<256, kOutStages>::kBytes, st>>>(
+      mla::tc_gemm_kernel<256, kOutAStages, kOutBStages, mla::kEpiStore, true>
+          <<<grid, mla::kGemmThreads, mla::GemmSmem<256, kOutAStages, kOutBStages>::kBytes, st>>>(
               ma, c->map_wov, (int)nq, (int)kin, 0, ep, c->status);
     } else {
-      mla::tc_gemm_kernel<128, kOutStages, mla::kEpiStore>
-          <<<grid, mla::kGemmThreads, mla::GemmSmem<128, kOutStages>::kBytes, st>>>(
+      mla::tc_gemm_kernel<128, kOutAStages, kOutBStages, mla::kEpiStore, true>
+          <<<grid, mla::kGemmThreads, mla::GemmSmem<128, kOutAStages, kOutBStages>::kBytes, st>>>(
               ma, c->map_wov, (int)nq, (int)kin, 0, ep, c->status);
     }
     if ((s = check_launch("output projection")) != MLA_OK) return s;

@@ -1,7 +1,9 @@
 // window_attn.cuh - latent-window attention on tcgen05 (sm_100a).
 //
 // Rows r = (query token, head) of the absorbed, rotated, pre-scaled queries Qp[r] (224 =
-// 192 latent + 32 RoPE channels) attend to every key j of the window plus the chunk:
+// 192 latent + 32 RoPE channels) attend to every key j of the window plus the chunk.  Qp, the
+// latent cache, P and o_lat are fp16 (16-bit like the paper's bf16/fp16 cache; fp16 keeps three
+// more mantissa bits); every MMA accumulates in fp32:
 //
 //   s_j = Qp[r] . [c_kv_j | k_rope_j]          (log2-domain scores: Qp carries scale*log2 e)
 //   o_lat[r] = sum_j 2^(s_j - m) c_kv_j / sum_j 2^(s_j - m)
@@ -21,8 +23,8 @@
 //               S is double-buffered in TMEM so S_{j+1} runs while softmax works on S_j.
 //   warps 2..5  softmax: one row per thread, tcgen05.ld of its S row, running max with lazy
 //               rescaling (O is rescaled in TMEM only when the max grows by > 2^8), ex2,
-//               P_j as bf16 into shared memory (P_IN_TMEM = false) or tensor memory (true);
-//               finally O / l -> bf16 -> o_lat, staged for coalesced 384-byte row stores.
+//               P_j as fp16 into shared memory (P_IN_TMEM = false) or tensor memory (true);
+//               finally O / l -> fp16 -> o_lat, staged for coalesced 384-byte row stores.
 //
 // TMEM columns: S0 [0,128), S1 [128,256), O [256,448), P [448,512) (P_IN_TMEM only).
 #pragma once
@@ -52,7 +54,7 @@ struct AttnSmem {
 struct AttnArgs {
   int32_t rows;       // R = n_q * n_heads valid rows per stream
   int32_t n_keys;     // keys per stream (window + chunk)
-  __nv_bfloat16* o_lat;
+  __half* o_lat;               // fp16
   int64_t o_lat_batch_stride;  // elements
 };
 
@@ -143,8 +145,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc_s = idesc_bf16_f32(128, kTileKeys, false);
-      constexpr uint32_t idesc_o = idesc_bf16_f32(128, 192, true);
+      constexpr uint32_t idesc_s = idesc_f32acc(128, kTileKeys, false, true);
+      constexpr uint32_t idesc_o = idesc_f32acc(128, 192, true, true);
       const uint32_t q_base = smem_u32(smem + L::kQ);
       bool ok = mbar_wait(q_full, 0, status);
       for (int j = 0; ok && j <= nt; ++j) {
@@ -224,9 +226,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         for (int i = 0; i < kTileKeys; ++i)
           if (i >= valid) s[i] = -INFINITY;
       }
-      float mx = s[0];
+      // Row max with 8 independent partial maxima: one softmax warp per SM sub-partition, so
+      // a serial 128-long dependency chain would sit on the critical path of every tile.
+      float pm[8];
 #pragma unroll
-      for (int i = 1; i < kTileKeys; ++i) mx = fmaxf(mx, s[i]);
+      for (int k = 0; k < 8; ++k) pm[k] = s[k];
+#pragma unroll
+      for (int i = 8; i < kTileKeys; ++i) pm[i & 7] = fmaxf(pm[i & 7], s[i]);
+      const float mx = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
+                             fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
       float alpha = 1.f;
       bool rescale = false;
       if (j == 0) {
@@ -237,16 +245,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         rescale = true;
         l_sum *= alpha;
       }
-      float tile_sum = 0.f;
+      float ps[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
       uint32_t pk[kTileKeys / 2];
 #pragma unroll
       for (int i = 0; i < kTileKeys / 2; ++i) {
         const float p0 = ex2_approx(s[2 * i] - m_used);
         const float p1 = ex2_approx(s[2 * i + 1] - m_used);
-        pk[i] = pack_bf16x2(p0, p1);
-        tile_sum += p0 + p1;
+        pk[i] = pack_f16x2(p0, p1);
+        ps[i & 7] += p0 + p1;
       }
-      l_sum += tile_sum;
+      l_sum += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
 
       // P buffer and O become free once PV_{j-1} has completed.
       if (j >= 1 && !mbar_wait(pv_done, (uint32_t)(j - 1) & 1u, status)) { ok = false; break; }
@@ -297,14 +305,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           reinterpret_cast<uint4*>(st_row + c * 64)[q] = make_uint4(
-              pack_bf16x2(__uint_as_float(o[8 * q + 0]) * inv_l, __uint_as_float(o[8 * q + 1]) * inv_l),
-              pack_bf16x2(__uint_as_float(o[8 * q + 2]) * inv_l, __uint_as_float(o[8 * q + 3]) * inv_l),
-              pack_bf16x2(__uint_as_float(o[8 * q + 4]) * inv_l, __uint_as_float(o[8 * q + 5]) * inv_l),
-              pack_bf16x2(__uint_as_float(o[8 * q + 6]) * inv_l, __uint_as_float(o[8 * q + 7]) * inv_l));
+              pack_f16x2(__uint_as_float(o[8 * q + 0]) * inv_l, __uint_as_float(o[8 * q + 1]) * inv_l),
+              pack_f16x2(__uint_as_float(o[8 * q + 2]) * inv_l, __uint_as_float(o[8 * q + 3]) * inv_l),
+              pack_f16x2(__uint_as_float(o[8 * q + 4]) * inv_l, __uint_as_float(o[8 * q + 5]) * inv_l),
+              pack_f16x2(__uint_as_float(o[8 * q + 6]) * inv_l, __uint_as_float(o[8 * q + 7]) * inv_l));
         }
       }
       __syncwarp();
-      __nv_bfloat16* out = args.o_lat + z * args.o_lat_batch_stride;
+      __half* out = args.o_lat + z * args.o_lat_batch_stride;
       for (int rr = 0; rr < 32; ++rr) {
         const int trow = sub * 32 + rr;
         const int gr = m0 + trow;

@@ -230,11 +230,14 @@ class OracleLayer:
         Q = np.concatenate([q_nope, q_rope], axis=1)
         return Q, K, v
 
-    def attention(self, x_chunk, rows=None, positions: str = "local", return_parts: bool = False):
+    def attention(self, x_chunk, rows=None, positions: str = "local", return_parts: bool = False,
+                  heads=None):
         """Output [n_q, d] for the query chunk x_chunk [n_q, d] (or for the query rows `rows` only).
 
         With return_parts, also returns per head the softmax matrix P [n_h, n_q, N], the
         latent-space output P c [n_q, n_h, d_c] and the head outputs O [n_q, n_h, d_head].
+        `heads` restricts the work to a subset of heads (the other heads contribute zero to the
+        output); it exists only to time bounded samples and is never used for parity.
         """
         d = self.d
         ctx = self.keys_and_queries(x_chunk, positions)
@@ -243,7 +246,7 @@ class OracleLayer:
         O = np.zeros((nq, nh, dv))
         Pc = np.zeros((nq, nh, d["d_latent"]))
         Ps = []
-        for h in range(nh):
+        for h in (range(nh) if heads is None else heads):
             Q, K, V = self.head_qkv(ctx, h, rows)
             S = (Q @ K.T) * self.scale                       # [n_q, N]
             S = S - S.max(axis=1, keepdims=True)

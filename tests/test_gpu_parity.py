@@ -73,7 +73,11 @@ def full_check(pair: Pair, x_chunk, what: str, intermediates: bool = True):
             qp = pair.gpu.copy_buffer(0, (pair.w.batch, pair.gpu.cfg.max_chunk_frames * pair.F * 12, 224))
             assert_close(qp[b, :nq * 12], oracle_qp(pair, x_chunk[b], b), f"{what}: Qp (stream {b})")
             ol = pair.gpu.copy_buffer(1, (pair.w.batch, pair.gpu.cfg.max_chunk_frames * pair.F * 12, 192))
-            assert_close(ol[b, :nq * 12], parts["Pc"].reshape(-1, 192), f"{what}: o_lat (stream {b})")
+            # o_lat is an internal bf16 intermediate, not an output: its RMS is well below its
+            # peaks (rows that attend sharply copy one latent), so bf16 rounding of the queries
+            # shows up as a larger max-abs/RMS than in the projected output.  Same L2 bar.
+            assert_close(ol[b, :nq * 12], parts["Pc"].reshape(-1, 192), f"{what}: o_lat (stream {b})",
+                         max_tol=1e-1)
     pair.check_status()
     return out
 
