@@ -126,6 +126,28 @@ mla_status mla_cache_append(mla_cache* c, const void* x, int32_t n_frames, void*
 mla_status mla_window_attention(mla_cache* c, const void* x_chunk, int32_t n_frames, void* out,
                                 void* stream);
 
+/* Same computation and result as mla_window_attention, for callers that must not allocate
+ * device memory while they run: code whose device memory belongs to a pooled or budgeted
+ * allocator it may not bypass, and latency-critical loops that cannot afford the implicit
+ * device synchronisation a cudaMalloc/cudaFree can cause.  The paper has no counterpart; this
+ * is a property of the library, not of the method.
+ *
+ * The per-call scratch - absorbed queries and the latent-space attention output, 832 bytes per
+ * (stream, query token, head) - lives in one fixed 32 MiB array inside the library on every GPU
+ * that loads it (held until the process exits), not in the cache.  This call allocates nothing:
+ * no cudaMalloc, no cudaFree, no allocating library routine.  The cache itself still has to be
+ * created once, beforehand, with mla_cache_create.
+ *  - Limit: batch * n_frames * F * n_heads * 832 bytes (plus 256 for alignment) must fit in
+ *    32 MiB, else MLA_ERR_INVALID_ARGUMENT with the required size in mla_last_error().
+ *  - The first call on a device looks up the array's device address (once per device, with
+ *    the cache's device current); make that first call before any stream capture.
+ *  - Every call on a device shares the one array and leaves the last call's contents in it.
+ *    Nothing in it has to start at zero (each call writes every row it reads back), but calls
+ *    whose kernels overlap on the GPU (other streams, other caches) race on it: serialise them.
+ *  - Arguments, layouts, stream ordering and errors otherwise as mla_window_attention. */
+mla_status mla_window_attention_noalloc(mla_cache* c, const void* x_chunk, int32_t n_frames,
+                                        void* out, void* stream);
+
 /* Free everything the cache owns (synchronises the device first).  NULL-safe. */
 void mla_cache_destroy(mla_cache* c);
 

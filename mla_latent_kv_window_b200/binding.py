@@ -26,7 +26,8 @@ KERNEL_NAMES = ("append", "qproj", "attention", "oproj")
 
 EXPORTED = (
     "mla_config_check", "mla_ring_slot", "mla_ring_bytes", "mla_cache_device_bytes",
-    "mla_cache_create", "mla_cache_append", "mla_window_attention", "mla_cache_destroy",
+    "mla_cache_create", "mla_cache_append", "mla_window_attention", "mla_window_attention_noalloc",
+    "mla_cache_destroy",
     "mla_cache_state", "mla_cache_sync", "mla_cache_read", "mla_cache_debug_buffers", "mla_cache_copy_buffer",
     "mla_cache_profile_enable", "mla_cache_profile_read", "mla_status_string", "mla_last_error",
 )
@@ -83,6 +84,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "mla_cache_create": (I32, [P(mla_config), P(mla_weights), VP, P(VP)]),
         "mla_cache_append": (I32, [VP, VP, I32, VP]),
         "mla_window_attention": (I32, [VP, VP, I32, VP, VP]),
+        "mla_window_attention_noalloc": (I32, [VP, VP, I32, VP, VP]),
         "mla_cache_destroy": (None, [VP]),
         "mla_cache_state": (I32, [VP, P(I64), P(I32)]),
         "mla_cache_sync": (I32, [VP, VP]),
@@ -173,6 +175,14 @@ def mla_window_attention(cache: int, x_chunk, n_frames: int, out, stream=None) -
     _check(load_library().mla_window_attention(cache, _dev_ptr(x_chunk, "x_chunk"), n_frames,
                                                _dev_ptr(out, "out"), _stream_handle(stream)),
            "mla_window_attention")
+
+
+def mla_window_attention_noalloc(cache: int, x_chunk, n_frames: int, out, stream=None) -> None:
+    """mla_window_attention with its per-call scratch in the library's fixed 32 MiB device array
+    (no device allocation in the call); see include/mla.h for the size limit and sharing rules."""
+    _check(load_library().mla_window_attention_noalloc(cache, _dev_ptr(x_chunk, "x_chunk"), n_frames,
+                                                       _dev_ptr(out, "out"), _stream_handle(stream)),
+           "mla_window_attention_noalloc")
 
 
 def mla_cache_destroy(cache: int) -> None:

@@ -288,6 +288,43 @@ mla_status launch_latent_gemm(mla_cache* c, const void* x, int64_t rows, int64_t
 
 }  // namespace
 
+// ------------------------------------------------------------------------------ no-alloc variant
+// Scratch of mla_window_attention_noalloc: the absorbed queries (Qp) and the latent-space
+// attention output (o_lat) of one call, in a fixed per-device array instead of cache-owned
+// buffers.  Every GPU that loads this library holds these 32 MiB until the process exits.
+constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device.  In host code the array's name
+// is only a host-side stand-in, so the address is looked up once per device (with that device
+// current) and cached.
+mla_status noalloc_scratch(void** out) {
+  int dev = 0;
+  MLA_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kMaxDevices) return fail(MLA_ERR_UNSUPPORTED, "device index %d too large", dev);
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || p == nullptr)
+      return fail(MLA_ERR_CUDA, "cudaGetSymbolAddress of the no-alloc scratch failed: %s",
+                  cudaGetErrorString(e));
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return MLA_OK;
+}
+
+size_t align256(size_t n) { return (n + 255) & ~size_t(255); }
+
+}  // namespace
+
 extern "C" {
 
 const char* mla_status_string(mla_status s) {
@@ -590,6 +627,125 @@ mla_status mla_window_attention(mla_cache* c, const void* x_chunk, int32_t n_fra
               ma, c->map_wov, (int)nq, (int)kin, 0, ep, c->status);
     }
     if ((s = check_launch("output projection")) != MLA_OK) return s;
+  }
+  return MLA_OK;
+}
+
+mla_status mla_window_attention_noalloc(mla_cache* c, const void* x_chunk, int32_t n_frames,
+                                        void* out, void* stream) {
+  if (!c || !x_chunk || !out) return fail(MLA_ERR_INVALID_ARGUMENT, "NULL argument");
+  const mla_config& cfg = c->cfg;
+  if (n_frames < 1 || n_frames > cfg.max_chunk_frames)
+    return fail(MLA_ERR_INVALID_ARGUMENT, "n_frames must be in [1, max_chunk_frames=%d]",
+                cfg.max_chunk_frames);
+  if (!aligned16(x_chunk) || !aligned16(out))
+    return fail(MLA_ERR_INVALID_ARGUMENT, "x_chunk and out must be 16-byte aligned");
+  const int64_t nq = (int64_t)n_frames * c->F;
+  const int64_t R = nq * cfg.n_heads;                    // Qp / o_lat rows per stream
+  const size_t qp_bytes = align256((size_t)cfg.batch * R * kQK * 2);
+  const size_t ol_bytes = (size_t)cfg.batch * R * kLatent * 2;
+  if (qp_bytes + ol_bytes > kNoAllocScratchBytes)
+    return fail(MLA_ERR_INVALID_ARGUMENT,
+                "no-alloc scratch too small: this call needs %zu bytes (batch * tokens * heads * "
+                "832 B), the fixed scratch holds %zu; use mla_window_attention instead",
+                qp_bytes + ol_bytes, kNoAllocScratchBytes);
+  int dev = 0;
+  MLA_CUDA(cudaGetDevice(&dev));
+  if (dev != c->device)
+    return fail(MLA_ERR_STATE, "the cache lives on device %d but device %d is current",
+                c->device, dev);
+  void* scratch = nullptr;
+  mla_status s = noalloc_scratch(&scratch);
+  if (s != MLA_OK) return s;
+  __half* qp = static_cast<__half*>(scratch);
+  __half* o_lat = reinterpret_cast<__half*>(static_cast<unsigned char*>(scratch) + qp_bytes);
+
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t valid = c->frames_appended < cfg.window_frames ? c->frames_appended
+                                                               : cfg.window_frames;
+  const int64_t base_row = valid * c->F;
+  const int64_t n_keys = base_row + nq;
+
+  // 1. absorbed queries (into the scratch) + chunk latents (into the cache's chunk tail)
+  {
+    CUtensorMap map_x;
+    if ((s = make_map(&map_x, x_chunk, cfg.hidden, nq, cfg.batch, (uint64_t)cfg.hidden * 2,
+                      (uint64_t)nq * cfg.hidden * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B)) != MLA_OK)
+      return s;
+    EpiArgs ep{};
+    ep.ckv = c->ckv;
+    ep.krope = c->krope;
+    ep.rows_per_stream = c->rows_per_stream;
+    ep.qp = qp;
+    ep.qp_rows_per_stream = R;
+    ep.latent_y = cfg.n_heads;
+    ep.n_heads = cfg.n_heads;
+    ep.ring_mode = 0;
+    ep.t0 = c->frames_appended;
+    ep.window_frames = cfg.window_frames;
+    ep.tokens_per_frame = c->F;
+    ep.frame_w = cfg.frame_w;
+    ep.base_row = base_row;
+    ep.q_scale = c->softmax_scale * 1.4426950408889634f;
+    ep.rope = c->rope;
+    using Sm = mla::GemmSmem<kQK, kProjAStages, kProjBStages>;
+    dim3 grid((unsigned)((nq + 127) / 128), (unsigned)(cfg.n_heads + 1), (unsigned)cfg.batch);
+    mla::tc_gemm_kernel<kQK, kProjAStages, kProjBStages, mla::kEpiLatent, false>
+        <<<grid, mla::kGemmThreads, Sm::kBytes, st>>>(map_x, c->map_wqcat, (int)nq, cfg.hidden,
+                                                     0, ep, c->status);
+    if ((s = check_launch("no-alloc latent projection")) != MLA_OK) return s;
+  }
+  // 2. window attention, o_lat into the scratch
+  {
+    CUtensorMap mqc, mqr, mkc, mkr;
+    if ((s = make_map(&mqc, qp, kQK, R, cfg.batch, kQK * 2, (uint64_t)R * kQK * 2, 64, 128,
+                      CU_TENSOR_MAP_SWIZZLE_128B, true)) != MLA_OK)
+      return s;
+    if ((s = make_map(&mqr, qp, kQK, R, cfg.batch, kQK * 2, (uint64_t)R * kQK * 2, 32, 128,
+                      CU_TENSOR_MAP_SWIZZLE_64B, true)) != MLA_OK)
+      return s;
+    if ((s = make_map(&mkc, c->ckv, kLatent, n_keys, cfg.batch, kLatent * 2,
+                      (uint64_t)c->rows_per_stream * kLatent * 2, 64, 128,
+                      CU_TENSOR_MAP_SWIZZLE_128B, true)) != MLA_OK)
+      return s;
+    if ((s = make_map(&mkr, c->krope, kRope, n_keys, cfg.batch, kRope * 2,
+                      (uint64_t)c->rows_per_stream * kRope * 2, 32, 128,
+                      CU_TENSOR_MAP_SWIZZLE_64B, true)) != MLA_OK)
+      return s;
+    mla::AttnArgs a{};
+    a.rows = (int32_t)R;
+    a.n_keys = (int32_t)n_keys;
+    a.o_lat = o_lat;
+    a.o_lat_batch_stride = R * kLatent;
+    using Sm = mla::AttnSmem<kAttnStages, kAttnPInTmem>;
+    dim3 grid((unsigned)((R + 127) / 128), (unsigned)cfg.batch);
+    mla::window_attn_kernel<kAttnStages, kAttnPInTmem>
+        <<<grid, mla::kAttnThreads, Sm::kBytes, st>>>(mqc, mqr, mkc, mkr, a, c->status);
+    if ((s = check_launch("no-alloc window attention")) != MLA_OK) return s;
+  }
+  // 3. output projection from the scratch o_lat
+  {
+    CUtensorMap ma;
+    const uint64_t kin = (uint64_t)cfg.n_heads * kLatent;
+    if ((s = make_map(&ma, o_lat, kin, nq, cfg.batch, kin * 2, (uint64_t)nq * kin * 2, 64, 128,
+                      CU_TENSOR_MAP_SWIZZLE_128B, true)) != MLA_OK)
+      return s;
+    EpiArgs ep{};
+    ep.out = static_cast<__nv_bfloat16*>(out);
+    ep.out_batch_stride = nq * cfg.hidden;
+    ep.ld_out = cfg.hidden;
+    dim3 grid((unsigned)((nq + 127) / 128), (unsigned)(cfg.hidden / c->out_bn),
+              (unsigned)cfg.batch);
+    if (c->out_bn == 256) {
+      mla::tc_gemm_kernel<256, kOutAStages, kOutBStages, mla::kEpiStore, true>
+          <<<grid, mla::kGemmThreads, mla::GemmSmem<256, kOutAStages, kOutBStages>::kBytes, st>>>(
+              ma, c->map_wov, (int)nq, (int)kin, 0, ep, c->status);
+    } else {
+      mla::tc_gemm_kernel<128, kOutAStages, kOutBStages, mla::kEpiStore, true>
+          <<<grid, mla::kGemmThreads, mla::GemmSmem<128, kOutAStages, kOutBStages>::kBytes, st>>>(
+              ma, c->map_wov, (int)nq, (int)kin, 0, ep, c->status);
+    }
+    if ((s = check_launch("no-alloc output projection")) != MLA_OK) return s;
   }
   return MLA_OK;
 }
