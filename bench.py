@@ -103,7 +103,7 @@ def peaks():
 
 def kernel_source_hash() -> str:
     h = hashlib.sha256()
-    for f in ("ptx.cuh", "gemm_tc.cuh", "window_attn.cuh", "mla_api.cu"):
+    for f in ("ptx.cuh", "gemm_tc.cuh", "window_attn.cuh", "dense_attn.cuh", "mla_api.cu"):
         h.update(open(os.path.join(ROOT, "mla_latent_kv_window_b200", "csrc", f), "rb").read())
     return h.hexdigest()[:16]
 
@@ -314,6 +314,7 @@ def run_ours(args, rank, local, world):
     e2e_value = world * nq * e2e_steps / (e2e_ms / 1e3)
 
     status_ok = all(B.mla_cache_sync(c.handle) == 0 for c in caches)
+    layout = layout_baseline(B, w, dims, dev, stream, attn_ms, attn_flop) if rank == 0 else None
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -362,12 +363,85 @@ def run_ours(args, rank, local, world):
             "device_status_ok": status_ok,
             "clocks": clk,
         }
+        if layout is not None:
+            line["layout_baseline"] = layout
         if cpu is not None:
             line["cpu_baseline"] = cpu
         print(json.dumps(line), flush=True)
     for c in caches:
         c.close()
     replicas.shutdown()
+
+
+def _event_ms(fn, stream, reps=10, warm=3):
+    import torch
+    for _ in range(warm):
+        fn()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(reps):
+        fn()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / reps
+
+
+def layout_baseline(B, w, dims, dev, stream, latent_ms, latent_flop):
+    """The layout comparison of the long-window workload: dense per-head 12 x 128 K/V attention at
+    the 21-frame window (same keys as the latent kernel above), and the latent kernel at a
+    63-frame window (98,280 cached tokens, about as many bytes as 4.6 dense frames)."""
+    import torch
+
+    import mla_synth
+    F, nq = w.F, w.query_frames * w.F
+    n_kv = w.window_frames * F + nq
+    H = dims["n_heads"]
+    q = mla_synth.normal_bf16((1, nq, H, 128), 1.0, 1).to(dev)
+    k = mla_synth.normal_bf16((1, n_kv, H, 128), 1.0, 2).to(dev)
+    v = mla_synth.normal_bf16((1, n_kv, H, 128), 1.0, 3).to(dev)
+    o = torch.empty_like(q)
+    dense_ms = _event_ms(lambda: B.mla_dense_attention(q, k, v, o, 0.0, stream), stream)
+    dense_ok = B.mla_dense_sync(stream) == 0
+    dense_flop = 4 * nq * n_kv * 128 * H
+    del q, k, v, o
+    w63 = mla_synth.WORKLOADS["wan_w63_q1"]
+    wts = {kk: vv.to(dev) for kk, vv in mla_synth.make_weights(dims, mla_synth.weight_seed(w63, 0)).items()}
+    c63 = B.LatentWindowCache(dims, wts, w63.frame_h, w63.frame_w, w63.window_frames, 1)
+    c63.append(mla_synth.make_hidden(1, 63 * F, dims["hidden"], mla_synth.fill_seed(w63, 0)).to(dev))
+    x = mla_synth.make_hidden(1, F, dims["hidden"], mla_synth.chunk_seed(w63, 0, 0)).to(dev)
+    out = torch.empty_like(x)
+    B.mla_cache_profile_enable(c63.handle, True)
+    for _ in range(3):
+        c63.attention(x, out)
+    torch.cuda.synchronize()
+    B.mla_cache_profile_read(c63.handle)
+    for _ in range(10):
+        c63.attention(x, out)
+    torch.cuda.synchronize()
+    p63 = B.mla_cache_profile_read(c63.handle)
+    ok63 = B.mla_cache_sync(c63.handle) == 0
+    c63.close()
+    a63_ms = p63["attention"][0] / max(p63["attention"][1], 1)
+    keys63 = 63 * F + F
+    flop63 = FLOP_PER_QHK * nq * H * keys63
+    cache_bytes = lambda per_tok, frames: frames * F * per_tok * 2
+    return {
+        "dense_per_head_21_frames": {
+            "kernel": "dense_attn_kernel (12 x 128 K and V per token, bf16)", "keys": n_kv,
+            "ms": round(dense_ms, 4), "tflops": round(dense_flop / (dense_ms / 1e3) / 1e12, 1),
+            "query_tokens_per_s": round(nq / (dense_ms / 1e3), 1),
+            "cache_bytes_per_layer": cache_bytes(3072, w.window_frames), "status_ok": dense_ok},
+        "latent_21_frames": {
+            "ms": round(latent_ms, 4), "tflops": round(latent_flop / (latent_ms / 1e3) / 1e12, 1),
+            "query_tokens_per_s": round(nq / (latent_ms / 1e3), 1),
+            "cache_bytes_per_layer": cache_bytes(224, w.window_frames)},
+        "latent_63_frames": {
+            "keys": keys63, "ms": round(a63_ms, 4), "tflops": round(flop63 / (a63_ms / 1e3) / 1e12, 1),
+            "query_tokens_per_s": round(nq / (a63_ms / 1e3), 1),
+            "cache_bytes_per_layer": cache_bytes(224, 63), "status_ok": ok63},
+        "note": "dense counts 512 flop per (query, head, key); latent 832 (absorbed scores + P.c_kv)",
+    }
 
 
 # ---------------------------------------------------------------------------- the oracle on CPU

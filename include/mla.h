@@ -148,6 +148,22 @@ mla_status mla_window_attention(mla_cache* c, const void* x_chunk, int32_t n_fra
 mla_status mla_window_attention_noalloc(mla_cache* c, const void* x_chunk, int32_t n_frames,
                                         void* out, void* stream);
 
+/* Dense per-head attention, the layout VideoMLA replaces ([VideoMLA] §1: every cached token
+ * keeps 12 x 128 keys and 12 x 128 values, 3,072 scalars): the measurement baseline of the
+ * latent-window kernel.  Stateless; no device memory is allocated.
+ *   q   [batch][n_q][n_heads][d_head]  bf16      k, v [batch][n_kv][n_heads][d_head]  bf16
+ *   out [batch][n_q][n_heads][d_head]  bf16      out = softmax(scale q k^T) v per head
+ * softmax_scale 0 -> 1/sqrt(d_head).  Built for d_head == 128 (MLA_ERR_UNSUPPORTED otherwise).
+ * Every query attends to all n_kv keys (no mask).  Device waits are bounded; a timeout is
+ * reported by mla_dense_sync (one status word per device, shared by all dense calls). */
+mla_status mla_dense_attention(const void* q, const void* k, const void* v, void* out,
+                               int32_t batch, int32_t n_q, int32_t n_kv, int32_t n_heads,
+                               int32_t d_head, float softmax_scale, void* stream);
+
+/* Synchronise `stream` and return the dense kernels' device status word (MLA_OK or
+ * MLA_ERR_DEVICE_TIMEOUT). */
+mla_status mla_dense_sync(void* stream);
+
 /* Free everything the cache owns (synchronises the device first).  NULL-safe. */
 void mla_cache_destroy(mla_cache* c);
 

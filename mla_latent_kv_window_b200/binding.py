@@ -27,7 +27,7 @@ KERNEL_NAMES = ("append", "qproj", "attention", "oproj")
 EXPORTED = (
     "mla_config_check", "mla_ring_slot", "mla_ring_bytes", "mla_cache_device_bytes",
     "mla_cache_create", "mla_cache_append", "mla_window_attention", "mla_window_attention_noalloc",
-    "mla_cache_destroy",
+    "mla_cache_destroy", "mla_dense_attention", "mla_dense_sync",
     "mla_cache_state", "mla_cache_sync", "mla_cache_read", "mla_cache_debug_buffers", "mla_cache_copy_buffer",
     "mla_cache_profile_enable", "mla_cache_profile_read", "mla_status_string", "mla_last_error",
 )
@@ -85,6 +85,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "mla_cache_append": (I32, [VP, VP, I32, VP]),
         "mla_window_attention": (I32, [VP, VP, I32, VP, VP]),
         "mla_window_attention_noalloc": (I32, [VP, VP, I32, VP, VP]),
+        "mla_dense_attention": (I32, [VP, VP, VP, VP, I32, I32, I32, I32, I32, ctypes.c_float, VP]),
+        "mla_dense_sync": (I32, [VP]),
         "mla_cache_destroy": (None, [VP]),
         "mla_cache_state": (I32, [VP, P(I64), P(I32)]),
         "mla_cache_sync": (I32, [VP, VP]),
@@ -183,6 +185,19 @@ def mla_window_attention_noalloc(cache: int, x_chunk, n_frames: int, out, stream
     _check(load_library().mla_window_attention_noalloc(cache, _dev_ptr(x_chunk, "x_chunk"), n_frames,
                                                        _dev_ptr(out, "out"), _stream_handle(stream)),
            "mla_window_attention_noalloc")
+
+
+def mla_dense_attention(q, k, v, out, softmax_scale: float = 0.0, stream=None) -> None:
+    """Dense per-head attention baseline: q [B, n_q, H, 128], k/v [B, n_kv, H, 128], out like q (bf16)."""
+    B, nq, H, D = q.shape
+    _check(load_library().mla_dense_attention(_dev_ptr(q, "q"), _dev_ptr(k, "k"), _dev_ptr(v, "v"),
+                                              _dev_ptr(out, "out"), B, nq, k.shape[1], H, D,
+                                              float(softmax_scale), _stream_handle(stream)),
+           "mla_dense_attention")
+
+
+def mla_dense_sync(stream=None) -> int:
+    return load_library().mla_dense_sync(_stream_handle(stream))
 
 
 def mla_cache_destroy(cache: int) -> None:

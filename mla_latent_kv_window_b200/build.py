@@ -9,7 +9,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libmla.so")
 SOURCES = [os.path.join(HERE, "csrc", "mla_api.cu")]
-DEPS = SOURCES + [os.path.join(HERE, "csrc", f) for f in ("ptx.cuh", "gemm_tc.cuh", "window_attn.cuh")] + \
+DEPS = SOURCES + [os.path.join(HERE, "csrc", f) for f in ("ptx.cuh", "gemm_tc.cuh", "window_attn.cuh", "dense_attn.cuh")] + \
     [os.path.join(ROOT, "include", "mla.h")]
 
 

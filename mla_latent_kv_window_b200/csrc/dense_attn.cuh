@@ -1,0 +1,274 @@
+// dense_attn.cuh - dense per-head attention (12 x 128 keys and values per token), the layout the
+// VideoMLA paper page replaces (§1: 2 x 12 x 128 = 3,072 cached scalars per token).  Built as
+// the measurement baseline next to the latent-window kernel, on the same sm_100a machinery.
+//
+//   out[q, h] = sum_j softmax_j(scale * Q[q, h] . K[j, h]) V[j, h]
+//
+// One CTA owns 128 query rows of one head.  Warp roles (192 threads):
+//   warp 0      TMA producer: the Q tile once (2 x 64-column SW128 boxes), then per 128-key tile
+//               K (2 boxes) and V (2 boxes) of this head into a KV_STAGES-deep ring.
+//   warp 1      TMEM allocator + single-thread MMA issuer:
+//                 S_j = Q K_j^T   M=128 N=128 K=128 (8 k-steps, both K-major)
+//                 O  += P_j V_j   M=128 N=128 K=128 (8 k-steps, V read MN-major, P from TMEM)
+//   warps 2..5  softmax (one row per thread, base 2, lazy O rescale), then O / l -> bf16 out.
+// TMEM columns: S0 [0,128), S1 [128,256), O [256,384), P [384,448).
+#pragma once
+
+#include "ptx.cuh"
+
+namespace mla {
+
+constexpr int kDenseThreads = 192;
+constexpr float kDenseRescaleLog2 = 8.0f;  // lazy O rescale when the max grows by > 2^8
+
+template <int KV_STAGES>
+struct DenseSmem {
+  static constexpr int kAtom = 128 * 128;                 // 128 rows x 64 bf16 (SW128)
+  static constexpr int kQ = 0;                            // 2 atoms
+  static constexpr int kKV = 2 * kAtom;
+  static constexpr int kStage = 4 * kAtom;                // K (2 atoms) + V (2 atoms)
+  static constexpr int kBar = kKV + KV_STAGES * kStage;
+  static constexpr int kBytes = kBar + 256 + 1024;
+  static_assert(kBytes <= 232448, "dense attention tile does not fit in shared memory");
+};
+
+struct DenseArgs {
+  int32_t n_q;         // query tokens per stream
+  int32_t n_kv;        // keys per stream
+  int32_t n_heads;
+  float scale_log2;    // softmax_scale * log2(e)
+  __nv_bfloat16* out;  // [B][n_q][n_heads][128]
+};
+
+template <int KV_STAGES>
+__global__ void __launch_bounds__(kDenseThreads, 1)
+    dense_attn_kernel(const __grid_constant__ CUtensorMap map_q,
+                      const __grid_constant__ CUtensorMap map_k,
+                      const __grid_constant__ CUtensorMap map_v, DenseArgs args, int* status) {
+  using L = DenseSmem<KV_STAGES>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
+  uint64_t* q_full = bars;
+  uint64_t* kv_full = bars + 1;
+  uint64_t* kv_empty = kv_full + KV_STAGES;
+  uint64_t* s_full = kv_empty + KV_STAGES;
+  uint64_t* s_free = s_full + 2;
+  uint64_t* p_full = s_free + 2;
+  uint64_t* pv_done = p_full + 1;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(pv_done + 1);
+
+  const uint32_t warp = warp_id();
+  const uint32_t lane = lane_id();
+  const int m0 = blockIdx.x * 128;
+  const int h = blockIdx.y;
+  const int z = blockIdx.z;
+  const int n_kv = args.n_kv;
+  const int nt = (n_kv + 127) / 128;
+  const int col0 = h * 128;  // this head's columns in the [tokens][n_heads * 128] views
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int s = 0; s < KV_STAGES; ++s) {
+      mbar_init(&kv_full[s], 1);
+      mbar_init(&kv_empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&s_full[s], 1);
+      mbar_init(&s_free[s], 128);
+    }
+    mbar_init(p_full, 128);
+    mbar_init(pv_done, 1);
+    fence_mbar_init();
+    tma_prefetch(&map_q);
+    tma_prefetch(&map_k);
+    tma_prefetch(&map_v);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  const uint32_t tmem_o = tmem + 256;
+  const uint32_t tmem_p = tmem + 384;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      const uint64_t keep = l2_policy_evict_last();   // K/V are re-read by every row tile of h
+      const uint64_t once = l2_policy_evict_first();
+      mbar_arrive_expect_tx(q_full, 2 * L::kAtom);
+      for (int a = 0; a < 2; ++a)
+        tma_load_3d_hint(smem + L::kQ + a * L::kAtom, &map_q, q_full, col0 + a * 64, m0, z, once);
+      int issued = 0;
+      for (int j = 0; j < nt; ++j) {
+        const int st = j % KV_STAGES;
+        if (!mbar_wait(&kv_empty[st], ((uint32_t)(j / KV_STAGES) & 1u) ^ 1u, status)) break;
+        uint8_t* kv = smem + L::kKV + st * L::kStage;
+        mbar_arrive_expect_tx(&kv_full[st], L::kStage);
+        for (int a = 0; a < 2; ++a) {
+          tma_load_3d_hint(kv + a * L::kAtom, &map_k, &kv_full[st], col0 + a * 64, j * 128, z, keep);
+          tma_load_3d_hint(kv + (2 + a) * L::kAtom, &map_v, &kv_full[st], col0 + a * 64, j * 128, z,
+                           keep);
+        }
+        issued = j + 1;
+      }
+      for (int j = issued > KV_STAGES ? issued - KV_STAGES : 0; j < issued; ++j)
+        mbar_wait(&kv_full[j % KV_STAGES], (uint32_t)(j / KV_STAGES) & 1u, status);
+      mbar_wait(q_full, 0, status);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = idesc_f32acc(128, 128, false, false);
+      constexpr uint32_t idesc_o = idesc_f32acc(128, 128, true, false);
+      const uint32_t q_base = smem_u32(smem + L::kQ);
+      bool ok = mbar_wait(q_full, 0, status);
+      for (int j = 0; ok && j <= nt; ++j) {
+        if (j < nt) {
+          const int st = j % KV_STAGES;
+          const int sb = j & 1;
+          if (!mbar_wait(&kv_full[st], (uint32_t)(j / KV_STAGES) & 1u, status)) break;
+          if (j >= 2 && !mbar_wait(&s_free[sb], (uint32_t)((j >> 1) - 1) & 1u, status)) break;
+          tc_fence_after();
+          const uint32_t k_base = smem_u32(smem + L::kKV + st * L::kStage);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t off = (kk >> 2) * L::kAtom + (kk & 3) * 32;
+            umma_ss(tmem + sb * 128, smem_desc(q_base + off, 16, 1024, kSwizzle128B),
+                    smem_desc(k_base + off, 16, 1024, kSwizzle128B), idesc_s, kk > 0 ? 1u : 0u);
+          }
+          tc_commit(&s_full[sb]);
+        }
+        if (j >= 1) {
+          const int jj = j - 1;
+          const int st = jj % KV_STAGES;
+          if (!mbar_wait(p_full, (uint32_t)jj & 1u, status)) break;
+          tc_fence_after();
+          const uint32_t v_base = smem_u32(smem + L::kKV + st * L::kStage + 2 * L::kAtom);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint64_t db = smem_desc(v_base + kk * 2048, L::kAtom, 1024, kSwizzle128B);
+            umma_ts(tmem_o, tmem_p + kk * 8, db, idesc_o, (jj > 0 || kk > 0) ? 1u : 0u);
+          }
+          tc_commit(pv_done);
+          tc_commit(&kv_empty[st]);
+        }
+      }
+    }
+  } else {
+    const uint32_t sub = warp & 3u;
+    const int row = sub * 32 + lane;
+    const uint32_t lane_off = (sub * 32u) << 16;
+    const float c = args.scale_log2;
+    float m_used = -INFINITY;   // running max of the raw scores
+    float l_sum = 0.f;
+    bool ok = true;
+    for (int j = 0; j < nt; ++j) {
+      const int sb = j & 1;
+      if (!mbar_wait(&s_full[sb], (uint32_t)(j >> 1) & 1u, status)) { ok = false; break; }
+      tc_fence_after();
+      float s[128];
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        tmem_ld32(tmem + lane_off + sb * 128 + q * 32, reinterpret_cast<uint32_t*>(s) + q * 32);
+      tmem_ld_wait();
+      tc_fence_before();
+      mbar_arrive(&s_free[sb]);
+      const int valid = n_kv - j * 128;
+      if (valid < 128) {
+#pragma unroll
+        for (int i = 0; i < 128; ++i)
+          if (i >= valid) s[i] = -INFINITY;
+      }
+      float pm[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) pm[k] = s[k];
+#pragma unroll
+      for (int i = 8; i < 128; ++i) pm[i & 7] = fmaxf(pm[i & 7], s[i]);
+      const float mx = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
+                             fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
+      float alpha = 1.f;
+      bool rescale = false;
+      if (j == 0) {
+        m_used = mx;
+      } else if ((mx - m_used) * c > kDenseRescaleLog2) {
+        alpha = ex2_approx((m_used - mx) * c);
+        m_used = mx;
+        rescale = true;
+        l_sum *= alpha;
+      }
+      const float mc = m_used * c;
+      float ps[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      uint32_t pk[64];
+#pragma unroll
+      for (int i = 0; i < 64; ++i) {
+        const float p0 = ex2_approx(fmaf(s[2 * i], c, -mc));
+        const float p1 = ex2_approx(fmaf(s[2 * i + 1], c, -mc));
+        pk[i] = pack_bf16x2(p0, p1);
+        ps[i & 7] += p0 + p1;
+      }
+      l_sum += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
+      if (j >= 1 && !mbar_wait(pv_done, (uint32_t)(j - 1) & 1u, status)) { ok = false; break; }
+      tc_fence_after();
+      if (__any_sync(0xffffffffu, rescale)) {
+#pragma unroll 1
+        for (int q = 0; q < 4; ++q) {
+          uint32_t o[32];
+          tmem_ld32(tmem_o + lane_off + q * 32, o);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          tmem_st32(tmem_o + lane_off + q * 32, o);
+        }
+        tmem_st_wait();
+      }
+      tmem_st32(tmem_p + lane_off, pk);
+      tmem_st32(tmem_p + lane_off + 32, pk + 32);
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(p_full);
+    }
+    if (ok && mbar_wait(pv_done, (uint32_t)(nt - 1) & 1u, status)) {
+      tc_fence_after();
+      const float inv_l = 1.f / l_sum;
+      constexpr int kStride = 272;  // 256 bytes of bf16 + 16 padding
+      uint8_t* st_row = smem + L::kKV + row * kStride;
+#pragma unroll 1
+      for (int q = 0; q < 4; ++q) {
+        uint32_t o[32];
+        tmem_ld32(tmem_o + lane_off + q * 32, o);
+        tmem_ld_wait();
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          reinterpret_cast<uint4*>(st_row + q * 64)[v] = make_uint4(
+              pack_bf16x2(__uint_as_float(o[8 * v + 0]) * inv_l, __uint_as_float(o[8 * v + 1]) * inv_l),
+              pack_bf16x2(__uint_as_float(o[8 * v + 2]) * inv_l, __uint_as_float(o[8 * v + 3]) * inv_l),
+              pack_bf16x2(__uint_as_float(o[8 * v + 4]) * inv_l, __uint_as_float(o[8 * v + 5]) * inv_l),
+              pack_bf16x2(__uint_as_float(o[8 * v + 6]) * inv_l, __uint_as_float(o[8 * v + 7]) * inv_l));
+        }
+      }
+      __syncwarp();
+      for (int rr = 0; rr < 32; rr += 2) {   // two rows per pass, 16 lanes x 16 bytes each
+        const int trow = sub * 32 + rr + (lane >> 4);
+        const int q = m0 + trow;
+        if (q < args.n_q) {
+          __nv_bfloat16* o = args.out + (((int64_t)z * args.n_q + q) * args.n_heads + h) * 128;
+          reinterpret_cast<uint4*>(o)[lane & 15] =
+              reinterpret_cast<const uint4*>(smem + L::kKV + trow * kStride)[lane & 15];
+        }
+      }
+    }
+    tc_fence_before();
+  }
+
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace mla

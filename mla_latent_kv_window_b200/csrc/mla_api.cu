@@ -22,6 +22,7 @@
 #include "../../include/mla.h"
 #include "gemm_tc.cuh"
 #include "window_attn.cuh"
+#include "dense_attn.cuh"
 
 namespace {
 
@@ -322,6 +323,41 @@ mla_status noalloc_scratch(void** out) {
 }
 
 size_t align256(size_t n) { return (n + 255) & ~size_t(255); }
+
+}  // namespace
+
+// ------------------------------------------------------------------------------ dense baseline
+// Status word of the stateless dense-attention entry point, one per device.
+static __device__ int g_dense_status;
+
+namespace {
+
+constexpr int kDenseStages = 3;
+std::mutex g_dense_mu;
+int* g_dense_status_ptr[64] = {};
+
+mla_status dense_status_word(int** out) {
+  int dev = 0;
+  MLA_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return fail(MLA_ERR_UNSUPPORTED, "device index %d too large", dev);
+  std::lock_guard<std::mutex> lock(g_dense_mu);
+  if (!g_dense_status_ptr[dev]) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_dense_status);
+    if (e != cudaSuccess || p == nullptr)
+      return fail(MLA_ERR_CUDA, "cudaGetSymbolAddress of the dense status word failed: %s",
+                  cudaGetErrorString(e));
+    const cudaError_t e2 =
+        cudaFuncSetAttribute(mla::dense_attn_kernel<kDenseStages>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             mla::DenseSmem<kDenseStages>::kBytes);
+    if (e2 != cudaSuccess)
+      return fail(MLA_ERR_CUDA, "cudaFuncSetAttribute failed: %s", cudaGetErrorString(e2));
+    g_dense_status_ptr[dev] = static_cast<int*>(p);
+  }
+  *out = g_dense_status_ptr[dev];
+  return MLA_OK;
+}
 
 }  // namespace
 
@@ -747,6 +783,58 @@ mla_status mla_window_attention_noalloc(mla_cache* c, const void* x_chunk, int32
     }
     if ((s = check_launch("no-alloc output projection")) != MLA_OK) return s;
   }
+  return MLA_OK;
+}
+
+mla_status mla_dense_attention(const void* q, const void* k, const void* v, void* out,
+                               int32_t batch, int32_t n_q, int32_t n_kv, int32_t n_heads,
+                               int32_t d_head, float softmax_scale, void* stream) {
+  if (!q || !k || !v || !out) return fail(MLA_ERR_INVALID_ARGUMENT, "NULL argument");
+  if (batch < 1 || n_q < 1 || n_kv < 1 || n_heads < 1)
+    return fail(MLA_ERR_INVALID_ARGUMENT, "batch, n_q, n_kv and n_heads must be >= 1");
+  if (d_head != 128) return fail(MLA_ERR_UNSUPPORTED, "the dense kernel is built for d_head = 128");
+  if (!(softmax_scale >= 0.f) || !std::isfinite(softmax_scale))
+    return fail(MLA_ERR_INVALID_ARGUMENT, "softmax_scale must be finite and >= 0");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
+    return fail(MLA_ERR_INVALID_ARGUMENT, "q, k, v and out must be 16-byte aligned");
+  if (batch > 65535 || n_heads > 65535 || (int64_t)n_q * n_heads * 128 > ((int64_t)1 << 40))
+    return fail(MLA_ERR_UNSUPPORTED, "problem too large for one launch");
+  int* status = nullptr;
+  mla_status s = dense_status_word(&status);
+  if (s != MLA_OK) return s;
+  const uint64_t row = (uint64_t)n_heads * 128;
+  CUtensorMap mq, mk, mv;
+  if ((s = make_map(&mq, q, row, n_q, batch, row * 2, row * n_q * 2, 64, 128,
+                    CU_TENSOR_MAP_SWIZZLE_128B)) != MLA_OK)
+    return s;
+  if ((s = make_map(&mk, k, row, n_kv, batch, row * 2, row * n_kv * 2, 64, 128,
+                    CU_TENSOR_MAP_SWIZZLE_128B)) != MLA_OK)
+    return s;
+  if ((s = make_map(&mv, v, row, n_kv, batch, row * 2, row * n_kv * 2, 64, 128,
+                    CU_TENSOR_MAP_SWIZZLE_128B)) != MLA_OK)
+    return s;
+  mla::DenseArgs a{};
+  a.n_q = n_q;
+  a.n_kv = n_kv;
+  a.n_heads = n_heads;
+  const float scale = softmax_scale > 0.f ? softmax_scale : (float)(1.0 / std::sqrt(128.0));
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.out = static_cast<__nv_bfloat16*>(out);
+  dim3 grid((unsigned)((n_q + 127) / 128), (unsigned)n_heads, (unsigned)batch);
+  mla::dense_attn_kernel<kDenseStages>
+      <<<grid, mla::kDenseThreads, mla::DenseSmem<kDenseStages>::kBytes,
+         reinterpret_cast<cudaStream_t>(stream)>>>(mq, mk, mv, a, status);
+  return check_launch("dense attention");
+}
+
+mla_status mla_dense_sync(void* stream) {
+  int* status = nullptr;
+  mla_status s = dense_status_word(&status);
+  if (s != MLA_OK) return s;
+  MLA_CUDA(cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)));
+  int word = 0;
+  MLA_CUDA(cudaMemcpy(&word, status, sizeof(int), cudaMemcpyDeviceToHost));
+  if (word != 0) return fail((mla_status)word, "the dense kernel recorded device status %d", word);
   return MLA_OK;
 }
 
