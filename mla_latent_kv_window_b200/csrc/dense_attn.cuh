@@ -175,6 +175,8 @@ __global__ void __launch_bounds__(kDenseThreads, 1)
       for (int q = 0; q < 4; ++q)
         tmem_ld32(tmem + lane_off + sb * 128 + q * 32, reinterpret_cast<uint32_t*>(s) + q * 32);
       tmem_ld_wait();
+#pragma unroll
+      for (int q = 0; q < 4; ++q) tmem_regs_ready(reinterpret_cast<uint32_t*>(s) + q * 32);
       tc_fence_before();
       mbar_arrive(&s_free[sb]);
       const int valid = n_kv - j * 128;
@@ -219,6 +221,7 @@ __global__ void __launch_bounds__(kDenseThreads, 1)
           uint32_t o[32];
           tmem_ld32(tmem_o + lane_off + q * 32, o);
           tmem_ld_wait();
+          tmem_regs_ready(o);
 #pragma unroll
           for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
           tmem_st32(tmem_o + lane_off + q * 32, o);
@@ -241,6 +244,7 @@ __global__ void __launch_bounds__(kDenseThreads, 1)
         uint32_t o[32];
         tmem_ld32(tmem_o + lane_off + q * 32, o);
         tmem_ld_wait();
+        tmem_regs_ready(o);
 #pragma unroll
         for (int v = 0; v < 4; ++v) {
           reinterpret_cast<uint4*>(st_row + q * 64)[v] = make_uint4(

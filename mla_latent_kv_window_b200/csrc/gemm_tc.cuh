@@ -3,17 +3,26 @@
 //   D[m, n] = sum_k A[z][m, k] * B[n, k]    (A: [batch][M][K], B: [N][K], K-major, both bf16 or
 //                                            both fp16, fp32 accumulation)
 //
-// One CTA computes a 128 x BN tile with fp32 accumulation in tensor memory:
+// Persistent: one CTA per SM walks the tiles t = blockIdx.x, blockIdx.x + gridDim.x, ... of a
+// (row tile, column block, batch) grid.  Each 128 x BN tile accumulates in fp32 tensor memory:
 //   warp 0      TMA producer of A k-blocks (64 wide) into an A_STAGES-deep ring
 //   warp 6      TMA producer of B k-blocks into a B_STAGES-deep ring
 //   warp 1      TMEM allocator + single-thread tcgen05.mma issuer (M=128, N=BN, K=16 steps)
-//   warps 2..5  epilogue: tcgen05.ld of the accumulator (one row per thread), fused row
-//               transform, staged through shared memory for coalesced 16-byte row stores.
-// A (hidden states, streamed once from HBM) and B (weights, shared by every CTA and
-// L2-resident) have separate rings so that A can run far ahead of the short-latency B loads;
-// each CTA starts its k-loop at a rotated block so the CTAs do not all hit the same weight
-// block at once.
-//
+//   warps 2..5  epilogue: tcgen05.ld of the accumulator (one row per thread; the next 32-column
+//               chunk is loaded while the current one is converted), fused row transform into
+//               a padded shared-memory staging row, then one bulk async copy per contiguous
+//               destination segment of the row (c_kv 384 B + k_rope 64 B, Qp 448 B, or the
+//               output row), issued by the owning thread.
+// The rings run continuously across tile boundaries.  With M_SUB = 1 the accumulator is
+// double-buffered in TMEM (2 x 256 columns), so the epilogue of tile i overlaps the MMAs of
+// tile i+1.  With M_SUB = 2 a tile is 256 rows: two M=128 accumulators (TMEM columns [0,256)
+// and [256,512)) share every weight k-block, halving the weight bytes per row - the right
+// trade when there are more tiles than SMs and the per-SM load path is the limit; the loads
+// of tile i+1 still stream during the epilogue of tile i.
+// A (activations, streamed once from HBM) and B (weights, shared by every CTA and L2-resident)
+// have separate rings so that A can run ahead of the short-latency B loads; each tile starts
+// its k-loop at a rotated block so concurrent CTAs do not all hit the same weight block.
+
 // Epilogues (kEpi):
 //   kEpiStore   bf16 store of the tile into out[z][m][n]                (output projection)
 //   kEpiLatent  columns 0..191 -> c_kv, 192..223 -> RoPE3D -> k_rope, written as fp16 to ring
@@ -36,8 +45,11 @@ constexpr int kEpiLatent = 1;
 constexpr int kGemmThreads = 224;
 
 // Rotary bands of the d_rope = 32 positional channels: pair p rotates by pos[axis[p]] * freq[p].
+// Each frequency is carried as an unevaluated float sum hi + lo (|lo| <= ulp(hi) / 2), so that
+// pos * freq is formed to about 2^-45 relative in fp32 arithmetic.
 struct RopeBands {
-  double freq[16];
+  float freq_hi[16];
+  float freq_lo[16];
   int axis[16];  // 0 = t, 1 = h, 2 = w
 };
 
@@ -64,41 +76,63 @@ struct EpiArgs {
   RopeBands rope;
 };
 
-template <int BN, int A_STAGES, int B_STAGES>
+template <int BN, int A_STAGES, int B_STAGES, int M_SUB = 1>
 struct GemmSmem {
-  static constexpr int kABytes = 128 * 64 * 2;
+  static constexpr int kABytes = M_SUB * 128 * 64 * 2;
   static constexpr int kBBytes = BN * 64 * 2;
   static constexpr int kBOffset = A_STAGES * kABytes;
-  static constexpr int kBarOffset = kBOffset + B_STAGES * kBBytes;
-  static constexpr int kBytes = kBarOffset + 512 + 1024;  // barriers + alignment slack
+  static constexpr int kStageStride = BN * 2 + 16;          // padded staging row (no bank conflicts)
+  static constexpr int kStagingOffset = kBOffset + B_STAGES * kBBytes;
+  static constexpr int kBarOffset = kStagingOffset + 128 * kStageStride;
+  static constexpr int kBytes = kBarOffset + 512 + 1024;    // barriers + alignment slack
   static_assert(kABytes % 1024 == 0 && kBBytes % 1024 == 0, "stage atoms must stay 1 KB aligned");
-  static_assert(kBarOffset >= 128 * (BN * 2 + 16), "staging must fit in the rings");
   static_assert(kBytes <= 232448, "GEMM tile does not fit in shared memory");
 };
 
+// Tile grid of one GEMM launch: row tiles (of 128 * M_SUB rows) x column blocks of BN x batch.
+struct GemmTiles {
+  int32_t m_tiles, n_blocks, batch;
+  __host__ __device__ int32_t count() const { return m_tiles * n_blocks * batch; }
+};
+
+// Rotate the 16 (re, im) pairs of v by pos * freq.  The angle is formed as p + e with
+// p = fl(pos * hi), e = (pos * hi - p) + pos * lo (exact product error by FMA), then reduced to
+// [-pi, pi] by Cody-Waite reduction with 2 pi split into two floats (accurate for integer
+// positions below 2^24), and evaluated with the hardware sine/cosine.
 __device__ __forceinline__ void rope_rotate32(float* v, int64_t t, int h, int w,
                                               const RopeBands& rb) {
+  constexpr float kInv2Pi = 0.15915494309189535f;
+  constexpr float kTwoPiHi = 6.28318548202514648f;       // fl(2 pi)
+  constexpr float kTwoPiLo = -1.7484556000744e-07f;      // 2 pi - fl(2 pi)
 #pragma unroll
   for (int p = 0; p < 16; ++p) {
     const int ax = rb.axis[p];
-    const double pos = ax == 0 ? (double)t : (ax == 1 ? (double)h : (double)w);
-    double ang = pos * rb.freq[p];
-    ang -= 6.283185307179586 * rint(ang * 0.15915494309189535);  // reduce to [-pi, pi]
-    float s, c;
-    __sincosf((float)ang, &s, &c);
+    const float pos = ax == 0 ? (float)t : (ax == 1 ? (float)h : (float)w);
+    const float hi = rb.freq_hi[p];
+    const float prod = pos * hi;
+    const float err = fmaf(pos, hi, -prod) + pos * rb.freq_lo[p];
+    const float k = rintf(prod * kInv2Pi);
+    float r = fmaf(-k, kTwoPiHi, prod);
+    r = fmaf(-k, kTwoPiLo, r) + err;
+    float sn, cs;
+    __sincosf(r, &sn, &cs);
     const float a = v[2 * p], b = v[2 * p + 1];
-    v[2 * p] = a * c - b * s;
-    v[2 * p + 1] = a * s + b * c;
+    v[2 * p] = a * cs - b * sn;
+    v[2 * p + 1] = a * sn + b * cs;
   }
 }
 
-template <int BN, int A_STAGES, int B_STAGES, int kEpi, bool kF16In>
+template <int BN, int A_STAGES, int B_STAGES, int kEpi, bool kF16In, int M_SUB>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
                    const __grid_constant__ CUtensorMap map_b, int32_t M, int32_t K,
-                   int32_t b_row0, EpiArgs ep, int* status) {
-  using L = GemmSmem<BN, A_STAGES, B_STAGES>;
+                   int32_t b_row0, GemmTiles tiles, EpiArgs ep, int* status) {
+  using L = GemmSmem<BN, A_STAGES, B_STAGES, M_SUB>;
+  static_assert(M_SUB == 1 || M_SUB == 2, "tiles are 128 or 256 rows");
+  constexpr int kAccBufs = M_SUB == 1 ? 2 : 1;   // accumulator buffers in 512 TMEM columns
+  constexpr int kTileRows = 128 * M_SUB;
   static_assert(kEpi != kEpiLatent || BN == 224, "the latent epilogue owns 192 + 32 columns");
+  static_assert(BN <= 256, "one accumulator buffer holds at most 256 columns");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -106,17 +140,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint64_t* a_empty = a_full + A_STAGES;
   uint64_t* b_full = a_empty + A_STAGES;
   uint64_t* b_empty = b_full + B_STAGES;
-  uint64_t* acc_full = b_empty + B_STAGES;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(acc_full + 1);
+  uint64_t* acc_full = b_empty + B_STAGES;     // [2]
+  uint64_t* acc_empty = acc_full + 2;          // [2]
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(acc_empty + 2);
 
   const uint32_t warp = warp_id();
   const uint32_t lane = lane_id();
-  const int m0 = blockIdx.x * 128;
-  const int y = blockIdx.y;
-  const int z = blockIdx.z;
   const int num_kb = K / 64;
-  const int kb_rot = (int)((blockIdx.x * 7u + blockIdx.y * 3u + blockIdx.z) % (unsigned)num_kb);
-  constexpr uint32_t kTmemCols = BN <= 128 ? 128 : 256;
+  const int n_tiles = tiles.count();
+  const int my_tiles = n_tiles > (int)blockIdx.x
+                           ? (n_tiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < A_STAGES; ++s) {
@@ -127,19 +160,31 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       mbar_init(&b_full[s], 1);
       mbar_init(&b_empty[s], 1);
     }
-    mbar_init(acc_full, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&acc_full[s], 1);
+      mbar_init(&acc_empty[s], 128);
+    }
     fence_mbar_init();
     tma_prefetch(&map_a);
     tma_prefetch(&map_b);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_holder, kTmemCols);
+    tmem_alloc(tmem_holder, 512);
     tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
+
+  // Tile t -> (row tile, column block, batch); consecutive tiles share the column block.
+  auto tile_coords = [&](int t, int& m0, int& y, int& z) {
+    const int per_batch = tiles.m_tiles * tiles.n_blocks;
+    z = t / per_batch;
+    const int r = t - z * per_batch;
+    y = r / tiles.m_tiles;
+    m0 = (r - y * tiles.m_tiles) * kTileRows;
+  };
 
   if (warp == 0 || warp == 6) {
     // ------------------------------------------------------------------ TMA producers
@@ -150,143 +195,169 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint64_t* empty = is_a ? a_empty : b_empty;
       const uint32_t bytes = is_a ? L::kABytes : L::kBBytes;
       const uint64_t policy = is_a ? l2_policy_evict_first() : l2_policy_evict_last();
-      int issued = 0;
-      for (int kb = 0; kb < num_kb; ++kb) {
-        const int s = kb % stages;
-        if (!mbar_wait(&empty[s], ((uint32_t)(kb / stages) & 1u) ^ 1u, status)) break;
-        const int kx = ((kb + kb_rot) % num_kb) * 64;
-        mbar_arrive_expect_tx(&full[s], bytes);
-        if (is_a)
-          tma_load_3d_hint(smem + s * L::kABytes, &map_a, &full[s], kx, m0, z, policy);
-        else
-          tma_load_3d_hint(smem + L::kBOffset + s * L::kBBytes, &map_b, &full[s], kx,
-                           b_row0 + y * BN, 0, policy);
-        issued = kb + 1;
+      int g = 0;  // k-blocks issued so far (continuous across tiles)
+      bool ok = true;
+      for (int i = 0; i < my_tiles && ok; ++i) {
+        int m0, y, z;
+        tile_coords(blockIdx.x + i * gridDim.x, m0, y, z);
+        const int rot = (int)((blockIdx.x + i * gridDim.x) * 7u % (unsigned)num_kb);
+        for (int kb = 0; kb < num_kb; ++kb, ++g) {
+          const int s = g % stages;
+          if (!mbar_wait(&empty[s], ((uint32_t)(g / stages) & 1u) ^ 1u, status)) { ok = false; break; }
+          const int kx = ((kb + rot) % num_kb) * 64;
+          mbar_arrive_expect_tx(&full[s], bytes);
+          if (is_a)
+            tma_load_3d_hint(smem + s * L::kABytes, &map_a, &full[s], kx, m0, z, policy);
+          else
+            tma_load_3d_hint(smem + L::kBOffset + s * L::kBBytes, &map_b, &full[s], kx,
+                             b_row0 + y * BN, 0, policy);
+        }
       }
       // Drain: never leave the CTA with a copy still landing in its shared memory.
-      for (int kb = issued > stages ? issued - stages : 0; kb < issued; ++kb)
-        mbar_wait(&full[kb % stages], (uint32_t)(kb / stages) & 1u, status);
+      for (int q = g > stages ? g - stages : 0; q < g; ++q)
+        mbar_wait(&full[q % stages], (uint32_t)(q / stages) & 1u, status);
     }
   } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_f32acc(128, BN, false, kF16In);
-      for (int kb = 0; kb < num_kb; ++kb) {
-        const int sa = kb % A_STAGES;
-        const int sb = kb % B_STAGES;
-        if (!mbar_wait(&a_full[sa], (uint32_t)(kb / A_STAGES) & 1u, status)) break;
-        if (!mbar_wait(&b_full[sb], (uint32_t)(kb / B_STAGES) & 1u, status)) break;
+      int g = 0;
+      bool ok = true;
+      for (int i = 0; i < my_tiles && ok; ++i) {
+        const int buf = i % kAccBufs;
+        if (!mbar_wait(&acc_empty[buf], ((uint32_t)(i / kAccBufs) & 1u) ^ 1u, status)) break;
         tc_fence_after();
-        const uint32_t a_addr = smem_u32(smem + sa * L::kABytes);
-        const uint32_t b_addr = smem_u32(smem + L::kBOffset + sb * L::kBBytes);
+        const uint32_t acc = tmem + buf * 256;
+        for (int kb = 0; kb < num_kb; ++kb, ++g) {
+          const int sa = g % A_STAGES;
+          const int sb = g % B_STAGES;
+          if (!mbar_wait(&a_full[sa], (uint32_t)(g / A_STAGES) & 1u, status) ||
+              !mbar_wait(&b_full[sb], (uint32_t)(g / B_STAGES) & 1u, status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(smem + sa * L::kABytes);
+          const uint32_t b_addr = smem_u32(smem + L::kBOffset + sb * L::kBBytes);
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const uint64_t da = smem_desc(a_addr + k * 32, 16, 1024, kSwizzle128B);
-          const uint64_t db = smem_desc(b_addr + k * 32, 16, 1024, kSwizzle128B);
-          umma_ss(tmem, da, db, idesc, (kb | k) != 0 ? 1u : 0u);
+          for (int k = 0; k < 4; ++k) {
+            const uint64_t db = smem_desc(b_addr + k * 32, 16, 1024, kSwizzle128B);
+#pragma unroll
+            for (int sub = 0; sub < M_SUB; ++sub) {   // rows 128*sub.. of the A box
+              const uint64_t da = smem_desc(a_addr + sub * 16384 + k * 32, 16, 1024, kSwizzle128B);
+              umma_ss(acc + sub * 256, da, db, idesc, (kb | k) != 0 ? 1u : 0u);
+            }
+          }
+          tc_commit(&a_empty[sa]);
+          tc_commit(&b_empty[sb]);
         }
-        tc_commit(&a_empty[sa]);
-        tc_commit(&b_empty[sb]);
+        tc_commit(&acc_full[buf]);
       }
-      tc_commit(acc_full);
     }
   } else {
     // ------------------------------------------------------------------ epilogue warps
-    const uint32_t sub = warp & 3u;            // TMEM lane quarter this warp may access
-    const int row = sub * 32 + lane;           // tile row owned by this thread
-    const int m = m0 + row;
-    const bool ok = mbar_wait(acc_full, 0, status);
-    tc_fence_after();
-    constexpr int kStageStride = BN * 2 + 16;  // bytes per staged row (bank-conflict padding)
-    uint8_t* stage_row = smem + row * kStageStride;
-    const uint32_t tbase = tmem + ((sub * 32u) << 16);
-
-    // Row geometry for the latent / query epilogue.
-    bool latent = false;
-    int64_t t = 0;
-    int hh = 0, ww = 0;
-    if constexpr (kEpi == kEpiLatent) {
-      latent = y >= ep.latent_y;
-      const int F = ep.tokens_per_frame;
-      t = ep.t0 + m / F;
-      const int k = m % F;
-      hh = k / ep.frame_w;
-      ww = k % ep.frame_w;
-    }
-    if (ok) {
+    const uint32_t sub_q = warp & 3u;          // TMEM lane quarter this warp may access
+    const int row = sub_q * 32 + lane;         // row of each 128-row sub-tile owned by this thread
+    uint8_t* stage_row = smem + L::kStagingOffset + row * L::kStageStride;
+    for (int i = 0; i < my_tiles; ++i) {
+      const int buf = i % kAccBufs;
+      int m0t, y, z;
+      tile_coords(blockIdx.x + i * gridDim.x, m0t, y, z);
+      if (!mbar_wait_warp_sleepy(&acc_full[buf], (uint32_t)(i / kAccBufs) & 1u, status)) break;
+      tc_fence_after();
 #pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld32(tbase + c * 32, r);
-        tmem_ld_wait();
-        float v[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+      for (int sub = 0; sub < M_SUB; ++sub) {
+        const int m = m0t + sub * 128 + row;
+        const bool valid = m < M;
+        const uint32_t tbase = tmem + (buf + sub) * 256 + ((sub_q * 32u) << 16);
+
+        // This thread's destination row(s), computed once per tile.
+        void* dst_main = nullptr;    // columns [0, 192) (latent), [0, 224) (query), [0, BN) (store)
+        void* dst_rope = nullptr;    // latent rows: the k_rope plane (columns [192, 224))
+        bool latent = false;
+        int64_t t = 0;
+        int hh = 0, ww = 0;
         if constexpr (kEpi == kEpiLatent) {
-          if (c == 6) rope_rotate32(v, t, hh, ww, ep.rope);   // columns 192..223
-          if (!latent) {
-#pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] *= ep.q_scale;
-          }
-        }
-        uint4* dst = reinterpret_cast<uint4*>(stage_row + c * 64);
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          if constexpr (kEpi == kEpiLatent) {
-            dst[q] = make_uint4(pack_f16x2(v[8 * q + 0], v[8 * q + 1]),
-                                pack_f16x2(v[8 * q + 2], v[8 * q + 3]),
-                                pack_f16x2(v[8 * q + 4], v[8 * q + 5]),
-                                pack_f16x2(v[8 * q + 6], v[8 * q + 7]));
-          } else {
-            dst[q] = make_uint4(pack_bf16x2(v[8 * q + 0], v[8 * q + 1]),
-                                pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
-                                pack_bf16x2(v[8 * q + 4], v[8 * q + 5]),
-                                pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
-          }
-        }
-      }
-    }
-    tc_fence_before();
-    __syncwarp();
-    // Coalesced copy-out: the warp walks its own 32 rows, one 16-byte chunk per lane.
-    if (ok) {
-      constexpr int kChunks = BN / 8;  // 16-byte chunks per row
-      for (int rr = 0; rr < 32; ++rr) {
-        const int trow = sub * 32 + rr;
-        const int gm = m0 + trow;
-        if (gm >= M) break;
-        const uint4* src = reinterpret_cast<const uint4*>(smem + trow * kStageStride);
-        if constexpr (kEpi == kEpiStore) {
-          __nv_bfloat16* o = ep.out + z * ep.out_batch_stride + (int64_t)gm * ep.ld_out + y * BN;
-          for (int q = lane; q < kChunks; q += 32) reinterpret_cast<uint4*>(o)[q] = src[q];
-        } else {
+          latent = y >= ep.latent_y;
+          const int F = ep.tokens_per_frame;
+          const int fi = m / F;               // frame within this call
+          const int k = m - fi * F;
+          t = ep.t0 + fi;
+          hh = k / ep.frame_w;
+          ww = k - hh * ep.frame_w;
           if (latent) {
-            int64_t dst_row;
-            if (ep.ring_mode) {
-              const int F = ep.tokens_per_frame;
-              const int64_t f = ep.t0 + gm / F;
-              dst_row = (f % ep.window_frames) * F + gm % F;
-            } else {
-              dst_row = ep.base_row + gm;
+            const int64_t dst_row =
+                (ep.ring_mode ? (int64_t)(t % ep.window_frames) * F + k : ep.base_row + m) +
+                (int64_t)z * ep.rows_per_stream;
+            dst_main = ep.ckv + dst_row * 192;
+            dst_rope = ep.krope + dst_row * 32;
+          } else {
+            const int64_t qrow = (int64_t)z * ep.qp_rows_per_stream + (int64_t)m * ep.n_heads + y;
+            dst_main = ep.qp + qrow * 224;
+          }
+        } else {
+          dst_main = ep.out + z * ep.out_batch_stride + (int64_t)m * ep.ld_out + y * BN;
+        }
+
+        // The staging row is free once this thread's previous bulk copies have read it.
+        bulk_wait_read_all();
+        uint32_t r[2][32];
+        tmem_ld32(tbase, r[0]);
+#pragma unroll
+        for (int c = 0; c < BN / 32; ++c) {
+          uint32_t* cur = r[c & 1];
+          tmem_ld_wait();
+          tmem_regs_ready(cur);
+          if (c + 1 < BN / 32) tmem_ld32(tbase + (c + 1) * 32, r[(c + 1) & 1]);
+          float v[32];
+#pragma unroll
+          for (int q = 0; q < 32; ++q) v[q] = __uint_as_float(cur[q]);
+          if constexpr (kEpi == kEpiLatent) {
+            if (c == 6) rope_rotate32(v, t, hh, ww, ep.rope);   // columns 192..223
+            if (!latent) {
+#pragma unroll
+              for (int q = 0; q < 32; ++q) v[q] *= ep.q_scale;
             }
-            dst_row += z * ep.rows_per_stream;
-            if (lane < 24) {
-              reinterpret_cast<uint4*>(ep.ckv + dst_row * 192)[lane] = src[lane];
-            } else if (lane < 28) {
-              reinterpret_cast<uint4*>(ep.krope + dst_row * 32)[lane - 24] = src[lane];
+          }
+          uint4* st4 = reinterpret_cast<uint4*>(stage_row + c * 64);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            if constexpr (kEpi == kEpiLatent)
+              st4[q] = make_uint4(pack_f16x2(v[8 * q + 0], v[8 * q + 1]), pack_f16x2(v[8 * q + 2], v[8 * q + 3]),
+                                  pack_f16x2(v[8 * q + 4], v[8 * q + 5]), pack_f16x2(v[8 * q + 6], v[8 * q + 7]));
+            else
+              st4[q] = make_uint4(pack_bf16x2(v[8 * q + 0], v[8 * q + 1]), pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
+                                  pack_bf16x2(v[8 * q + 4], v[8 * q + 5]), pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
+          }
+        }
+        if (sub == M_SUB - 1) {
+          // Every accumulator of this tile has been read: the buffer is free for the MMAs.
+          tc_fence_before();
+          mbar_arrive(&acc_empty[buf]);
+        }
+        if (valid) {
+          fence_proxy_async_smem();   // staging writes -> visible to the bulk-copy engine
+          if constexpr (kEpi == kEpiLatent) {
+            if (latent) {
+              bulk_store(dst_main, stage_row, 384);
+              bulk_store(dst_rope, stage_row + 384, 64);
+            } else {
+              bulk_store(dst_main, stage_row, 448);
             }
           } else {
-            const int64_t qrow = z * ep.qp_rows_per_stream + (int64_t)gm * ep.n_heads + y;
-            if (lane < 28) reinterpret_cast<uint4*>(ep.qp + qrow * 224)[lane] = src[lane];
+            bulk_store(dst_main, stage_row, BN * 2);
           }
+          bulk_commit();
         }
       }
     }
+    bulk_wait_all();
   }
 
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, kTmemCols);
+    tmem_dealloc(tmem, 512);
   }
 }
 

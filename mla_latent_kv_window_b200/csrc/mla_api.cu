@@ -33,13 +33,16 @@ constexpr int kLatent = 192;
 constexpr int kRope = 32;
 constexpr int kQK = kLatent + kRope;  // 224
 
-// Pipeline depths of the launched kernel variants (A = activations, B = weights).
-constexpr int kProjAStages = 8;     // 8 x 16 KB of hidden states in flight per SM (HBM latency)
+// Pipeline depths of the launched kernel variants (A = activations, B = weights); each GEMM
+// CTA runs alone on its SM.  The weight ring is deep too: its L2 latency sets the k-block rate
+// when only a few CTAs run.
+constexpr int kProjAStages = 5;     // 5 x 16 KB of hidden states in flight per SM (HBM latency)
 constexpr int kProjBStages = 3;     // 3 x 28 KB of L2-resident weights
-constexpr int kOutAStages = 6;
-constexpr int kOutBStages = 3;
-constexpr int kAttnStages = 3;      // 3 KV tiles in flight (P kept in tensor memory)
-constexpr bool kAttnPInTmem = true;
+constexpr int kProjWideAStages = 3; // 256-row tiles: 3 x 32 KB of hidden states
+constexpr int kProjWideBStages = 2;
+constexpr int kOutAStages = 5;
+constexpr int kOutBStages = 2;
+constexpr int kAttnStages = 4;      // 4 key tiles in flight (Q and P live in tensor memory)
 
 thread_local std::string g_last_error;
 
@@ -166,6 +169,26 @@ mla_status set_smem(K kernel, int bytes) {
   return MLA_OK;
 }
 
+mla_status check_launch(const char* what) {
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(MLA_ERR_CUDA, "%s launch failed: %s", what, cudaGetErrorString(e));
+  return MLA_OK;
+}
+
+// Persistent GEMM launch: one CTA per SM at most, each walking its share of the tiles.
+template <int BN, int SA, int SB, int EPI, bool F16, int M_SUB = 1>
+mla_status launch_gemm(const CUtensorMap& ma, const CUtensorMap& mb, int M, int K, int b_row0,
+                       mla::GemmTiles tiles, const EpiArgs& ep, int* status, int num_sms,
+                       cudaStream_t st, const char* what) {
+  const int n = tiles.count();
+  if (n <= 0) return MLA_OK;
+  const int grid = n < num_sms ? n : num_sms;
+  mla::tc_gemm_kernel<BN, SA, SB, EPI, F16, M_SUB>
+      <<<grid, mla::kGemmThreads, mla::GemmSmem<BN, SA, SB, M_SUB>::kBytes, st>>>(
+          ma, mb, M, K, b_row0, tiles, ep, status);
+  return check_launch(what);
+}
+
 }  // namespace
 
 // ------------------------------------------------------------------------------ the cache
@@ -178,6 +201,7 @@ struct mla_cache {
   float softmax_scale = 0.f;
   RopeBands rope{};
   int device = 0;
+  int num_sms = 148;
 
   __half* ckv = nullptr;           // fp16 latent planes (ring + chunk tail)
   __half* krope = nullptr;
@@ -220,8 +244,8 @@ struct ProfScope {
   int kind;
   cudaStream_t s;
   cudaEvent_t a = nullptr;
-  ProfScope(mla_cache* c_, int k, cudaStream_t s_) : c(c_), kind(k), s(s_) {
-    if (c->profiling && (a = take_event(c)) != nullptr) cudaEventRecord(a, s);
+  ProfScope(mla_cache* c_, int k, cudaStream_t s_, bool enabled = true) : c(c_), kind(k), s(s_) {
+    if (enabled && c->profiling && (a = take_event(c)) != nullptr) cudaEventRecord(a, s);
   }
   ~ProfScope() {
     if (!a) return;
@@ -235,40 +259,42 @@ struct ProfScope {
   }
 };
 
-mla_status check_launch(const char* what) {
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return fail(MLA_ERR_CUDA, "%s launch failed: %s", what, cudaGetErrorString(e));
-  return MLA_OK;
-}
-
+// Band frequencies base^(-2i/d_a), computed in double and carried as float hi + lo.
 RopeBands make_bands(const mla_config& cfg) {
   RopeBands rb{};
   int p = 0;
   const int dims[3] = {cfg.rope_t, cfg.rope_h, cfg.rope_w};
   for (int a = 0; a < 3; ++a)
     for (int i = 0; i < dims[a] / 2; ++i, ++p) {
+      const double f = std::pow(cfg.rope_base, -2.0 * i / dims[a]);
       rb.axis[p] = a;
-      rb.freq[p] = std::pow(cfg.rope_base, -2.0 * i / dims[a]);
+      rb.freq_hi[p] = (float)f;
+      rb.freq_lo[p] = (float)(f - (double)rb.freq_hi[p]);
     }
   return rb;
 }
 
-// Launch the latent/query projection GEMM over `rows` rows of x per stream.
+// Launch the latent/query projection GEMM over `rows` rows of x per stream.  Query rows go to
+// `qp` (rows_per_stream qp_rows); launches with more 128-row tiles than SMs use 256-row tiles so
+// each weight k-block serves twice as many rows.
 mla_status launch_latent_gemm(mla_cache* c, const void* x, int64_t rows, int64_t x_batch_rows,
                               int grid_y, int latent_y, int b_row0, int ring_mode, int64_t t0,
-                              int64_t base_row, cudaStream_t st) {
+                              int64_t base_row, cudaStream_t st, __half* qp = nullptr,
+                              int64_t qp_rows = 0) {
   const mla_config& cfg = c->cfg;
+  const int64_t tiles128 = (rows + 127) / 128;
+  const bool wide = tiles128 * grid_y * cfg.batch > c->num_sms;
   CUtensorMap map_x;
   mla_status s = make_map(&map_x, x, cfg.hidden, rows, cfg.batch, (uint64_t)cfg.hidden * 2,
-                          (uint64_t)x_batch_rows * cfg.hidden * 2, 64, 128,
+                          (uint64_t)x_batch_rows * cfg.hidden * 2, 64, wide ? 256 : 128,
                           CU_TENSOR_MAP_SWIZZLE_128B);
   if (s != MLA_OK) return s;
   EpiArgs ep{};
   ep.ckv = c->ckv;
   ep.krope = c->krope;
   ep.rows_per_stream = c->rows_per_stream;
-  ep.qp = c->qp;
-  ep.qp_rows_per_stream = c->max_q_tokens * cfg.n_heads;
+  ep.qp = qp ? qp : c->qp;
+  ep.qp_rows_per_stream = qp ? qp_rows : c->max_q_tokens * cfg.n_heads;
   ep.latent_y = latent_y;
   ep.n_heads = cfg.n_heads;
   ep.ring_mode = ring_mode;
@@ -279,12 +305,46 @@ mla_status launch_latent_gemm(mla_cache* c, const void* x, int64_t rows, int64_t
   ep.base_row = base_row;
   ep.q_scale = c->softmax_scale * 1.4426950408889634f;
   ep.rope = c->rope;
-  using Sm = mla::GemmSmem<kQK, kProjAStages, kProjBStages>;
-  dim3 grid((unsigned)((rows + 127) / 128), (unsigned)grid_y, (unsigned)cfg.batch);
-  mla::tc_gemm_kernel<kQK, kProjAStages, kProjBStages, mla::kEpiLatent, false>
-      <<<grid, mla::kGemmThreads, Sm::kBytes, st>>>(map_x, c->map_wqcat, (int)rows, cfg.hidden,
-                                                   b_row0, ep, c->status);
-  return check_launch("latent projection");
+  if (wide) {
+    const mla::GemmTiles tiles{(int32_t)((rows + 255) / 256), grid_y, cfg.batch};
+    return launch_gemm<kQK, kProjWideAStages, kProjWideBStages, mla::kEpiLatent, false, 2>(
+        map_x, c->map_wqcat, (int)rows, cfg.hidden, b_row0, tiles, ep, c->status, c->num_sms, st,
+        "latent projection");
+  }
+  const mla::GemmTiles tiles{(int32_t)tiles128, grid_y, cfg.batch};
+  return launch_gemm<kQK, kProjAStages, kProjBStages, mla::kEpiLatent, false, 1>(
+      map_x, c->map_wqcat, (int)rows, cfg.hidden, b_row0, tiles, ep, c->status, c->num_sms, st,
+      "latent projection");
+}
+
+// Window attention of R query rows per stream over keys [0, n_keys) of every stream's ring.
+mla_status launch_attention(mla_cache* c, const __half* qp, int64_t qp_batch_stride, int64_t R,
+                            int64_t n_keys, __half* o_lat, int64_t o_lat_batch_stride,
+                            cudaStream_t st, bool profile) {
+  const mla_config& cfg = c->cfg;
+  CUtensorMap mkc, mkr;
+  mla_status s;
+  if ((s = make_map(&mkc, c->ckv, kLatent, n_keys, cfg.batch, kLatent * 2,
+                    (uint64_t)c->rows_per_stream * kLatent * 2, 64, 128,
+                    CU_TENSOR_MAP_SWIZZLE_128B, true)) != MLA_OK)
+    return s;
+  if ((s = make_map(&mkr, c->krope, kRope, n_keys, cfg.batch, kRope * 2,
+                    (uint64_t)c->rows_per_stream * kRope * 2, 32, 128,
+                    CU_TENSOR_MAP_SWIZZLE_64B, true)) != MLA_OK)
+    return s;
+  mla::AttnArgs a{};
+  a.qp = qp;
+  a.qp_batch_stride = qp_batch_stride;
+  a.rows = (int32_t)R;
+  a.n_keys = (int32_t)n_keys;
+  a.o_lat = o_lat;
+  a.o_lat_batch_stride = o_lat_batch_stride;
+  using Sm = mla::AttnSmem<kAttnStages>;
+  dim3 grid((unsigned)((R + 127) / 128), (unsigned)cfg.batch);
+  ProfScope p(c, MLA_KERNEL_ATTENTION, st, profile);
+  mla::window_attn_kernel<kAttnStages><<<grid, mla::kAttnThreads, Sm::kBytes, st>>>(mkc, mkr, a,
+                                                                                   c->status);
+  return check_launch("window attention");
 }
 
 }  // namespace
@@ -484,6 +544,9 @@ mla_status mla_cache_create(const mla_config* cfg, const mla_weights* w, void* s
   c->rope = make_bands(*cfg);
   c->out_bn = cfg->hidden % 256 == 0 ? 256 : 128;
   cudaGetDevice(&c->device);
+  if (cudaDeviceGetAttribute(&c->num_sms, cudaDevAttrMultiProcessorCount, c->device) != cudaSuccess ||
+      c->num_sms <= 0)
+    c->num_sms = 148;
 
   auto cleanup = [&](mla_status r) {
     mla_cache_destroy(c);
@@ -538,17 +601,20 @@ mla_status mla_cache_create(const mla_config* cfg, const mla_weights* w, void* s
   static std::once_flag attr_once;
   static mla_status attr_status = MLA_OK;
   std::call_once(attr_once, [] {
-    mla_status r = set_smem(mla::tc_gemm_kernel<kQK, kProjAStages, kProjBStages, mla::kEpiLatent, false>,
-                            mla::GemmSmem<kQK, kProjAStages, kProjBStages>::kBytes);
+    mla_status r = set_smem(mla::tc_gemm_kernel<kQK, kProjAStages, kProjBStages, mla::kEpiLatent, false, 1>,
+                            mla::GemmSmem<kQK, kProjAStages, kProjBStages, 1>::kBytes);
     if (r == MLA_OK)
-      r = set_smem(mla::tc_gemm_kernel<256, kOutAStages, kOutBStages, mla::kEpiStore, true>,
+      r = set_smem(mla::tc_gemm_kernel<kQK, kProjWideAStages, kProjWideBStages, mla::kEpiLatent, false, 2>,
+                   mla::GemmSmem<kQK, kProjWideAStages, kProjWideBStages, 2>::kBytes);
+    if (r == MLA_OK)
+      r = set_smem(mla::tc_gemm_kernel<256, kOutAStages, kOutBStages, mla::kEpiStore, true, 1>,
                    mla::GemmSmem<256, kOutAStages, kOutBStages>::kBytes);
     if (r == MLA_OK)
-      r = set_smem(mla::tc_gemm_kernel<128, kOutAStages, kOutBStages, mla::kEpiStore, true>,
+      r = set_smem(mla::tc_gemm_kernel<128, kOutAStages, kOutBStages, mla::kEpiStore, true, 1>,
                    mla::GemmSmem<128, kOutAStages, kOutBStages>::kBytes);
     if (r == MLA_OK)
-      r = set_smem(mla::window_attn_kernel<kAttnStages, kAttnPInTmem>,
-                   mla::AttnSmem<kAttnStages, kAttnPInTmem>::kBytes);
+      r = set_smem(mla::window_attn_kernel<kAttnStages>,
+                   mla::AttnSmem<kAttnStages>::kBytes);
     attr_status = r;
   });
   if (attr_status != MLA_OK) return cleanup(attr_status);
@@ -610,32 +676,9 @@ mla_status mla_window_attention(mla_cache* c, const void* x_chunk, int32_t n_fra
   {
     const int64_t R = nq * cfg.n_heads;
     const uint64_t qp_rows = (uint64_t)c->max_q_tokens * cfg.n_heads;
-    CUtensorMap mqc, mqr, mkc, mkr;
-    if ((s = make_map(&mqc, c->qp, kQK, R, cfg.batch, kQK * 2, qp_rows * kQK * 2, 64, 128,
-                      CU_TENSOR_MAP_SWIZZLE_128B, true)) != MLA_OK)
+    if ((s = launch_attention(c, c->qp, (int64_t)qp_rows * kQK, R, n_keys, c->o_lat,
+                              (int64_t)c->max_q_tokens * cfg.n_heads * kLatent, st, true)) != MLA_OK)
       return s;
-    if ((s = make_map(&mqr, c->qp, kQK, R, cfg.batch, kQK * 2, qp_rows * kQK * 2, 32, 128,
-                      CU_TENSOR_MAP_SWIZZLE_64B, true)) != MLA_OK)
-      return s;
-    if ((s = make_map(&mkc, c->ckv, kLatent, n_keys, cfg.batch, kLatent * 2,
-                      (uint64_t)c->rows_per_stream * kLatent * 2, 64, 128,
-                      CU_TENSOR_MAP_SWIZZLE_128B, true)) != MLA_OK)
-      return s;
-    if ((s = make_map(&mkr, c->krope, kRope, n_keys, cfg.batch, kRope * 2,
-                      (uint64_t)c->rows_per_stream * kRope * 2, 32, 128,
-                      CU_TENSOR_MAP_SWIZZLE_64B, true)) != MLA_OK)
-      return s;
-    mla::AttnArgs a{};
-    a.rows = (int32_t)R;
-    a.n_keys = (int32_t)n_keys;
-    a.o_lat = c->o_lat;
-    a.o_lat_batch_stride = (int64_t)c->max_q_tokens * cfg.n_heads * kLatent;
-    using Sm = mla::AttnSmem<kAttnStages, kAttnPInTmem>;
-    dim3 grid((unsigned)((R + 127) / 128), (unsigned)cfg.batch);
-    ProfScope p(c, MLA_KERNEL_ATTENTION, st);
-    mla::window_attn_kernel<kAttnStages, kAttnPInTmem>
-        <<<grid, mla::kAttnThreads, Sm::kBytes, st>>>(mqc, mqr, mkc, mkr, a, c->status);
-    if ((s = check_launch("window attention")) != MLA_OK) return s;
   }
 
   // 3. output projection out = o_lat W_OV^T
@@ -651,18 +694,16 @@ mla_status mla_window_attention(mla_cache* c, const void* x_chunk, int32_t n_fra
     ep.out_batch_stride = nq * cfg.hidden;
     ep.ld_out = cfg.hidden;
     ProfScope p(c, MLA_KERNEL_OPROJ, st);
-    dim3 grid((unsigned)((nq + 127) / 128), (unsigned)(cfg.hidden / c->out_bn),
-              (unsigned)cfg.batch);
-    if (c->out_bn == 256) {
-      mla::tc_gemm_kernel<256, kOutAStages, kOutBStages, mla::kEpiStore, true>
-          <<<grid, mla::kGemmThreads, mla::GemmSmem<256, kOutAStages, kOutBStages>::kBytes, st>>>(
-              ma, c->map_wov, (int)nq, (int)kin, 0, ep, c->status);
-    } else {
-      mla::tc_gemm_kernel<128, kOutAStages, kOutBStages, mla::kEpiStore, true>
-          <<<grid, mla::kGemmThreads, mla::GemmSmem<128, kOutAStages, kOutBStages>::kBytes, st>>>(
-              ma, c->map_wov, (int)nq, (int)kin, 0, ep, c->status);
-    }
-    if ((s = check_launch("output projection")) != MLA_OK) return s;
+    const mla::GemmTiles tiles{(int32_t)((nq + 127) / 128), cfg.hidden / c->out_bn, cfg.batch};
+    if (c->out_bn == 256)
+      s = launch_gemm<256, kOutAStages, kOutBStages, mla::kEpiStore, true>(
+          ma, c->map_wov, (int)nq, (int)kin, 0, tiles, ep, c->status, c->num_sms, st,
+          "output projection");
+    else
+      s = launch_gemm<128, kOutAStages, kOutBStages, mla::kEpiStore, true>(
+          ma, c->map_wov, (int)nq, (int)kin, 0, tiles, ep, c->status, c->num_sms, st,
+          "output projection");
+    if (s != MLA_OK) return s;
   }
   return MLA_OK;
 }
@@ -703,62 +744,12 @@ mla_status mla_window_attention_noalloc(mla_cache* c, const void* x_chunk, int32
   const int64_t n_keys = base_row + nq;
 
   // 1. absorbed queries (into the scratch) + chunk latents (into the cache's chunk tail)
-  {
-    CUtensorMap map_x;
-    if ((s = make_map(&map_x, x_chunk, cfg.hidden, nq, cfg.batch, (uint64_t)cfg.hidden * 2,
-                      (uint64_t)nq * cfg.hidden * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B)) != MLA_OK)
-      return s;
-    EpiArgs ep{};
-    ep.ckv = c->ckv;
-    ep.krope = c->krope;
-    ep.rows_per_stream = c->rows_per_stream;
-    ep.qp = qp;
-    ep.qp_rows_per_stream = R;
-    ep.latent_y = cfg.n_heads;
-    ep.n_heads = cfg.n_heads;
-    ep.ring_mode = 0;
-    ep.t0 = c->frames_appended;
-    ep.window_frames = cfg.window_frames;
-    ep.tokens_per_frame = c->F;
-    ep.frame_w = cfg.frame_w;
-    ep.base_row = base_row;
-    ep.q_scale = c->softmax_scale * 1.4426950408889634f;
-    ep.rope = c->rope;
-    using Sm = mla::GemmSmem<kQK, kProjAStages, kProjBStages>;
-    dim3 grid((unsigned)((nq + 127) / 128), (unsigned)(cfg.n_heads + 1), (unsigned)cfg.batch);
-    mla::tc_gemm_kernel<kQK, kProjAStages, kProjBStages, mla::kEpiLatent, false>
-        <<<grid, mla::kGemmThreads, Sm::kBytes, st>>>(map_x, c->map_wqcat, (int)nq, cfg.hidden,
-                                                     0, ep, c->status);
-    if ((s = check_launch("no-alloc latent projection")) != MLA_OK) return s;
-  }
+  if ((s = launch_latent_gemm(c, x_chunk, nq, nq, cfg.n_heads + 1, cfg.n_heads, 0, 0,
+                              c->frames_appended, base_row, st, qp, R)) != MLA_OK)
+    return s;
   // 2. window attention, o_lat into the scratch
-  {
-    CUtensorMap mqc, mqr, mkc, mkr;
-    if ((s = make_map(&mqc, qp, kQK, R, cfg.batch, kQK * 2, (uint64_t)R * kQK * 2, 64, 128,
-                      CU_TENSOR_MAP_SWIZZLE_128B, true)) != MLA_OK)
-      return s;
-    if ((s = make_map(&mqr, qp, kQK, R, cfg.batch, kQK * 2, (uint64_t)R * kQK * 2, 32, 128,
-                      CU_TENSOR_MAP_SWIZZLE_64B, true)) != MLA_OK)
-      return s;
-    if ((s = make_map(&mkc, c->ckv, kLatent, n_keys, cfg.batch, kLatent * 2,
-                      (uint64_t)c->rows_per_stream * kLatent * 2, 64, 128,
-                      CU_TENSOR_MAP_SWIZZLE_128B, true)) != MLA_OK)
-      return s;
-    if ((s = make_map(&mkr, c->krope, kRope, n_keys, cfg.batch, kRope * 2,
-                      (uint64_t)c->rows_per_stream * kRope * 2, 32, 128,
-                      CU_TENSOR_MAP_SWIZZLE_64B, true)) != MLA_OK)
-      return s;
-    mla::AttnArgs a{};
-    a.rows = (int32_t)R;
-    a.n_keys = (int32_t)n_keys;
-    a.o_lat = o_lat;
-    a.o_lat_batch_stride = R * kLatent;
-    using Sm = mla::AttnSmem<kAttnStages, kAttnPInTmem>;
-    dim3 grid((unsigned)((R + 127) / 128), (unsigned)cfg.batch);
-    mla::window_attn_kernel<kAttnStages, kAttnPInTmem>
-        <<<grid, mla::kAttnThreads, Sm::kBytes, st>>>(mqc, mqr, mkc, mkr, a, c->status);
-    if ((s = check_launch("no-alloc window attention")) != MLA_OK) return s;
-  }
+  if ((s = launch_attention(c, qp, R * kQK, R, n_keys, o_lat, R * kLatent, st, false)) != MLA_OK)
+    return s;
   // 3. output projection from the scratch o_lat
   {
     CUtensorMap ma;
@@ -770,18 +761,16 @@ mla_status mla_window_attention_noalloc(mla_cache* c, const void* x_chunk, int32
     ep.out = static_cast<__nv_bfloat16*>(out);
     ep.out_batch_stride = nq * cfg.hidden;
     ep.ld_out = cfg.hidden;
-    dim3 grid((unsigned)((nq + 127) / 128), (unsigned)(cfg.hidden / c->out_bn),
-              (unsigned)cfg.batch);
-    if (c->out_bn == 256) {
-      mla::tc_gemm_kernel<256, kOutAStages, kOutBStages, mla::kEpiStore, true>
-          <<<grid, mla::kGemmThreads, mla::GemmSmem<256, kOutAStages, kOutBStages>::kBytes, st>>>(
-              ma, c->map_wov, (int)nq, (int)kin, 0, ep, c->status);
-    } else {
-      mla::tc_gemm_kernel<128, kOutAStages, kOutBStages, mla::kEpiStore, true>
-          <<<grid, mla::kGemmThreads, mla::GemmSmem<128, kOutAStages, kOutBStages>::kBytes, st>>>(
-              ma, c->map_wov, (int)nq, (int)kin, 0, ep, c->status);
-    }
-    if ((s = check_launch("no-alloc output projection")) != MLA_OK) return s;
+    const mla::GemmTiles tiles{(int32_t)((nq + 127) / 128), cfg.hidden / c->out_bn, cfg.batch};
+    if (c->out_bn == 256)
+      s = launch_gemm<256, kOutAStages, kOutBStages, mla::kEpiStore, true>(
+          ma, c->map_wov, (int)nq, (int)kin, 0, tiles, ep, c->status, c->num_sms, st,
+          "no-alloc output projection");
+    else
+      s = launch_gemm<128, kOutAStages, kOutBStages, mla::kEpiStore, true>(
+          ma, c->map_wov, (int)nq, (int)kin, 0, tiles, ep, c->status, c->num_sms, st,
+          "no-alloc output projection");
+    if (s != MLA_OK) return s;
   }
   return MLA_OK;
 }

@@ -76,6 +76,37 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* s
   }
 }
 
+// Whole-warp wait for a phase that may take many microseconds (e.g. an epilogue waiting for a
+// tile's MMAs): only lane 0 polls, with a growing __nanosleep back-off, so that 32 threads do
+// not hammer the barrier's shared-memory word (and the status word's L2 line) while the
+// producer and MMA warps need shared-memory bandwidth.  Same bounded-timeout contract as
+// mbar_wait; the result is broadcast to the warp.  Must be called by all 32 lanes.
+__device__ __forceinline__ bool mbar_wait_warp_sleepy(uint64_t* bar, uint32_t parity, int* status) {
+  uint32_t ok = 1;
+  if ((threadIdx.x & 31u) == 0) {
+    if (!mbar_try_wait(bar, parity)) {
+      const uint64_t t0 = global_timer_ns();
+      uint32_t sleep_ns = 32;
+      for (uint32_t n = 1;; ++n) {
+        __nanosleep(sleep_ns);
+        if (sleep_ns < 256) sleep_ns <<= 1;
+        if (mbar_try_wait(bar, parity)) break;
+        if ((n & 63u) == 0u) {
+          if (*reinterpret_cast<volatile int*>(status) != 0) { ok = 0; break; }
+          if (global_timer_ns() - t0 > kWaitLimitNs) {
+            atomicCAS(status, 0, kStatusTimeout);
+            ok = 0;
+            break;
+          }
+        }
+      }
+    }
+  }
+  ok = __shfl_sync(0xffffffffu, ok, 0);
+  __syncwarp();
+  return ok != 0;
+}
+
 // Named barrier over a subset of warps (id 1..15; id 0 is __syncthreads).
 __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
@@ -113,6 +144,25 @@ __device__ __forceinline__ uint64_t l2_policy_evict_last() {
   uint64_t p;
   asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
   return p;
+}
+
+// Bulk (non-tensor) asynchronous copy shared -> global of `bytes` (multiple of 16, both
+// addresses 16-byte aligned), tracked by the issuing thread's bulk async-group.
+__device__ __forceinline__ void bulk_store(void* gdst, const void* ssrc, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst),
+               "r"(smem_u32(ssrc)), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// Wait until this thread's committed bulk copies have finished reading shared memory.
+__device__ __forceinline__ void bulk_wait_read_all() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// Wait until this thread's committed bulk copies have completed.
+__device__ __forceinline__ void bulk_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 
 // Generic-proxy shared-memory writes -> visible to the async proxy (tensor core, TMA).
@@ -217,8 +267,28 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* r) {
       "r"(r[29]), "r"(r[30]), "r"(r[31])
       : "memory");
 }
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15])
+      : "memory");
+}
 __device__ __forceinline__ void tmem_ld_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+// After tmem_ld_wait: tell the compiler these 32 registers are (re)defined here, so no use of
+// a tcgen05.ld result can be scheduled above the wait that makes it valid.
+__device__ __forceinline__ void tmem_regs_ready(uint32_t* r) {
+  asm volatile(""
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
+                 "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]),
+                 "+r"(r[13]), "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]),
+                 "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), "+r"(r[24]),
+                 "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]),
+                 "+r"(r[31]));
 }
 __device__ __forceinline__ void tmem_st_wait() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");

@@ -12,21 +12,24 @@
 // k_h = [c W_UK[h]^T | k_R] and values v_h = c W_UV[h]^T are never built; all heads read the
 // same head-shared latent tile, which makes the contraction an MQA-shaped dense GEMM.
 //
-// One CTA owns 128 rows.  Warp roles (192 threads):
-//   warp 0      TMA producer: the Q tile once, then 128-key tiles of c_kv (3 x 64-column
-//               128B-swizzled boxes) and k_rope (one 32-column 64B-swizzled box) into a
-//               KV_STAGES-deep ring.  Keys past n_keys are zero-filled by the tensor map.
+// One CTA owns 128 rows.  Shared-memory bandwidth is the scarce resource here (the MMAs, the
+// TMA writes and the softmax all share it), so both MMAs take their A operand from tensor
+// memory and shared memory only holds the streamed key tiles:
+//   warp 0      TMA producer: 128-key tiles of c_kv (3 x 64-column 128B-swizzled boxes) and
+//               k_rope (one 32-column 64B-swizzled box) into a KV_STAGES-deep ring.  Keys past
+//               n_keys are zero-filled by the tensor map.
 //   warp 1      TMEM allocator + single-thread MMA issuer:
-//                 S_j  = Q K_j^T     M=128 N=128 K=224 (14 k-steps; both operands K-major)
-//                 O   += P_j C_j     M=128 N=192 K=128 (8 k-steps; C_j is the SAME smem tile
-//                                    read MN-major, P_j from shared or tensor memory)
-//               S is double-buffered in TMEM so S_{j+1} runs while softmax works on S_j.
-//   warps 2..5  softmax: one row per thread, tcgen05.ld of its S row, running max with lazy
-//               rescaling (O is rescaled in TMEM only when the max grows by > 2^8), ex2,
-//               P_j as fp16 into shared memory (P_IN_TMEM = false) or tensor memory (true);
-//               finally O / l -> fp16 -> o_lat, staged for coalesced 384-byte row stores.
+//                 S_j  = Q K_j^T     M=128 N=128 K=224 (14 k-steps; Q from TMEM, K_j K-major)
+//                 O   += P_j C_j     M=128 N=192 K=128 (8 k-steps; P_j from TMEM, C_j is the
+//                                    SAME smem tile as K_j, read MN-major)
+//               S_{j+1} is issued as soon as the softmax has copied S_j to registers, so it
+//               runs while the softmax works on tile j.
+//   warps 2..5  first load this CTA's Qp rows into TMEM (one row per thread), then softmax:
+//               one row per thread, running max with lazy rescaling (O is rescaled in TMEM
+//               only when the max grows by > 2^8), ex2, P_j as fp16 into TMEM; finally O / l ->
+//               fp16 o_lat, staged in shared memory and written by one bulk copy per row.
 //
-// TMEM columns: S0 [0,128), S1 [128,256), O [256,448), P [448,512) (P_IN_TMEM only).
+// TMEM columns: S [0,128), P [128,192), Q [192,304), O [304,496).
 #pragma once
 
 #include "ptx.cuh"
@@ -37,44 +40,49 @@ constexpr int kAttnThreads = 192;
 constexpr int kTileKeys = 128;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: lazy O rescale when max grows > 2^8
 
-template <int KV_STAGES, bool P_IN_TMEM>
+template <int KV_STAGES>
 struct AttnSmem {
-  static constexpr int kAtomC = 128 * 128;           // 128 rows x 64 bf16 (SW128)
-  static constexpr int kAtomR = 128 * 64;            // 128 rows x 32 bf16 (SW64)
-  static constexpr int kTileBytes = 3 * kAtomC + kAtomR;   // 57344: one Q or KV tile
-  static constexpr int kQ = 0;
-  static constexpr int kKV = kTileBytes;
-  static constexpr int kP = kKV + KV_STAGES * kTileBytes;
-  static constexpr int kPBytes = P_IN_TMEM ? 0 : 2 * kAtomC;
-  static constexpr int kBar = kP + kPBytes;
+  static constexpr int kAtomC = 128 * 128;           // 128 keys x 64 fp16 (SW128)
+  static constexpr int kAtomR = 128 * 64;            // 128 keys x 32 fp16 (SW64)
+  static constexpr int kTileBytes = 3 * kAtomC + kAtomR;   // 57344: one key tile
+  static constexpr int kKV = 0;
+  static constexpr int kBar = kKV + KV_STAGES * kTileBytes;
   static constexpr int kBytes = kBar + 256 + 1024;
+  static constexpr int kStageStride = 400;           // o_lat staging row: 384 B + 16 padding
   static_assert(kBytes <= 232448, "attention tile does not fit in shared memory");
+  static_assert(128 * kStageStride <= kTileBytes, "o_lat staging must fit in one KV stage");
 };
 
+// TMEM column map (512 allocated).
+constexpr uint32_t kTmemS = 0;
+constexpr uint32_t kTmemP = 128;
+constexpr uint32_t kTmemQ = 192;
+constexpr uint32_t kTmemO = 304;
+
 struct AttnArgs {
-  int32_t rows;       // R = n_q * n_heads valid rows per stream
-  int32_t n_keys;     // keys per stream (window + chunk)
+  const __half* qp;            // [batch][qp_rows][224] fp16
+  int64_t qp_batch_stride;     // elements
+  int32_t rows;                // R = n_q * n_heads valid rows per stream
+  int32_t n_keys;              // keys per stream (window + chunk)
   __half* o_lat;               // fp16
   int64_t o_lat_batch_stride;  // elements
 };
 
-template <int KV_STAGES, bool P_IN_TMEM>
+template <int KV_STAGES>
 __global__ void __launch_bounds__(kAttnThreads, 1)
-    window_attn_kernel(const __grid_constant__ CUtensorMap map_qc,
-                       const __grid_constant__ CUtensorMap map_qr,
-                       const __grid_constant__ CUtensorMap map_kc,
+    window_attn_kernel(const __grid_constant__ CUtensorMap map_kc,
                        const __grid_constant__ CUtensorMap map_kr, AttnArgs args, int* status) {
-  using L = AttnSmem<KV_STAGES, P_IN_TMEM>;
+  using L = AttnSmem<KV_STAGES>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
-  uint64_t* q_full = bars;
+  uint64_t* q_ready = bars;
   uint64_t* kv_full = bars + 1;                  // [KV_STAGES]
   uint64_t* kv_empty = kv_full + KV_STAGES;      // [KV_STAGES]
-  uint64_t* s_full = kv_empty + KV_STAGES;       // [2]
-  uint64_t* s_free = s_full + 2;                 // [2]
-  uint64_t* p_full = s_free + 2;
+  uint64_t* s_full = kv_empty + KV_STAGES;
+  uint64_t* s_free = s_full + 1;
+  uint64_t* p_full = s_free + 1;
   uint64_t* pv_done = p_full + 1;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(pv_done + 1);
 
@@ -86,20 +94,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const int nt = (n_keys + kTileKeys - 1) / kTileKeys;
 
   if (threadIdx.x == 0) {
-    mbar_init(q_full, 1);
+    mbar_init(q_ready, 128);
     for (int s = 0; s < KV_STAGES; ++s) {
       mbar_init(&kv_full[s], 1);
       mbar_init(&kv_empty[s], 1);
     }
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&s_full[s], 1);
-      mbar_init(&s_free[s], 128);
-    }
+    mbar_init(s_full, 1);
+    mbar_init(s_free, 128);
     mbar_init(p_full, 128);
     mbar_init(pv_done, 1);
     fence_mbar_init();
-    tma_prefetch(&map_qc);
-    tma_prefetch(&map_qr);
     tma_prefetch(&map_kc);
     tma_prefetch(&map_kr);
   }
@@ -111,19 +115,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
-  const uint32_t tmem_o = tmem + 256;
-  const uint32_t tmem_p = tmem + 448;
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
       const uint64_t keep = l2_policy_evict_last();    // keys are re-read by every row tile
-      const uint64_t once = l2_policy_evict_first();   // the Q tile is read once
-      uint8_t* q = smem + L::kQ;
-      mbar_arrive_expect_tx(q_full, L::kTileBytes);
-      for (int a = 0; a < 3; ++a)
-        tma_load_3d_hint(q + a * L::kAtomC, &map_qc, q_full, a * 64, m0, z, once);
-      tma_load_3d_hint(q + 3 * L::kAtomC, &map_qr, q_full, 192, m0, z, once);
       int issued = 0;
       for (int j = 0; j < nt; ++j) {
         const int st = j % KV_STAGES;
@@ -140,38 +136,33 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       // Drain: never leave the CTA with a copy still landing in its shared memory.
       for (int j = issued > KV_STAGES ? issued - KV_STAGES : 0; j < issued; ++j)
         mbar_wait(&kv_full[j % KV_STAGES], (uint32_t)(j / KV_STAGES) & 1u, status);
-      mbar_wait(q_full, 0, status);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_f32acc(128, kTileKeys, false, true);
       constexpr uint32_t idesc_o = idesc_f32acc(128, 192, true, true);
-      const uint32_t q_base = smem_u32(smem + L::kQ);
-      bool ok = mbar_wait(q_full, 0, status);
+      bool ok = mbar_wait(q_ready, 0, status);
       for (int j = 0; ok && j <= nt; ++j) {
         if (j < nt) {
           const int st = j % KV_STAGES;
-          const int sb = j & 1;
           if (!mbar_wait(&kv_full[st], (uint32_t)(j / KV_STAGES) & 1u, status)) break;
-          if (j >= 2 && !mbar_wait(&s_free[sb], (uint32_t)((j >> 1) - 1) & 1u, status)) break;
+          // S is single-buffered: the softmax must have copied S_{j-1} to registers.
+          if (j >= 1 && !mbar_wait(s_free, (uint32_t)(j - 1) & 1u, status)) break;
           tc_fence_after();
           const uint32_t kv_base = smem_u32(smem + L::kKV + st * L::kTileBytes);
 #pragma unroll
           for (int kk = 0; kk < 14; ++kk) {
-            uint64_t da, db;
-            if (kk < 12) {
-              const uint32_t off = (kk >> 2) * L::kAtomC + (kk & 3) * 32;
-              da = smem_desc(q_base + off, 16, 1024, kSwizzle128B);
-              db = smem_desc(kv_base + off, 16, 1024, kSwizzle128B);
-            } else {
-              const uint32_t off = 3 * L::kAtomC + (kk - 12) * 32;
-              da = smem_desc(q_base + off, 16, 512, kSwizzle64B);
-              db = smem_desc(kv_base + off, 16, 512, kSwizzle64B);
-            }
-            umma_ss(tmem + sb * kTileKeys, da, db, idesc_s, kk > 0 ? 1u : 0u);
+            // A = Q from TMEM: 16 fp16 of K per step = 8 packed columns.
+            uint64_t db;
+            if (kk < 12)
+              db = smem_desc(kv_base + (kk >> 2) * L::kAtomC + (kk & 3) * 32, 16, 1024,
+                             kSwizzle128B);
+            else
+              db = smem_desc(kv_base + 3 * L::kAtomC + (kk - 12) * 32, 16, 512, kSwizzle64B);
+            umma_ts(tmem + kTmemS, tmem + kTmemQ + kk * 8, db, idesc_s, kk > 0 ? 1u : 0u);
           }
-          tc_commit(&s_full[sb]);
+          tc_commit(s_full);
         }
         if (j >= 1) {
           const int jj = j - 1;
@@ -184,15 +175,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             // C_j read MN-major: 16 keys per step = two 8-row core groups of 1 KB; the three
             // 64-column atoms are 16 KB apart (leading byte offset).
             const uint64_t db = smem_desc(c_base + kk * 2048, L::kAtomC, 1024, kSwizzle128B);
-            const uint32_t acc = (jj > 0 || kk > 0) ? 1u : 0u;
-            if constexpr (P_IN_TMEM) {
-              umma_ts(tmem_o, tmem_p + kk * 8, db, idesc_o, acc);
-            } else {
-              const uint32_t p_base = smem_u32(smem + L::kP);
-              const uint64_t da = smem_desc(p_base + (kk >> 2) * L::kAtomC + (kk & 3) * 32, 16,
-                                            1024, kSwizzle128B);
-              umma_ss(tmem_o, da, db, idesc_o, acc);
-            }
+            umma_ts(tmem + kTmemO, tmem + kTmemP + kk * 8, db, idesc_o,
+                    (jj > 0 || kk > 0) ? 1u : 0u);
           }
           tc_commit(pv_done);
           tc_commit(&kv_empty[st]);
@@ -201,24 +185,53 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
   } else {
     // ------------------------------------------------------------------ softmax warps
-    const uint32_t sub = warp & 3u;
-    const int row = sub * 32 + lane;
-    const uint32_t lane_off = (sub * 32u) << 16;
+    const uint32_t quarter = warp & 3u;          // TMEM lane quarter (rows 32q .. 32q+31)
+    const int row = quarter * 32 + lane;
+    const uint32_t lane_off = (quarter * 32u) << 16;
+
+    // Q rows -> TMEM (A operand of S): row r's 224 fp16 = 112 packed columns at lane r.
+    {
+      const int gr = m0 + row;
+      const uint4* src = reinterpret_cast<const uint4*>(args.qp + z * args.qp_batch_stride +
+                                                        (int64_t)gr * 224);
+      const bool in = gr < args.rows;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {                // columns [32c, 32c + 32) of 112
+        uint32_t q[32];
+        const int n16 = c < 3 ? 8 : 4;             // 16-byte pieces in this chunk (last: 16 cols)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const uint4 v = (in && i < n16) ? src[c * 8 + i] : make_uint4(0u, 0u, 0u, 0u);
+          q[4 * i + 0] = v.x;
+          q[4 * i + 1] = v.y;
+          q[4 * i + 2] = v.z;
+          q[4 * i + 3] = v.w;
+        }
+        if (c < 3)
+          tmem_st32(tmem + kTmemQ + lane_off + c * 32, q);
+        else
+          tmem_st16(tmem + kTmemQ + lane_off + 96, q);      // columns [96, 112)
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(q_ready);
+    }
+
     float m_used = -INFINITY;
     float l_sum = 0.f;
     bool ok = true;
     for (int j = 0; j < nt; ++j) {
-      const int sb = j & 1;
-      if (!mbar_wait(&s_full[sb], (uint32_t)(j >> 1) & 1u, status)) { ok = false; break; }
+      if (!mbar_wait(s_full, (uint32_t)j & 1u, status)) { ok = false; break; }
       tc_fence_after();
       float s[kTileKeys];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        tmem_ld32(tmem + lane_off + sb * kTileKeys + c * 32, reinterpret_cast<uint32_t*>(s) + c * 32);
-      }
+      for (int c = 0; c < 4; ++c)
+        tmem_ld32(tmem + kTmemS + lane_off + c * 32, reinterpret_cast<uint32_t*>(s) + c * 32);
       tmem_ld_wait();
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_regs_ready(reinterpret_cast<uint32_t*>(s) + c * 32);
       tc_fence_before();
-      mbar_arrive(&s_free[sb]);
+      mbar_arrive(s_free);
 
       const int valid = n_keys - j * kTileKeys;   // keys of this tile that exist
       if (valid < kTileKeys) {
@@ -226,8 +239,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         for (int i = 0; i < kTileKeys; ++i)
           if (i >= valid) s[i] = -INFINITY;
       }
-      // Row max with 8 independent partial maxima: one softmax warp per SM sub-partition, so
-      // a serial 128-long dependency chain would sit on the critical path of every tile.
+      // Row max with 8 independent partial maxima.
       float pm[8];
 #pragma unroll
       for (int k = 0; k < 8; ++k) pm[k] = s[k];
@@ -263,29 +275,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll 1
         for (int c = 0; c < 6; ++c) {
           uint32_t o[32];
-          tmem_ld32(tmem_o + lane_off + c * 32, o);
+          tmem_ld32(tmem + kTmemO + lane_off + c * 32, o);
           tmem_ld_wait();
+          tmem_regs_ready(o);
 #pragma unroll
           for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-          tmem_st32(tmem_o + lane_off + c * 32, o);
+          tmem_st32(tmem + kTmemO + lane_off + c * 32, o);
         }
         tmem_st_wait();
       }
-      if constexpr (P_IN_TMEM) {
-        tmem_st32(tmem_p + lane_off, pk);
-        tmem_st32(tmem_p + lane_off + 32, pk + 32);
-        tmem_st_wait();
-      } else {
-        uint8_t* p_row = smem + L::kP + row * 128;
-#pragma unroll
-        for (int c = 0; c < 16; ++c) {   // 16-byte chunk c = keys 8c..8c+7
-          const int atom = c >> 3;
-          const int phys = (c & 7) ^ (row & 7);
-          *reinterpret_cast<uint4*>(p_row + atom * L::kAtomC + phys * 16) =
-              make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-        }
-        fence_proxy_async_smem();
-      }
+      tmem_st32(tmem + kTmemP + lane_off, pk);
+      tmem_st32(tmem + kTmemP + lane_off + 32, pk + 32);
+      tmem_st_wait();
       tc_fence_before();
       mbar_arrive(p_full);
     }
@@ -294,14 +295,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     if (ok && mbar_wait(pv_done, (uint32_t)(nt - 1) & 1u, status)) {
       tc_fence_after();
       const float inv_l = 1.f / l_sum;
-      // Stage in the (now idle) first KV stage: 128 rows x (384 + 16) bytes.
-      constexpr int kStride = 400;
-      uint8_t* st_row = smem + L::kKV + row * kStride;
+      // Stage the row in the (now idle) first KV stage, then one bulk copy of 384 bytes.
+      uint8_t* st_row = smem + L::kKV + row * L::kStageStride;
 #pragma unroll 1
       for (int c = 0; c < 6; ++c) {
         uint32_t o[32];
-        tmem_ld32(tmem_o + lane_off + c * 32, o);
+        tmem_ld32(tmem + kTmemO + lane_off + c * 32, o);
         tmem_ld_wait();
+        tmem_regs_ready(o);
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           reinterpret_cast<uint4*>(st_row + c * 64)[q] = make_uint4(
@@ -311,16 +312,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
               pack_f16x2(__uint_as_float(o[8 * q + 6]) * inv_l, __uint_as_float(o[8 * q + 7]) * inv_l));
         }
       }
-      __syncwarp();
-      __half* out = args.o_lat + z * args.o_lat_batch_stride;
-      for (int rr = 0; rr < 32; ++rr) {
-        const int trow = sub * 32 + rr;
-        const int gr = m0 + trow;
-        if (gr >= args.rows) break;
-        if (lane < 24) {
-          reinterpret_cast<uint4*>(out + (int64_t)gr * 192)[lane] =
-              reinterpret_cast<const uint4*>(smem + L::kKV + trow * kStride)[lane];
-        }
+      const int gr = m0 + row;
+      if (gr < args.rows) {
+        fence_proxy_async_smem();
+        bulk_store(args.o_lat + z * args.o_lat_batch_stride + (int64_t)gr * 192, st_row, 384);
+        bulk_commit();
+        bulk_wait_all();
       }
     }
     tc_fence_before();
