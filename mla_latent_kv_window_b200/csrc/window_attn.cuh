@@ -16,14 +16,14 @@
 // TMA writes and the softmax all share it), so both MMAs take their A operand from tensor
 // memory and shared memory only holds the streamed key tiles:
 //   warp 0      TMA producer: 128-key tiles of c_kv (3 x 64-column 128B-swizzled boxes) and
-//               k_rope (one 32-column 64B-swizzled box) into a KV_STAGES-deep ring.  Keys past
-//               n_keys are zero-filled by the tensor map.
-//   warp 1      TMEM allocator + single-thread MMA issuer:
-//                 S_j  = Q K_j^T     M=128 N=128 K=224 (14 k-steps; Q from TMEM, K_j K-major)
-//                 O   += P_j C_j     M=128 N=192 K=128 (8 k-steps; P_j from TMEM, C_j is the
-//                                    SAME smem tile as K_j, read MN-major)
-//               S_{j+1} is issued as soon as the softmax has copied S_j to registers, so it
-//               runs while the softmax works on tile j.
+//               k_rope (one 32-column 64B-swizzled box) into a KV_STAGES-deep ring, starting at
+//               a CTA-dependent tile.  Keys past n_keys are zero-filled by the tensor map.
+//   warp 1      TMEM allocator + issuer of S_j = Q K_j^T  (M=128 N=128 K=224, 14 k-steps; Q
+//               from TMEM, K_j K-major).  S_{j+1} is issued as soon as the softmax has copied
+//               S_j to registers, so it runs while the softmax works on tile j.
+//   warp 6      issuer of O += P_j C_j  (M=128 N=192 K=128, 8 k-steps; P_j from TMEM, C_j is the
+//               SAME smem tile as K_j, read MN-major).  Two issuing threads keep the tensor
+//               pipe fed: neither stream waits behind the other's barrier checks.
 //   warps 2..5  first load this CTA's Qp rows into TMEM (one row per thread), then softmax:
 //               one row per thread, running max with lazy rescaling (O is rescaled in TMEM
 //               only when the max grows by > 2^8), ex2, P_j as fp16 into TMEM; finally O / l ->
@@ -36,7 +36,7 @@
 
 namespace mla {
 
-constexpr int kAttnThreads = 192;
+constexpr int kAttnThreads = 224;
 constexpr int kTileKeys = 128;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: lazy O rescale when max grows > 2^8
 
@@ -92,6 +92,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const int z = blockIdx.y;
   const int n_keys = args.n_keys;
   const int nt = (n_keys + kTileKeys - 1) / kTileKeys;
+  // Every CTA walks all key tiles, each from its own starting tile: CTAs that stream the same
+  // tiles in lockstep pile onto the same L2 lines (softmax does not depend on key order).
+  const int rot = (int)(((unsigned)blockIdx.x * 37u + (unsigned)blockIdx.y * 11u) % (unsigned)nt);
 
   if (threadIdx.x == 0) {
     mbar_init(q_ready, 128);
@@ -127,10 +130,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         if (!mbar_wait(&kv_empty[st], (round & 1u) ^ 1u, status)) break;
         uint8_t* kv = smem + L::kKV + st * L::kTileBytes;
         mbar_arrive_expect_tx(&kv_full[st], L::kTileBytes);
+        const int key0 = ((j + rot) % nt) * kTileKeys;
         for (int a = 0; a < 3; ++a)
-          tma_load_3d_hint(kv + a * L::kAtomC, &map_kc, &kv_full[st], a * 64, j * kTileKeys, z,
-                           keep);
-        tma_load_3d_hint(kv + 3 * L::kAtomC, &map_kr, &kv_full[st], 0, j * kTileKeys, z, keep);
+          tma_load_3d_hint(kv + a * L::kAtomC, &map_kc, &kv_full[st], a * 64, key0, z, keep);
+        tma_load_3d_hint(kv + 3 * L::kAtomC, &map_kr, &kv_full[st], 0, key0, z, keep);
         issued = j + 1;
       }
       // Drain: never leave the CTA with a copy still landing in its shared memory.
@@ -138,49 +141,53 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         mbar_wait(&kv_full[j % KV_STAGES], (uint32_t)(j / KV_STAGES) & 1u, status);
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------------ MMA issuer
+    // ------------------------------------------------------------------ S issuer
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_f32acc(128, kTileKeys, false, true);
-      constexpr uint32_t idesc_o = idesc_f32acc(128, 192, true, true);
       bool ok = mbar_wait(q_ready, 0, status);
-      for (int j = 0; ok && j <= nt; ++j) {
-        if (j < nt) {
-          const int st = j % KV_STAGES;
-          if (!mbar_wait(&kv_full[st], (uint32_t)(j / KV_STAGES) & 1u, status)) break;
-          // S is single-buffered: the softmax must have copied S_{j-1} to registers.
-          if (j >= 1 && !mbar_wait(s_free, (uint32_t)(j - 1) & 1u, status)) break;
-          tc_fence_after();
-          const uint32_t kv_base = smem_u32(smem + L::kKV + st * L::kTileBytes);
+      for (int j = 0; ok && j < nt; ++j) {
+        const int st = j % KV_STAGES;
+        if (!mbar_wait(&kv_full[st], (uint32_t)(j / KV_STAGES) & 1u, status)) break;
+        // S is single-buffered: the softmax must have copied S_{j-1} to registers.
+        if (j >= 1 && !mbar_wait(s_free, (uint32_t)(j - 1) & 1u, status)) break;
+        tc_fence_after();
+        const uint32_t kv_base = smem_u32(smem + L::kKV + st * L::kTileBytes);
 #pragma unroll
-          for (int kk = 0; kk < 14; ++kk) {
-            // A = Q from TMEM: 16 fp16 of K per step = 8 packed columns.
-            uint64_t db;
-            if (kk < 12)
-              db = smem_desc(kv_base + (kk >> 2) * L::kAtomC + (kk & 3) * 32, 16, 1024,
-                             kSwizzle128B);
-            else
-              db = smem_desc(kv_base + 3 * L::kAtomC + (kk - 12) * 32, 16, 512, kSwizzle64B);
-            umma_ts(tmem + kTmemS, tmem + kTmemQ + kk * 8, db, idesc_s, kk > 0 ? 1u : 0u);
-          }
-          tc_commit(s_full);
+        for (int kk = 0; kk < 14; ++kk) {
+          // A = Q from TMEM: 16 fp16 of K per step = 8 packed columns.
+          uint64_t db;
+          if (kk < 12)
+            db = smem_desc(kv_base + (kk >> 2) * L::kAtomC + (kk & 3) * 32, 16, 1024,
+                           kSwizzle128B);
+          else
+            db = smem_desc(kv_base + 3 * L::kAtomC + (kk - 12) * 32, 16, 512, kSwizzle64B);
+          umma_ts(tmem + kTmemS, tmem + kTmemQ + kk * 8, db, idesc_s, kk > 0 ? 1u : 0u);
         }
-        if (j >= 1) {
-          const int jj = j - 1;
-          const int st = jj % KV_STAGES;
-          if (!mbar_wait(p_full, (uint32_t)jj & 1u, status)) break;
-          tc_fence_after();
-          const uint32_t c_base = smem_u32(smem + L::kKV + st * L::kTileBytes);
+        tc_commit(s_full);
+      }
+    }
+  } else if (warp == 6) {
+    // ------------------------------------------------------------------ PV issuer
+    // A second issuing thread, so that the S and PV streams each wait only for their own
+    // inputs and the tensor pipe always has queued work.  tcgen05.commit tracks the MMAs of
+    // the committing thread; a key stage is released after PV_j, which (through P_j) follows
+    // S_j on the same stage.
+    if (lane == 0) {
+      constexpr uint32_t idesc_o = idesc_f32acc(128, 192, true, true);
+      for (int j = 0; j < nt; ++j) {
+        const int st = j % KV_STAGES;
+        if (!mbar_wait(p_full, (uint32_t)j & 1u, status)) break;
+        tc_fence_after();
+        const uint32_t c_base = smem_u32(smem + L::kKV + st * L::kTileBytes);
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            // C_j read MN-major: 16 keys per step = two 8-row core groups of 1 KB; the three
-            // 64-column atoms are 16 KB apart (leading byte offset).
-            const uint64_t db = smem_desc(c_base + kk * 2048, L::kAtomC, 1024, kSwizzle128B);
-            umma_ts(tmem + kTmemO, tmem + kTmemP + kk * 8, db, idesc_o,
-                    (jj > 0 || kk > 0) ? 1u : 0u);
-          }
-          tc_commit(pv_done);
-          tc_commit(&kv_empty[st]);
+        for (int kk = 0; kk < 8; ++kk) {
+          // C_j read MN-major: 16 keys per step = two 8-row core groups of 1 KB; the three
+          // 64-column atoms are 16 KB apart (leading byte offset).
+          const uint64_t db = smem_desc(c_base + kk * 2048, L::kAtomC, 1024, kSwizzle128B);
+          umma_ts(tmem + kTmemO, tmem + kTmemP + kk * 8, db, idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
         }
+        tc_commit(pv_done);
+        tc_commit(&kv_empty[st]);
       }
     }
   } else {
@@ -233,7 +240,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       tc_fence_before();
       mbar_arrive(s_free);
 
-      const int valid = n_keys - j * kTileKeys;   // keys of this tile that exist
+      const int valid = n_keys - ((j + rot) % nt) * kTileKeys;   // keys of this tile that exist
       if (valid < kTileKeys) {
 #pragma unroll
         for (int i = 0; i < kTileKeys; ++i)
