@@ -90,6 +90,7 @@ __global__ void __launch_bounds__(kDenseThreads, 1)
     tmem_relinquish();
   }
   tc_fence_before();
+  __syncwarp();      // reconverge single-lane branches: bar.sync must be warp-uniform
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
@@ -268,6 +269,7 @@ __global__ void __launch_bounds__(kDenseThreads, 1)
     tc_fence_before();
   }
 
+  __syncwarp();      // reconverge single-lane roles before the CTA-wide barrier
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();

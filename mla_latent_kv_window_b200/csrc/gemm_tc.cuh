@@ -6,13 +6,13 @@
 // Persistent: one CTA per SM walks the tiles t = blockIdx.x, blockIdx.x + gridDim.x, ... of a
 // (row tile, column block, batch) grid.  Each 128 x BN tile accumulates in fp32 tensor memory:
 //   warp 0      TMA producer of A k-blocks (64 wide) into an A_STAGES-deep ring
-//   warp 6      TMA producer of B k-blocks into a B_STAGES-deep ring
+//   warp 2      TMA producer of B k-blocks into a B_STAGES-deep ring
 //   warp 1      TMEM allocator + single-thread tcgen05.mma issuer (M=128, N=BN, K=16 steps)
-//   warps 2..5  epilogue: tcgen05.ld of the accumulator (one row per thread; the next 32-column
-//               chunk is loaded while the current one is converted), fused row transform into
-//               a padded shared-memory staging row, then one bulk async copy per contiguous
-//               destination segment of the row (c_kv 384 B + k_rope 64 B, Qp 448 B, or the
-//               output row), issued by the owning thread.
+//   warps 3..10 epilogue, two warps per TMEM lane quarter: each thread owns one row and one
+//               half of its 32-column chunks.  tcgen05.ld of the accumulator (the next chunk is
+//               loaded while the current one is converted), fused row transform into a padded
+//               shared-memory staging row, then one bulk async copy per contiguous destination
+//               segment of the half-row (c_kv / k_rope, Qp, or the output row).
 // The rings run continuously across tile boundaries.  With M_SUB = 1 the accumulator is
 // double-buffered in TMEM (2 x 256 columns), so the epilogue of tile i overlaps the MMAs of
 // tile i+1.  With M_SUB = 2 a tile is 256 rows: two M=128 accumulators (TMEM columns [0,256)
@@ -42,7 +42,8 @@ namespace mla {
 
 constexpr int kEpiStore = 0;
 constexpr int kEpiLatent = 1;
-constexpr int kGemmThreads = 224;
+constexpr int kGemmThreads = 352;
+constexpr int kEpiWarps = 8;       // two per TMEM lane quarter, each owning half of every row
 
 // Rotary bands of the d_rope = 32 positional channels: pair p rotates by pos[axis[p]] * freq[p].
 // Each frequency is carried as an unevaluated float sum hi + lo (|lo| <= ulp(hi) / 2), so that
@@ -162,7 +163,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&acc_full[s], 1);
-      mbar_init(&acc_empty[s], 128);
+      mbar_init(&acc_empty[s], kEpiWarps * 32);
     }
     fence_mbar_init();
     tma_prefetch(&map_a);
@@ -173,6 +174,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     tmem_relinquish();
   }
   tc_fence_before();
+  __syncwarp();      // reconverge single-lane branches: bar.sync must be warp-uniform
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
@@ -186,7 +188,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     m0 = (r - y * tiles.m_tiles) * kTileRows;
   };
 
-  if (warp == 0 || warp == 6) {
+  if (warp == 0 || warp == 2) {
     // ------------------------------------------------------------------ TMA producers
     if (lane == 0) {
       const bool is_a = warp == 0;
@@ -257,6 +259,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   } else {
     // ------------------------------------------------------------------ epilogue warps
     const uint32_t sub_q = warp & 3u;          // TMEM lane quarter this warp may access
+    const int half = (int)(warp - 3) >> 2;     // 0: first half of the chunks, 1: second half
+    constexpr int kChunks = BN / 32;
+    constexpr int kSplit = (kChunks + 1) / 2;
+    const int c_lo = half ? kSplit : 0;
+    const int c_hi = half ? kChunks : kSplit;
     const int row = sub_q * 32 + lane;         // row of each 128-row sub-tile owned by this thread
     uint8_t* stage_row = smem + L::kStagingOffset + row * L::kStageStride;
     for (int i = 0; i < my_tiles; ++i) {
@@ -271,9 +278,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const bool valid = m < M;
         const uint32_t tbase = tmem + (buf + sub) * 256 + ((sub_q * 32u) << 16);
 
-        // This thread's destination row(s), computed once per tile.
-        void* dst_main = nullptr;    // columns [0, 192) (latent), [0, 224) (query), [0, BN) (store)
-        void* dst_rope = nullptr;    // latent rows: the k_rope plane (columns [192, 224))
+        // This thread's destination row, computed once per tile.
+        uint8_t* dst_main = nullptr;  // byte 0 of the row: c_kv (latent), Qp (query), out (store)
+        uint8_t* dst_rope = nullptr;  // latent rows: the k_rope row (columns [192, 224))
         bool latent = false;
         int64_t t = 0;
         int hh = 0, ww = 0;
@@ -289,26 +296,29 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const int64_t dst_row =
                 (ep.ring_mode ? (int64_t)(t % ep.window_frames) * F + k : ep.base_row + m) +
                 (int64_t)z * ep.rows_per_stream;
-            dst_main = ep.ckv + dst_row * 192;
-            dst_rope = ep.krope + dst_row * 32;
+            dst_main = reinterpret_cast<uint8_t*>(ep.ckv + dst_row * 192);
+            dst_rope = reinterpret_cast<uint8_t*>(ep.krope + dst_row * 32);
           } else {
             const int64_t qrow = (int64_t)z * ep.qp_rows_per_stream + (int64_t)m * ep.n_heads + y;
-            dst_main = ep.qp + qrow * 224;
+            dst_main = reinterpret_cast<uint8_t*>(ep.qp + qrow * 224);
           }
         } else {
-          dst_main = ep.out + z * ep.out_batch_stride + (int64_t)m * ep.ld_out + y * BN;
+          dst_main = reinterpret_cast<uint8_t*>(ep.out + z * ep.out_batch_stride +
+                                                (int64_t)m * ep.ld_out + y * BN);
         }
 
-        // The staging row is free once this thread's previous bulk copies have read it.
+        // The staging half-row is free once this thread's previous bulk copies have read it.
         bulk_wait_read_all();
         uint32_t r[2][32];
-        tmem_ld32(tbase, r[0]);
+        tmem_ld32(tbase + c_lo * 32, r[0]);
 #pragma unroll
-        for (int c = 0; c < BN / 32; ++c) {
-          uint32_t* cur = r[c & 1];
+        for (int cc = 0; cc < kSplit; ++cc) {
+          const int c = c_lo + cc;
+          if (c >= c_hi) break;
+          uint32_t* cur = r[cc & 1];
           tmem_ld_wait();
           tmem_regs_ready(cur);
-          if (c + 1 < BN / 32) tmem_ld32(tbase + (c + 1) * 32, r[(c + 1) & 1]);
+          if (c + 1 < c_hi) tmem_ld32(tbase + (c + 1) * 32, r[(cc + 1) & 1]);
           float v[32];
 #pragma unroll
           for (int q = 0; q < 32; ++q) v[q] = __uint_as_float(cur[q]);
@@ -337,15 +347,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         if (valid) {
           fence_proxy_async_smem();   // staging writes -> visible to the bulk-copy engine
-          if constexpr (kEpi == kEpiLatent) {
-            if (latent) {
-              bulk_store(dst_main, stage_row, 384);
-              bulk_store(dst_rope, stage_row + 384, 64);
-            } else {
-              bulk_store(dst_main, stage_row, 448);
-            }
+          const uint32_t b0 = c_lo * 64;                       // byte range of this half-row
+          if (kEpi == kEpiLatent && latent && c_hi == 7) {
+            bulk_store(dst_main + b0, stage_row + b0, 384 - b0);   // rest of c_kv
+            bulk_store(dst_rope, stage_row + 384, 64);             // k_rope
           } else {
-            bulk_store(dst_main, stage_row, BN * 2);
+            bulk_store(dst_main + b0, stage_row + b0, (c_hi - c_lo) * 64);
           }
           bulk_commit();
         }
@@ -354,6 +361,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     bulk_wait_all();
   }
 
+  __syncwarp();      // reconverge single-lane roles before the CTA-wide barrier
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
