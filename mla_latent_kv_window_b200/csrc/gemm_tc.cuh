@@ -9,10 +9,12 @@
 //   warp 2      TMA producer of B k-blocks into a B_STAGES-deep ring
 //   warp 1      TMEM allocator + single-thread tcgen05.mma issuer (M=128, N=BN, K=16 steps)
 //   warps 3..10 epilogue, two warps per TMEM lane quarter: each thread owns one row and one
-//               half of its 32-column chunks.  tcgen05.ld of the accumulator (the next chunk is
-//               loaded while the current one is converted), fused row transform into a padded
-//               shared-memory staging row, then one bulk async copy per contiguous destination
-//               segment of the half-row (c_kv / k_rope, Qp, or the output row).
+//               half of the tile's 32-column chunks.  tcgen05.ld of the accumulator (the next
+//               chunk is loaded while the current one is converted), fused column transform,
+//               16-bit pack into a 32 x 32 staging box per (chunk, quarter), then one TMA tensor
+//               store per box issued by the warp's lane 0.  The boxes use the 64-byte swizzle of
+//               the output tensor maps, which also makes the row-per-thread writes bank-conflict
+//               free; rows past the end of the launch are clipped by the maps' extents.
 // The rings run continuously across tile boundaries.  With M_SUB = 1 the accumulator is
 // double-buffered in TMEM (2 x 256 columns), so the epilogue of tile i overlaps the MMAs of
 // tile i+1.  With M_SUB = 2 a tile is 256 rows: two M=128 accumulators (TMEM columns [0,256)
@@ -22,14 +24,21 @@
 // A (activations, streamed once from HBM) and B (weights, shared by every CTA and L2-resident)
 // have separate rings so that A can run ahead of the short-latency B loads; each tile starts
 // its k-loop at a rotated block so concurrent CTAs do not all hit the same weight block.
+// Launched with programmatic stream serialization, the prologue (barrier init, TMEM
+// allocation, tensor-map prefetch) overlaps the previous kernel's tail; every global access
+// comes after grid_dependency_wait().
 
-// Epilogues (kEpi):
-//   kEpiStore   bf16 store of the tile into out[z][m][n]                (output projection)
-//   kEpiLatent  columns 0..191 -> c_kv, 192..223 -> RoPE3D -> k_rope, written as fp16 to ring
-//               slots (t mod W)*F + k, or to the chunk tail; for blockIdx.y below latent_y the
-//               tile is one head's absorbed query [W_UK^T q_nope | RoPE3D(q_rope)] * scale ->
-//               Qp (fp16).  The latent path is 16-bit like the paper's cache; fp16 keeps three
-//               more mantissa bits than bf16 for the same bytes.
+// Output columns.  Column block y of a launch covers global columns col = b_row0 + y*BN + [0,BN),
+// the same index that selects the rows of B.  Each 32-column chunk goes to one output map:
+//   kEpiStore   map_o0 (bf16 out[z][m][col])                            (output projection)
+//   kEpiLatent  col < latent_col0: one head's absorbed query
+//               [W_UK^T q_nope | RoPE3D(q_rope)] * scale -> map_o0 = Qp[z][m][col] (fp16);
+//               latent_col0 + [0,192) -> map_o1 = c_kv, latent_col0 + [192,224) -> RoPE3D ->
+//               map_o2 = k_rope (fp16), at rows dst_row0 + m of the cache planes (the host
+//               encodes the maps at the destination rows, so each launch writes one
+//               contiguous row range per stream).  The latent path is 16-bit like the paper's
+//               cache; fp16 keeps three more mantissa bits than bf16 for the same bytes.
+//   RoPE applies to the chunks with col mod 224 == 192 (every 224-column block is 192 + 32).
 //
 // The latent epilogue is the fused "append" of the VideoMLA paper page: c_kv = x W_DKV^T and
 // the decoupled positional key k_R = RoPE3D(x W_KR^T) (§3.1, §3.2), one head-shared copy per
@@ -55,25 +64,12 @@ struct RopeBands {
 };
 
 struct EpiArgs {
-  // kEpiStore
-  __nv_bfloat16* out;
-  int64_t out_batch_stride;  // elements
-  int32_t ld_out;            // elements per output row
-  // kEpiLatent
-  __half* ckv;               // [batch][rows_per_stream][192] fp16
-  __half* krope;             // [batch][rows_per_stream][32]  fp16
-  int64_t rows_per_stream;
-  __half* qp;                // [batch][qp_rows_per_stream][224] fp16
-  int64_t qp_rows_per_stream;
-  int32_t latent_y;          // blockIdx.y >= latent_y -> latent tile, else query head blockIdx.y
-  int32_t n_heads;
-  int32_t ring_mode;         // 1: slot (t mod W)*F + k; 0: chunk tail row base_row + m
-  int64_t t0;                // temporal index of row 0's frame
-  int32_t window_frames;
+  int32_t n_cols;            // global columns < n_cols are stored; the rest of a block is padding
+  int32_t latent_col0;       // kEpiLatent: first column of the latent block (a multiple of 224)
+  int64_t t0;                // kEpiLatent: temporal index of row 0's frame
   int32_t tokens_per_frame;
   int32_t frame_w;
-  int64_t base_row;
-  float q_scale;             // softmax_scale * log2(e)
+  float q_scale;             // softmax_scale * log2(e), applied to the query columns
   RopeBands rope;
 };
 
@@ -82,11 +78,11 @@ struct GemmSmem {
   static constexpr int kABytes = M_SUB * 128 * 64 * 2;
   static constexpr int kBBytes = BN * 64 * 2;
   static constexpr int kBOffset = A_STAGES * kABytes;
-  static constexpr int kStageStride = BN * 2 + 16;          // padded staging row (no bank conflicts)
-  static constexpr int kStagingOffset = kBOffset + B_STAGES * kBBytes;
-  static constexpr int kBarOffset = kStagingOffset + 128 * kStageStride;
+  static constexpr int kStagingOffset = kBOffset + B_STAGES * kBBytes;   // (BN/32) x 4 boxes of 2 KB
+  static constexpr int kBarOffset = kStagingOffset + 128 * BN * 2;
   static constexpr int kBytes = kBarOffset + 512 + 1024;    // barriers + alignment slack
   static_assert(kABytes % 1024 == 0 && kBBytes % 1024 == 0, "stage atoms must stay 1 KB aligned");
+  static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "column blocks are whole 32-column chunks");
   static_assert(kBytes <= 232448, "GEMM tile does not fit in shared memory");
 };
 
@@ -126,13 +122,15 @@ __device__ __forceinline__ void rope_rotate32(float* v, int64_t t, int h, int w,
 template <int BN, int A_STAGES, int B_STAGES, int kEpi, bool kF16In, int M_SUB>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
-                   const __grid_constant__ CUtensorMap map_b, int32_t M, int32_t K,
+                   const __grid_constant__ CUtensorMap map_b,
+                   const __grid_constant__ CUtensorMap map_o0,
+                   const __grid_constant__ CUtensorMap map_o1,
+                   const __grid_constant__ CUtensorMap map_o2, int32_t M, int32_t K,
                    int32_t b_row0, GemmTiles tiles, EpiArgs ep, int* status) {
   using L = GemmSmem<BN, A_STAGES, B_STAGES, M_SUB>;
   static_assert(M_SUB == 1 || M_SUB == 2, "tiles are 128 or 256 rows");
   constexpr int kAccBufs = M_SUB == 1 ? 2 : 1;   // accumulator buffers in 512 TMEM columns
   constexpr int kTileRows = 128 * M_SUB;
-  static_assert(kEpi != kEpiLatent || BN == 224, "the latent epilogue owns 192 + 32 columns");
   static_assert(BN <= 256, "one accumulator buffer holds at most 256 columns");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -153,6 +151,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                            ? (n_tiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
 
   if (threadIdx.x == 0) {
+    grid_launch_dependents();
     for (int s = 0; s < A_STAGES; ++s) {
       mbar_init(&a_full[s], 1);
       mbar_init(&a_empty[s], 1);
@@ -168,6 +167,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     fence_mbar_init();
     tma_prefetch(&map_a);
     tma_prefetch(&map_b);
+    tma_prefetch(&map_o0);
+    if (kEpi == kEpiLatent) {
+      tma_prefetch(&map_o1);
+      tma_prefetch(&map_o2);
+    }
   }
   if (warp == 1) {
     tmem_alloc(tmem_holder, 512);
@@ -178,6 +182,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
+  grid_dependency_wait();   // the previous kernel's outputs are visible from here on
 
   // Tile t -> (row tile, column block, batch); consecutive tiles share the column block.
   auto tile_coords = [&](int t, int& m0, int& y, int& z) {
@@ -258,59 +263,43 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
   } else {
     // ------------------------------------------------------------------ epilogue warps
-    const uint32_t sub_q = warp & 3u;          // TMEM lane quarter this warp may access
+    const uint32_t sub_q = warp & 3u;          // TMEM lane quarter = rows 32*sub_q.. of a sub-tile
     const int half = (int)(warp - 3) >> 2;     // 0: first half of the chunks, 1: second half
     constexpr int kChunks = BN / 32;
     constexpr int kSplit = (kChunks + 1) / 2;
     const int c_lo = half ? kSplit : 0;
     const int c_hi = half ? kChunks : kSplit;
     const int row = sub_q * 32 + lane;         // row of each 128-row sub-tile owned by this thread
-    uint8_t* stage_row = smem + L::kStagingOffset + row * L::kStageStride;
+    // Staging box (chunk c, quarter q) at (c*4 + q) * 2 KB: 32 rows of 64 B; 16-byte unit u of
+    // row r sits at slot u ^ ((r >> 1) & 3), the 64-byte swizzle of the output maps.
+    uint8_t* stage = smem + L::kStagingOffset;
+    const uint32_t swz = (lane >> 1) & 3u;
     for (int i = 0; i < my_tiles; ++i) {
       const int buf = i % kAccBufs;
       int m0t, y, z;
       tile_coords(blockIdx.x + i * gridDim.x, m0t, y, z);
       if (!mbar_wait_warp_sleepy(&acc_full[buf], (uint32_t)(i / kAccBufs) & 1u, status)) break;
       tc_fence_after();
+      const int col_base = b_row0 + y * BN;
 #pragma unroll 1
       for (int sub = 0; sub < M_SUB; ++sub) {
         const int m = m0t + sub * 128 + row;
-        const bool valid = m < M;
         const uint32_t tbase = tmem + (buf + sub) * 256 + ((sub_q * 32u) << 16);
-
-        // This thread's destination row, computed once per tile.
-        uint8_t* dst_main = nullptr;  // byte 0 of the row: c_kv (latent), Qp (query), out (store)
-        uint8_t* dst_rope = nullptr;  // latent rows: the k_rope row (columns [192, 224))
-        bool latent = false;
         int64_t t = 0;
         int hh = 0, ww = 0;
         if constexpr (kEpi == kEpiLatent) {
-          latent = y >= ep.latent_y;
           const int F = ep.tokens_per_frame;
-          const int fi = m / F;               // frame within this call
+          const int fi = m / F;               // frame within this launch
           const int k = m - fi * F;
           t = ep.t0 + fi;
           hh = k / ep.frame_w;
           ww = k - hh * ep.frame_w;
-          if (latent) {
-            const int64_t dst_row =
-                (ep.ring_mode ? (int64_t)(t % ep.window_frames) * F + k : ep.base_row + m) +
-                (int64_t)z * ep.rows_per_stream;
-            dst_main = reinterpret_cast<uint8_t*>(ep.ckv + dst_row * 192);
-            dst_rope = reinterpret_cast<uint8_t*>(ep.krope + dst_row * 32);
-          } else {
-            const int64_t qrow = (int64_t)z * ep.qp_rows_per_stream + (int64_t)m * ep.n_heads + y;
-            dst_main = reinterpret_cast<uint8_t*>(ep.qp + qrow * 224);
-          }
-        } else {
-          dst_main = reinterpret_cast<uint8_t*>(ep.out + z * ep.out_batch_stride +
-                                                (int64_t)m * ep.ld_out + y * BN);
         }
-
-        // The staging half-row is free once this thread's previous bulk copies have read it.
-        bulk_wait_read_all();
+        // The staging boxes are free once this warp's previous tensor stores have read them.
+        if (lane == 0) bulk_wait_read_all();
+        __syncwarp();
         uint32_t r[2][32];
-        tmem_ld32(tbase + c_lo * 32, r[0]);
+        if (c_lo < c_hi) tmem_ld32(tbase + c_lo * 32, r[0]);   // (BN = 32: half 1 owns nothing)
 #pragma unroll
         for (int cc = 0; cc < kSplit; ++cc) {
           const int c = c_lo + cc;
@@ -323,21 +312,24 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
           for (int q = 0; q < 32; ++q) v[q] = __uint_as_float(cur[q]);
           if constexpr (kEpi == kEpiLatent) {
-            if (c == 6) rope_rotate32(v, t, hh, ww, ep.rope);   // columns 192..223
-            if (!latent) {
+            const int col = col_base + c * 32;
+            if (col % 224 == 192) rope_rotate32(v, t, hh, ww, ep.rope);
+            if (col < ep.latent_col0) {
 #pragma unroll
               for (int q = 0; q < 32; ++q) v[q] *= ep.q_scale;
             }
           }
-          uint4* st4 = reinterpret_cast<uint4*>(stage_row + c * 64);
+          uint4* box = reinterpret_cast<uint4*>(stage + (c * 4 + sub_q) * 2048 + lane * 64);
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
+          for (int u = 0; u < 4; ++u) {
+            uint4 w;
             if constexpr (kEpi == kEpiLatent)
-              st4[q] = make_uint4(pack_f16x2(v[8 * q + 0], v[8 * q + 1]), pack_f16x2(v[8 * q + 2], v[8 * q + 3]),
-                                  pack_f16x2(v[8 * q + 4], v[8 * q + 5]), pack_f16x2(v[8 * q + 6], v[8 * q + 7]));
+              w = make_uint4(pack_f16x2(v[8 * u + 0], v[8 * u + 1]), pack_f16x2(v[8 * u + 2], v[8 * u + 3]),
+                             pack_f16x2(v[8 * u + 4], v[8 * u + 5]), pack_f16x2(v[8 * u + 6], v[8 * u + 7]));
             else
-              st4[q] = make_uint4(pack_bf16x2(v[8 * q + 0], v[8 * q + 1]), pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
-                                  pack_bf16x2(v[8 * q + 4], v[8 * q + 5]), pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
+              w = make_uint4(pack_bf16x2(v[8 * u + 0], v[8 * u + 1]), pack_bf16x2(v[8 * u + 2], v[8 * u + 3]),
+                             pack_bf16x2(v[8 * u + 4], v[8 * u + 5]), pack_bf16x2(v[8 * u + 6], v[8 * u + 7]));
+            box[u ^ swz] = w;
           }
         }
         if (sub == M_SUB - 1) {
@@ -345,20 +337,31 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           tc_fence_before();
           mbar_arrive(&acc_empty[buf]);
         }
-        if (valid) {
-          fence_proxy_async_smem();   // staging writes -> visible to the bulk-copy engine
-          const uint32_t b0 = c_lo * 64;                       // byte range of this half-row
-          if (kEpi == kEpiLatent && latent && c_hi == 7) {
-            bulk_store(dst_main + b0, stage_row + b0, 384 - b0);   // rest of c_kv
-            bulk_store(dst_rope, stage_row + 384, 64);             // k_rope
-          } else {
-            bulk_store(dst_main + b0, stage_row + b0, (c_hi - c_lo) * 64);
+        fence_proxy_async_smem();   // staging writes -> visible to the TMA engine
+        __syncwarp();
+        const int row0 = m0t + sub * 128 + (int)sub_q * 32;
+        if (lane == 0 && row0 < M) {
+          for (int c = c_lo; c < c_hi; ++c) {
+            const int col = col_base + c * 32;
+            if (col >= ep.n_cols) break;
+            const uint8_t* src = stage + (c * 4 + sub_q) * 2048;
+            if constexpr (kEpi == kEpiLatent) {
+              const int j = col - ep.latent_col0;
+              if (j < 0)
+                tma_store_3d(&map_o0, src, col, row0, z);
+              else if (j < 192)
+                tma_store_3d(&map_o1, src, j, row0, z);
+              else
+                tma_store_3d(&map_o2, src, j - 192, row0, z);
+            } else {
+              tma_store_3d(&map_o0, src, col, row0, z);
+            }
           }
           bulk_commit();
         }
       }
     }
-    bulk_wait_all();
+    if (lane == 0) bulk_wait_all();
   }
 
   __syncwarp();      // reconverge single-lane roles before the CTA-wide barrier

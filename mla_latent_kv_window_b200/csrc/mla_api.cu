@@ -7,7 +7,10 @@
 //        latent -> chunk tail rows (c_kv, RoPE3D k_rope)
 //   2. window_attn_kernel          o_lat[(q,h)] = softmax(Qp . [c_kv|k_rope]^T) c_kv
 //   3. tc_gemm<256, kEpiStore>    out = o_lat x W_OV^T,  W_OV[h] = W_O[:, h] W_UV[h]
-// An append is step 1's latent half written to ring slots (t mod W) * F + k.
+// An append is step 1's latent block alone, written to ring slots (t mod W) * F + k: one launch
+// per contiguous run of slots (two when the frames wrap around the end of the ring).
+// Every kernel of the path is launched with programmatic stream serialization, so its
+// prologue overlaps the tail of the kernel before it.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -17,6 +20,7 @@
 #include <cstring>
 #include <mutex>
 #include <string>
+#include <utility>
 #include <vector>
 
 #include "../../include/mla.h"
@@ -40,6 +44,8 @@ constexpr int kProjAStages = 5;     // 5 x 16 KB of hidden states in flight per 
 constexpr int kProjBStages = 3;     // 3 x 28 KB of L2-resident weights
 constexpr int kProjWideAStages = 3; // 256-row tiles: 3 x 32 KB of hidden states
 constexpr int kProjWideBStages = 2;
+constexpr int kProjNarrowAStages = 8;   // 32-column latent blocks: 8 x 16 KB + 4 x 4 KB
+constexpr int kProjNarrowBStages = 4;
 constexpr int kOutAStages = 5;
 constexpr int kOutBStages = 2;
 constexpr int kAttnStages = 4;      // 4 key tiles in flight (Q and P live in tensor memory)
@@ -106,6 +112,31 @@ mla_status make_map(CUtensorMap* map, const void* base, uint64_t inner, uint64_t
                 (int)r, (unsigned long long)inner, (unsigned long long)rows,
                 (unsigned long long)batch);
   return MLA_OK;
+}
+
+// Output map of a GEMM epilogue: 32 x 32 boxes with the 64-byte swizzle of its staging.
+mla_status make_out_map(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows,
+                        uint64_t batch, uint64_t row_bytes, uint64_t batch_bytes, bool f16) {
+  return make_map(map, base, inner, rows, batch, row_bytes, batch_bytes, 32, 32,
+                  CU_TENSOR_MAP_SWIZZLE_64B, f16);
+}
+
+// Launch with programmatic stream serialization (the kernel waits for its predecessor with
+// griddepcontrol.wait before touching global memory).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
 // ------------------------------------------------------------------------------ kernels
@@ -177,15 +208,18 @@ mla_status check_launch(const char* what) {
 
 // Persistent GEMM launch: one CTA per SM at most, each walking its share of the tiles.
 template <int BN, int SA, int SB, int EPI, bool F16, int M_SUB = 1>
-mla_status launch_gemm(const CUtensorMap& ma, const CUtensorMap& mb, int M, int K, int b_row0,
+mla_status launch_gemm(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& mo0,
+                       const CUtensorMap& mo1, const CUtensorMap& mo2, int M, int K, int b_row0,
                        mla::GemmTiles tiles, const EpiArgs& ep, int* status, int num_sms,
                        cudaStream_t st, const char* what) {
   const int n = tiles.count();
   if (n <= 0) return MLA_OK;
   const int grid = n < num_sms ? n : num_sms;
-  mla::tc_gemm_kernel<BN, SA, SB, EPI, F16, M_SUB>
-      <<<grid, mla::kGemmThreads, mla::GemmSmem<BN, SA, SB, M_SUB>::kBytes, st>>>(
-          ma, mb, M, K, b_row0, tiles, ep, status);
+  const cudaError_t e = launch_pdl(mla::tc_gemm_kernel<BN, SA, SB, EPI, F16, M_SUB>, dim3(grid),
+                                   dim3(mla::kGemmThreads),
+                                   mla::GemmSmem<BN, SA, SB, M_SUB>::kBytes, st, ma, mb, mo0, mo1,
+                                   mo2, M, K, b_row0, tiles, ep, status);
+  if (e != cudaSuccess) return fail(MLA_ERR_CUDA, "%s launch failed: %s", what, cudaGetErrorString(e));
   return check_launch(what);
 }
 
@@ -212,6 +246,7 @@ struct mla_cache {
   int* status = nullptr;
 
   CUtensorMap map_wqcat{};         // B operand of the projections: box 64 x 224
+  CUtensorMap map_wqcat32{};       // the same weights in 32-row boxes (32-column latent blocks)
   CUtensorMap map_wov{};           // B operand of the output projection: box 64 x out_bn
   int out_bn = 256;
 
@@ -274,47 +309,94 @@ RopeBands make_bands(const mla_config& cfg) {
   return rb;
 }
 
-// Launch the latent/query projection GEMM over `rows` rows of x per stream.  Query rows go to
-// `qp` (rows_per_stream qp_rows); launches with more 128-row tiles than SMs use 256-row tiles so
-// each weight k-block serves twice as many rows.
+// Launch the latent (and, with queries, the absorbed-query) projection GEMM over `rows` rows
+// of x per stream.  The latent rows land at cache rows [dst_row0, dst_row0 + rows) of every
+// stream; query rows go to qp ([batch][qp_tokens][n_heads * 224]).  Tile shape: 128-row tiles
+// while they fit the SMs in one wave, else 256-row tiles (each weight k-block then serves
+// twice as many rows); a latent-only launch with few row tiles splits its 224 columns into
+// seven 32-column blocks so that more SMs share the load.
 mla_status launch_latent_gemm(mla_cache* c, const void* x, int64_t rows, int64_t x_batch_rows,
-                              int grid_y, int latent_y, int b_row0, int ring_mode, int64_t t0,
-                              int64_t base_row, cudaStream_t st, __half* qp = nullptr,
-                              int64_t qp_rows = 0) {
+                              bool with_queries, int64_t t0, int64_t dst_row0, cudaStream_t st,
+                              __half* qp = nullptr, int64_t qp_tokens = 0) {
   const mla_config& cfg = c->cfg;
   const int64_t tiles128 = (rows + 127) / 128;
-  const bool wide = tiles128 * grid_y * cfg.batch > c->num_sms;
-  CUtensorMap map_x;
+  const int n_blocks224 = with_queries ? cfg.n_heads + 1 : 1;
+  const bool narrow_cols = !with_queries && tiles128 * 7 * cfg.batch <= c->num_sms;
+  const bool wide = !narrow_cols && tiles128 * n_blocks224 * cfg.batch > c->num_sms;
+  CUtensorMap map_x, map_ckv, map_krope, map_qp;
   mla_status s = make_map(&map_x, x, cfg.hidden, rows, cfg.batch, (uint64_t)cfg.hidden * 2,
                           (uint64_t)x_batch_rows * cfg.hidden * 2, 64, wide ? 256 : 128,
                           CU_TENSOR_MAP_SWIZZLE_128B);
   if (s != MLA_OK) return s;
+  const uint64_t plane_rows = (uint64_t)c->rows_per_stream;
+  if ((s = make_out_map(&map_ckv, c->ckv + dst_row0 * kLatent, kLatent, rows, cfg.batch,
+                        kLatent * 2, plane_rows * kLatent * 2, true)) != MLA_OK)
+    return s;
+  if ((s = make_out_map(&map_krope, c->krope + dst_row0 * kRope, kRope, rows, cfg.batch,
+                        kRope * 2, plane_rows * kRope * 2, true)) != MLA_OK)
+    return s;
+  if (with_queries) {
+    const uint64_t qcols = (uint64_t)cfg.n_heads * kQK;
+    if (!qp) {
+      qp = c->qp;
+      qp_tokens = c->max_q_tokens;
+    }
+    if ((s = make_out_map(&map_qp, qp, qcols, rows, cfg.batch, qcols * 2,
+                          (uint64_t)qp_tokens * qcols * 2, true)) != MLA_OK)
+      return s;
+  } else {
+    map_qp = map_ckv;   // no query columns in this launch
+  }
   EpiArgs ep{};
-  ep.ckv = c->ckv;
-  ep.krope = c->krope;
-  ep.rows_per_stream = c->rows_per_stream;
-  ep.qp = qp ? qp : c->qp;
-  ep.qp_rows_per_stream = qp ? qp_rows : c->max_q_tokens * cfg.n_heads;
-  ep.latent_y = latent_y;
-  ep.n_heads = cfg.n_heads;
-  ep.ring_mode = ring_mode;
+  ep.latent_col0 = cfg.n_heads * kQK;
+  ep.n_cols = (cfg.n_heads + 1) * kQK;
   ep.t0 = t0;
-  ep.window_frames = cfg.window_frames;
   ep.tokens_per_frame = c->F;
   ep.frame_w = cfg.frame_w;
-  ep.base_row = base_row;
   ep.q_scale = c->softmax_scale * 1.4426950408889634f;
   ep.rope = c->rope;
-  if (wide) {
-    const mla::GemmTiles tiles{(int32_t)((rows + 255) / 256), grid_y, cfg.batch};
-    return launch_gemm<kQK, kProjWideAStages, kProjWideBStages, mla::kEpiLatent, false, 2>(
-        map_x, c->map_wqcat, (int)rows, cfg.hidden, b_row0, tiles, ep, c->status, c->num_sms, st,
-        "latent projection");
+  const int b_row0 = with_queries ? 0 : cfg.n_heads * kQK;
+  if (narrow_cols) {
+    const mla::GemmTiles tiles{(int32_t)tiles128, kQK / 32, cfg.batch};
+    return launch_gemm<32, kProjNarrowAStages, kProjNarrowBStages, mla::kEpiLatent, false, 1>(
+        map_x, c->map_wqcat32, map_qp, map_ckv, map_krope, (int)rows, cfg.hidden, b_row0, tiles,
+        ep, c->status, c->num_sms, st, "latent projection");
   }
-  const mla::GemmTiles tiles{(int32_t)tiles128, grid_y, cfg.batch};
+  if (wide) {
+    const mla::GemmTiles tiles{(int32_t)((rows + 255) / 256), n_blocks224, cfg.batch};
+    return launch_gemm<kQK, kProjWideAStages, kProjWideBStages, mla::kEpiLatent, false, 2>(
+        map_x, c->map_wqcat, map_qp, map_ckv, map_krope, (int)rows, cfg.hidden, b_row0, tiles,
+        ep, c->status, c->num_sms, st, "latent projection");
+  }
+  const mla::GemmTiles tiles{(int32_t)tiles128, n_blocks224, cfg.batch};
   return launch_gemm<kQK, kProjAStages, kProjBStages, mla::kEpiLatent, false, 1>(
-      map_x, c->map_wqcat, (int)rows, cfg.hidden, b_row0, tiles, ep, c->status, c->num_sms, st,
-      "latent projection");
+      map_x, c->map_wqcat, map_qp, map_ckv, map_krope, (int)rows, cfg.hidden, b_row0, tiles, ep,
+      c->status, c->num_sms, st, "latent projection");
+}
+
+// Output projection out[z][m][:] = o_lat[z][m][:] W_OV^T over nq tokens per stream.
+mla_status launch_out_proj(mla_cache* c, const __half* o_lat, int64_t o_lat_tokens, int64_t nq,
+                           void* out, cudaStream_t st, const char* what) {
+  const mla_config& cfg = c->cfg;
+  CUtensorMap ma, mo;
+  mla_status s;
+  const uint64_t kin = (uint64_t)cfg.n_heads * kLatent;
+  if ((s = make_map(&ma, o_lat, kin, nq, cfg.batch, kin * 2, (uint64_t)o_lat_tokens * kin * 2,
+                    64, 128, CU_TENSOR_MAP_SWIZZLE_128B, true)) != MLA_OK)
+    return s;
+  if ((s = make_out_map(&mo, out, cfg.hidden, nq, cfg.batch, (uint64_t)cfg.hidden * 2,
+                        (uint64_t)nq * cfg.hidden * 2, false)) != MLA_OK)
+    return s;
+  EpiArgs ep{};
+  ep.n_cols = cfg.hidden;
+  const mla::GemmTiles tiles{(int32_t)((nq + 127) / 128), cfg.hidden / c->out_bn, cfg.batch};
+  if (c->out_bn == 256)
+    return launch_gemm<256, kOutAStages, kOutBStages, mla::kEpiStore, true>(
+        ma, c->map_wov, mo, mo, mo, (int)nq, (int)kin, 0, tiles, ep, c->status, c->num_sms, st,
+        what);
+  return launch_gemm<128, kOutAStages, kOutBStages, mla::kEpiStore, true>(
+      ma, c->map_wov, mo, mo, mo, (int)nq, (int)kin, 0, tiles, ep, c->status, c->num_sms, st,
+      what);
 }
 
 // Window attention of R query rows per stream over keys [0, n_keys) of every stream's ring.
@@ -342,8 +424,10 @@ mla_status launch_attention(mla_cache* c, const __half* qp, int64_t qp_batch_str
   using Sm = mla::AttnSmem<kAttnStages>;
   dim3 grid((unsigned)((R + 127) / 128), (unsigned)cfg.batch);
   ProfScope p(c, MLA_KERNEL_ATTENTION, st, profile);
-  mla::window_attn_kernel<kAttnStages><<<grid, mla::kAttnThreads, Sm::kBytes, st>>>(mkc, mkr, a,
-                                                                                   c->status);
+  const cudaError_t e = launch_pdl(mla::window_attn_kernel<kAttnStages>, grid,
+                                   dim3(mla::kAttnThreads), Sm::kBytes, st, mkc, mkr, a, c->status);
+  if (e != cudaSuccess)
+    return fail(MLA_ERR_CUDA, "window attention launch failed: %s", cudaGetErrorString(e));
   return check_launch("window attention");
 }
 
@@ -593,6 +677,10 @@ mla_status mla_cache_create(const mla_config* cfg, const mla_weights* w, void* s
                (uint64_t)k.hidden * 2, (uint64_t)(k.n_heads + 1) * kQK * k.hidden * 2, 64, kQK,
                CU_TENSOR_MAP_SWIZZLE_128B);
   if (s != MLA_OK) return cleanup(s);
+  s = make_map(&c->map_wqcat32, c->wqcat, k.hidden, (uint64_t)(k.n_heads + 1) * kQK, 1,
+               (uint64_t)k.hidden * 2, (uint64_t)(k.n_heads + 1) * kQK * k.hidden * 2, 64, 32,
+               CU_TENSOR_MAP_SWIZZLE_128B);
+  if (s != MLA_OK) return cleanup(s);
   s = make_map(&c->map_wov, c->wov, (uint64_t)k.n_heads * kLatent, k.hidden, 1,
                (uint64_t)k.n_heads * kLatent * 2, (uint64_t)k.hidden * k.n_heads * kLatent * 2,
                64, c->out_bn, CU_TENSOR_MAP_SWIZZLE_128B, true);
@@ -606,6 +694,9 @@ mla_status mla_cache_create(const mla_config* cfg, const mla_weights* w, void* s
     if (r == MLA_OK)
       r = set_smem(mla::tc_gemm_kernel<kQK, kProjWideAStages, kProjWideBStages, mla::kEpiLatent, false, 2>,
                    mla::GemmSmem<kQK, kProjWideAStages, kProjWideBStages, 2>::kBytes);
+    if (r == MLA_OK)
+      r = set_smem(mla::tc_gemm_kernel<32, kProjNarrowAStages, kProjNarrowBStages, mla::kEpiLatent, false, 1>,
+                   mla::GemmSmem<32, kProjNarrowAStages, kProjNarrowBStages, 1>::kBytes);
     if (r == MLA_OK)
       r = set_smem(mla::tc_gemm_kernel<256, kOutAStages, kOutBStages, mla::kEpiStore, true, 1>,
                    mla::GemmSmem<256, kOutAStages, kOutBStages>::kBytes);
@@ -633,14 +724,24 @@ mla_status mla_cache_append(mla_cache* c, const void* x, int32_t n_frames, void*
     return fail(MLA_ERR_INVALID_ARGUMENT, "too many frames in one append");
   const mla_config& cfg = c->cfg;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  // Only the last W frames of a long append survive in the ring.
   const int skip = n_frames > cfg.window_frames ? n_frames - cfg.window_frames : 0;
-  const int64_t rows = (int64_t)(n_frames - skip) * c->F;
-  const void* x0 = static_cast<const __nv_bfloat16*>(x) + (int64_t)skip * c->F * cfg.hidden;
-  mla_status s;
+  const int64_t x_batch_rows = (int64_t)n_frames * c->F;
+  mla_status s = MLA_OK;
   {
     ProfScope p(c, MLA_KERNEL_APPEND, st);
-    s = launch_latent_gemm(c, x0, rows, (int64_t)n_frames * c->F, 1, 0, cfg.n_heads * kQK, 1,
-                           c->frames_appended + skip, 0, st);
+    // Frames t go to slots (t mod W): one launch per run of consecutive slots.
+    int64_t t = c->frames_appended + skip;
+    int64_t left = n_frames - skip;
+    const __nv_bfloat16* xp = static_cast<const __nv_bfloat16*>(x) + (int64_t)skip * c->F * cfg.hidden;
+    while (left > 0 && s == MLA_OK) {
+      const int64_t slot = t % cfg.window_frames;
+      const int64_t nf = left < cfg.window_frames - slot ? left : cfg.window_frames - slot;
+      s = launch_latent_gemm(c, xp, nf * c->F, x_batch_rows, false, t, slot * c->F, st);
+      xp += nf * c->F * cfg.hidden;
+      t += nf;
+      left -= nf;
+    }
   }
   if (s != MLA_OK) return s;
   c->frames_appended += n_frames;
@@ -667,8 +768,7 @@ mla_status mla_window_attention(mla_cache* c, const void* x_chunk, int32_t n_fra
   // 1. absorbed queries + chunk latents (one GEMM over [heads | latent] column blocks)
   {
     ProfScope p(c, MLA_KERNEL_QPROJ, st);
-    s = launch_latent_gemm(c, x_chunk, nq, nq, cfg.n_heads + 1, cfg.n_heads, 0, 0,
-                           c->frames_appended, base_row, st);
+    s = launch_latent_gemm(c, x_chunk, nq, nq, true, c->frames_appended, base_row, st);
   }
   if (s != MLA_OK) return s;
 
@@ -683,29 +783,10 @@ mla_status mla_window_attention(mla_cache* c, const void* x_chunk, int32_t n_fra
 
   // 3. output projection out = o_lat W_OV^T
   {
-    CUtensorMap ma;
-    const uint64_t kin = (uint64_t)cfg.n_heads * kLatent;
-    if ((s = make_map(&ma, c->o_lat, kin, nq, cfg.batch, kin * 2,
-                      (uint64_t)c->max_q_tokens * kin * 2, 64, 128,
-                      CU_TENSOR_MAP_SWIZZLE_128B, true)) != MLA_OK)
-      return s;
-    EpiArgs ep{};
-    ep.out = static_cast<__nv_bfloat16*>(out);
-    ep.out_batch_stride = nq * cfg.hidden;
-    ep.ld_out = cfg.hidden;
     ProfScope p(c, MLA_KERNEL_OPROJ, st);
-    const mla::GemmTiles tiles{(int32_t)((nq + 127) / 128), cfg.hidden / c->out_bn, cfg.batch};
-    if (c->out_bn == 256)
-      s = launch_gemm<256, kOutAStages, kOutBStages, mla::kEpiStore, true>(
-          ma, c->map_wov, (int)nq, (int)kin, 0, tiles, ep, c->status, c->num_sms, st,
-          "output projection");
-    else
-      s = launch_gemm<128, kOutAStages, kOutBStages, mla::kEpiStore, true>(
-          ma, c->map_wov, (int)nq, (int)kin, 0, tiles, ep, c->status, c->num_sms, st,
-          "output projection");
-    if (s != MLA_OK) return s;
+    s = launch_out_proj(c, c->o_lat, c->max_q_tokens, nq, out, st, "output projection");
   }
-  return MLA_OK;
+  return s;
 }
 
 mla_status mla_window_attention_noalloc(mla_cache* c, const void* x_chunk, int32_t n_frames,
@@ -744,35 +825,14 @@ mla_status mla_window_attention_noalloc(mla_cache* c, const void* x_chunk, int32
   const int64_t n_keys = base_row + nq;
 
   // 1. absorbed queries (into the scratch) + chunk latents (into the cache's chunk tail)
-  if ((s = launch_latent_gemm(c, x_chunk, nq, nq, cfg.n_heads + 1, cfg.n_heads, 0, 0,
-                              c->frames_appended, base_row, st, qp, R)) != MLA_OK)
+  if ((s = launch_latent_gemm(c, x_chunk, nq, nq, true, c->frames_appended, base_row, st, qp,
+                              nq)) != MLA_OK)
     return s;
   // 2. window attention, o_lat into the scratch
   if ((s = launch_attention(c, qp, R * kQK, R, n_keys, o_lat, R * kLatent, st, false)) != MLA_OK)
     return s;
   // 3. output projection from the scratch o_lat
-  {
-    CUtensorMap ma;
-    const uint64_t kin = (uint64_t)cfg.n_heads * kLatent;
-    if ((s = make_map(&ma, o_lat, kin, nq, cfg.batch, kin * 2, (uint64_t)nq * kin * 2, 64, 128,
-                      CU_TENSOR_MAP_SWIZZLE_128B, true)) != MLA_OK)
-      return s;
-    EpiArgs ep{};
-    ep.out = static_cast<__nv_bfloat16*>(out);
-    ep.out_batch_stride = nq * cfg.hidden;
-    ep.ld_out = cfg.hidden;
-    const mla::GemmTiles tiles{(int32_t)((nq + 127) / 128), cfg.hidden / c->out_bn, cfg.batch};
-    if (c->out_bn == 256)
-      s = launch_gemm<256, kOutAStages, kOutBStages, mla::kEpiStore, true>(
-          ma, c->map_wov, (int)nq, (int)kin, 0, tiles, ep, c->status, c->num_sms, st,
-          "no-alloc output projection");
-    else
-      s = launch_gemm<128, kOutAStages, kOutBStages, mla::kEpiStore, true>(
-          ma, c->map_wov, (int)nq, (int)kin, 0, tiles, ep, c->status, c->num_sms, st,
-          "no-alloc output projection");
-    if (s != MLA_OK) return s;
-  }
-  return MLA_OK;
+  return launch_out_proj(c, o_lat, nq, nq, out, st, "no-alloc output projection");
 }
 
 mla_status mla_dense_attention(const void* q, const void* k, const void* v, void* out,

@@ -107,6 +107,18 @@ __device__ __forceinline__ bool mbar_wait_warp_sleepy(uint64_t* bar, uint32_t pa
   return ok != 0;
 }
 
+// Programmatic dependent launch.  A kernel launched with programmatic stream serialization may
+// start while its predecessor in the stream is still running; grid_dependency_wait() returns
+// once the predecessor has completed and its memory operations are visible, so every global
+// access that may touch the predecessor's data comes after it.  launch_dependents() lets the
+// next such kernel start its own prologue early.  Both are no-ops for a normal launch.
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void grid_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // Named barrier over a subset of warps (id 1..15; id 0 is __syncthreads).
 __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
@@ -151,6 +163,14 @@ __device__ __forceinline__ uint64_t l2_policy_evict_last() {
 __device__ __forceinline__ void bulk_store(void* gdst, const void* ssrc, uint32_t bytes) {
   asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst),
                "r"(smem_u32(ssrc)), "r"(bytes)
+               : "memory");
+}
+// 3-D tiled store of one shared-memory box to global memory (rows and columns outside the
+// tensor map's extent are not written), tracked by the issuing thread's bulk async-group.
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void* src, int32_t c0,
+                                             int32_t c1, int32_t c2) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];"
+               ::"l"(map), "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2)
                : "memory");
 }
 __device__ __forceinline__ void bulk_commit() {

@@ -97,6 +97,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const int rot = (int)(((unsigned)blockIdx.x * 37u + (unsigned)blockIdx.y * 11u) % (unsigned)nt);
 
   if (threadIdx.x == 0) {
+    grid_launch_dependents();
     mbar_init(q_ready, 128);
     for (int s = 0; s < KV_STAGES; ++s) {
       mbar_init(&kv_full[s], 1);
@@ -119,6 +120,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
+  grid_dependency_wait();   // the projection's Qp and chunk latents are visible from here on
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
