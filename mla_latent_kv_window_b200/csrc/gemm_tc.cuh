@@ -71,6 +71,8 @@ struct EpiArgs {
   int32_t frame_w;
   float q_scale;             // softmax_scale * log2(e), applied to the query columns
   RopeBands rope;
+  const float2* rope_hw;     // (cos, sin) tables: [frame_h][16] for h, then [frame_w][16] for w
+  int32_t frame_h;
 };
 
 template <int BN, int A_STAGES, int B_STAGES, int M_SUB = 1>
@@ -92,27 +94,35 @@ struct GemmTiles {
   __host__ __device__ int32_t count() const { return m_tiles * n_blocks * batch; }
 };
 
-// Rotate the 16 (re, im) pairs of v by pos * freq.  The angle is formed as p + e with
-// p = fl(pos * hi), e = (pos * hi - p) + pos * lo (exact product error by FMA), then reduced to
-// [-pi, pi] by Cody-Waite reduction with 2 pi split into two floats (accurate for integer
-// positions below 2^24), and evaluated with the hardware sine/cosine.
-__device__ __forceinline__ void rope_rotate32(float* v, int64_t t, int h, int w,
-                                              const RopeBands& rb) {
+// Rotate the 16 (re, im) pairs of v: pair p by pos[axis[p]] * freq[p].  The h and w factors
+// (cos, sin) come from tables tab_h / tab_w (16 pairs per position, computed in double on the
+// host and rounded once).  The t factors are formed here: the angle is p + e with
+// p = fl(t * hi), e = (t * hi - p) + t * lo (exact product error by FMA), reduced to [-pi, pi]
+// by Cody-Waite reduction with 2 pi split into two floats (accurate for integer t below
+// 2^24), and evaluated with the hardware sine/cosine.
+__device__ __forceinline__ void rope_rotate32(float* v, int64_t t, const float2* tab_h,
+                                              const float2* tab_w, const RopeBands& rb) {
   constexpr float kInv2Pi = 0.15915494309189535f;
   constexpr float kTwoPiHi = 6.28318548202514648f;       // fl(2 pi)
   constexpr float kTwoPiLo = -1.7484556000744e-07f;      // 2 pi - fl(2 pi)
+  const float tf = (float)t;
 #pragma unroll
   for (int p = 0; p < 16; ++p) {
     const int ax = rb.axis[p];
-    const float pos = ax == 0 ? (float)t : (ax == 1 ? (float)h : (float)w);
-    const float hi = rb.freq_hi[p];
-    const float prod = pos * hi;
-    const float err = fmaf(pos, hi, -prod) + pos * rb.freq_lo[p];
-    const float k = rintf(prod * kInv2Pi);
-    float r = fmaf(-k, kTwoPiHi, prod);
-    r = fmaf(-k, kTwoPiLo, r) + err;
     float sn, cs;
-    __sincosf(r, &sn, &cs);
+    if (ax == 0) {
+      const float hi = rb.freq_hi[p];
+      const float prod = tf * hi;
+      const float err = fmaf(tf, hi, -prod) + tf * rb.freq_lo[p];
+      const float k = rintf(prod * kInv2Pi);
+      float r = fmaf(-k, kTwoPiHi, prod);
+      r = fmaf(-k, kTwoPiLo, r) + err;
+      __sincosf(r, &sn, &cs);
+    } else {
+      const float2 f = __ldg((ax == 1 ? tab_h : tab_w) + p);
+      cs = f.x;
+      sn = f.y;
+    }
     const float a = v[2 * p], b = v[2 * p + 1];
     v[2 * p] = a * cs - b * sn;
     v[2 * p + 1] = a * sn + b * cs;
@@ -286,14 +296,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const int m = m0t + sub * 128 + row;
         const uint32_t tbase = tmem + (buf + sub) * 256 + ((sub_q * 32u) << 16);
         int64_t t = 0;
-        int hh = 0, ww = 0;
+        const float2* tab_h = nullptr;
+        const float2* tab_w = nullptr;
         if constexpr (kEpi == kEpiLatent) {
           const int F = ep.tokens_per_frame;
           const int fi = m / F;               // frame within this launch
           const int k = m - fi * F;
           t = ep.t0 + fi;
-          hh = k / ep.frame_w;
-          ww = k - hh * ep.frame_w;
+          const int hh = k / ep.frame_w;
+          tab_h = ep.rope_hw + hh * 16;
+          tab_w = ep.rope_hw + (ep.frame_h + k - hh * ep.frame_w) * 16;
         }
         // The staging boxes are free once this warp's previous tensor stores have read them.
         if (lane == 0) bulk_wait_read_all();
@@ -313,7 +325,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           for (int q = 0; q < 32; ++q) v[q] = __uint_as_float(cur[q]);
           if constexpr (kEpi == kEpiLatent) {
             const int col = col_base + c * 32;
-            if (col % 224 == 192) rope_rotate32(v, t, hh, ww, ep.rope);
+            if (col % 224 == 192) rope_rotate32(v, t, tab_h, tab_w, ep.rope);
             if (col < ep.latent_col0) {
 #pragma unroll
               for (int q = 0; q < 32; ++q) v[q] *= ep.q_scale;

@@ -46,8 +46,23 @@ constexpr int kProjWideAStages = 3; // 256-row tiles: 3 x 32 KB of hidden states
 constexpr int kProjWideBStages = 2;
 constexpr int kProjNarrowAStages = 8;   // 32-column latent blocks: 8 x 16 KB + 4 x 4 KB
 constexpr int kProjNarrowBStages = 4;
+constexpr int kProjMidAStages = 3;      // 256 x 160 tiles: 3 x 32 KB + 3 x 20 KB
+constexpr int kProjMidBStages = 3;
+constexpr int kOutBN = 192;             // output projection column block
 constexpr int kOutAStages = 5;
-constexpr int kOutBStages = 2;
+constexpr int kOutBStages = 3;
+
+// Tile shapes of the projection GEMMs with the steady-state time of one 64-wide k-block in
+// microseconds, measured on B200 for one CTA per SM.  A 128-row tile is held back by the
+// per-SM rate of its activation stream, so its k-block time barely depends on BN; a 256-row
+// tile moves twice the activations per k-block.  A launch picks the shape with the smallest
+// (waves of tiles) x (k-blocks) x (k-block time).
+struct TileShape {
+  int bn, m_sub;
+  double kb_us;
+};
+constexpr TileShape kShapeQ224{224, 1, 0.39}, kShapeQ160W{160, 2, 0.534},
+    kShapeQ224W{224, 2, 0.597}, kShapeL32{32, 1, 0.375};
 constexpr int kAttnStages = 4;      // 4 key tiles in flight (Q and P live in tensor memory)
 
 thread_local std::string g_last_error;
@@ -243,12 +258,13 @@ struct mla_cache {
   __half* o_lat = nullptr;         // fp16 P . c_kv
   __nv_bfloat16* wqcat = nullptr;  // bf16: multiplies the caller's bf16 hidden states
   __half* wov = nullptr;           // fp16: multiplies o_lat
+  float2* rope_hw = nullptr;       // RoPE (cos, sin) of the h and w bands, [frame_h + frame_w][16]
   int* status = nullptr;
 
   CUtensorMap map_wqcat{};         // B operand of the projections: box 64 x 224
-  CUtensorMap map_wqcat32{};       // the same weights in 32-row boxes (32-column latent blocks)
-  CUtensorMap map_wov{};           // B operand of the output projection: box 64 x out_bn
-  int out_bn = 256;
+  CUtensorMap map_wqcat160{};      // the same weights in 160-row boxes
+  CUtensorMap map_wqcat32{};       // ... and in 32-row boxes (32-column latent blocks)
+  CUtensorMap map_wov{};           // B operand of the output projection: box 64 x 192
 
   bool profiling = false;
   struct Rec {
@@ -309,23 +325,59 @@ RopeBands make_bands(const mla_config& cfg) {
   return rb;
 }
 
+// (cos, sin) of the h and w RoPE bands for every h in [0, frame_h) and w in [0, frame_w),
+// evaluated in double and rounded once: rows [0, frame_h) hold h, rows [frame_h, frame_h +
+// frame_w) hold w, 16 pairs each (pairs of the other axes hold (1, 0)).
+std::vector<float2> make_rope_hw(const mla_config& cfg) {
+  std::vector<float2> tab((size_t)(cfg.frame_h + cfg.frame_w) * 16, make_float2(1.f, 0.f));
+  int p = 0;
+  const int dims[3] = {cfg.rope_t, cfg.rope_h, cfg.rope_w};
+  for (int a = 0; a < 3; ++a)
+    for (int i = 0; i < dims[a] / 2; ++i, ++p) {
+      const double f = std::pow(cfg.rope_base, -2.0 * i / dims[a]);
+      if (a == 1)
+        for (int h = 0; h < cfg.frame_h; ++h)
+          tab[(size_t)h * 16 + p] = make_float2((float)std::cos(h * f), (float)std::sin(h * f));
+      if (a == 2)
+        for (int w = 0; w < cfg.frame_w; ++w)
+          tab[(size_t)(cfg.frame_h + w) * 16 + p] =
+              make_float2((float)std::cos(w * f), (float)std::sin(w * f));
+    }
+  return tab;
+}
+
 // Launch the latent (and, with queries, the absorbed-query) projection GEMM over `rows` rows
 // of x per stream.  The latent rows land at cache rows [dst_row0, dst_row0 + rows) of every
-// stream; query rows go to qp ([batch][qp_tokens][n_heads * 224]).  Tile shape: 128-row tiles
-// while they fit the SMs in one wave, else 256-row tiles (each weight k-block then serves
-// twice as many rows); a latent-only launch with few row tiles splits its 224 columns into
-// seven 32-column blocks so that more SMs share the load.
+// stream; query rows go to qp ([batch][qp_tokens][n_heads * 224]).  The tile shape is the
+// TileShape candidate with the least estimated time: with queries 128 x 224, 256 x 160 or
+// 256 x 224 tiles; latent only 128 x 32 (seven column blocks, so that a one-frame append
+// spreads over 91 SMs instead of 13), 128 x 224 or 256 x 224.
 mla_status launch_latent_gemm(mla_cache* c, const void* x, int64_t rows, int64_t x_batch_rows,
                               bool with_queries, int64_t t0, int64_t dst_row0, cudaStream_t st,
                               __half* qp = nullptr, int64_t qp_tokens = 0) {
   const mla_config& cfg = c->cfg;
-  const int64_t tiles128 = (rows + 127) / 128;
-  const int n_blocks224 = with_queries ? cfg.n_heads + 1 : 1;
-  const bool narrow_cols = !with_queries && tiles128 * 7 * cfg.batch <= c->num_sms;
-  const bool wide = !narrow_cols && tiles128 * n_blocks224 * cfg.batch > c->num_sms;
+  const int n_cols = with_queries ? (cfg.n_heads + 1) * kQK : kQK;   // columns of this launch
+  const int num_kb = cfg.hidden / 64;
+  // Pick the tile shape with the least estimated time (waves x k-blocks x k-block time).
+  auto tiles_of = [&](const TileShape& t) {
+    return mla::GemmTiles{(int32_t)((rows + 128 * t.m_sub - 1) / (128 * t.m_sub)),
+                          (n_cols + t.bn - 1) / t.bn, cfg.batch};
+  };
+  auto cost = [&](const TileShape& t) {
+    const int64_t n = tiles_of(t).count();
+    return (double)((n + c->num_sms - 1) / c->num_sms) * num_kb * t.kb_us;
+  };
+  const TileShape cands_q[3] = {kShapeQ224, kShapeQ160W, kShapeQ224W};
+  const TileShape cands_l[3] = {kShapeL32, kShapeQ224, kShapeQ224W};
+  const TileShape* cands = with_queries ? cands_q : cands_l;
+  TileShape shape = cands[0];
+  for (int i = 1; i < 3; ++i)
+    if (cost(cands[i]) < cost(shape)) shape = cands[i];
+  const mla::GemmTiles tiles = tiles_of(shape);
+
   CUtensorMap map_x, map_ckv, map_krope, map_qp;
   mla_status s = make_map(&map_x, x, cfg.hidden, rows, cfg.batch, (uint64_t)cfg.hidden * 2,
-                          (uint64_t)x_batch_rows * cfg.hidden * 2, 64, wide ? 256 : 128,
+                          (uint64_t)x_batch_rows * cfg.hidden * 2, 64, 128 * shape.m_sub,
                           CU_TENSOR_MAP_SWIZZLE_128B);
   if (s != MLA_OK) return s;
   const uint64_t plane_rows = (uint64_t)c->rows_per_stream;
@@ -355,23 +407,25 @@ mla_status launch_latent_gemm(mla_cache* c, const void* x, int64_t rows, int64_t
   ep.frame_w = cfg.frame_w;
   ep.q_scale = c->softmax_scale * 1.4426950408889634f;
   ep.rope = c->rope;
+  ep.rope_hw = c->rope_hw;
+  ep.frame_h = cfg.frame_h;
   const int b_row0 = with_queries ? 0 : cfg.n_heads * kQK;
-  if (narrow_cols) {
-    const mla::GemmTiles tiles{(int32_t)tiles128, kQK / 32, cfg.batch};
+  const char* what = "latent projection";
+  if (shape.bn == 32)
     return launch_gemm<32, kProjNarrowAStages, kProjNarrowBStages, mla::kEpiLatent, false, 1>(
         map_x, c->map_wqcat32, map_qp, map_ckv, map_krope, (int)rows, cfg.hidden, b_row0, tiles,
-        ep, c->status, c->num_sms, st, "latent projection");
-  }
-  if (wide) {
-    const mla::GemmTiles tiles{(int32_t)((rows + 255) / 256), n_blocks224, cfg.batch};
+        ep, c->status, c->num_sms, st, what);
+  if (shape.bn == 160)
+    return launch_gemm<160, kProjMidAStages, kProjMidBStages, mla::kEpiLatent, false, 2>(
+        map_x, c->map_wqcat160, map_qp, map_ckv, map_krope, (int)rows, cfg.hidden, b_row0, tiles,
+        ep, c->status, c->num_sms, st, what);
+  if (shape.m_sub == 2)
     return launch_gemm<kQK, kProjWideAStages, kProjWideBStages, mla::kEpiLatent, false, 2>(
         map_x, c->map_wqcat, map_qp, map_ckv, map_krope, (int)rows, cfg.hidden, b_row0, tiles,
-        ep, c->status, c->num_sms, st, "latent projection");
-  }
-  const mla::GemmTiles tiles{(int32_t)tiles128, n_blocks224, cfg.batch};
+        ep, c->status, c->num_sms, st, what);
   return launch_gemm<kQK, kProjAStages, kProjBStages, mla::kEpiLatent, false, 1>(
       map_x, c->map_wqcat, map_qp, map_ckv, map_krope, (int)rows, cfg.hidden, b_row0, tiles, ep,
-      c->status, c->num_sms, st, "latent projection");
+      c->status, c->num_sms, st, what);
 }
 
 // Output projection out[z][m][:] = o_lat[z][m][:] W_OV^T over nq tokens per stream.
@@ -389,12 +443,9 @@ mla_status launch_out_proj(mla_cache* c, const __half* o_lat, int64_t o_lat_toke
     return s;
   EpiArgs ep{};
   ep.n_cols = cfg.hidden;
-  const mla::GemmTiles tiles{(int32_t)((nq + 127) / 128), cfg.hidden / c->out_bn, cfg.batch};
-  if (c->out_bn == 256)
-    return launch_gemm<256, kOutAStages, kOutBStages, mla::kEpiStore, true>(
-        ma, c->map_wov, mo, mo, mo, (int)nq, (int)kin, 0, tiles, ep, c->status, c->num_sms, st,
-        what);
-  return launch_gemm<128, kOutAStages, kOutBStages, mla::kEpiStore, true>(
+  const mla::GemmTiles tiles{(int32_t)((nq + 127) / 128), (cfg.hidden + kOutBN - 1) / kOutBN,
+                             cfg.batch};
+  return launch_gemm<kOutBN, kOutAStages, kOutBStages, mla::kEpiStore, true>(
       ma, c->map_wov, mo, mo, mo, (int)nq, (int)kin, 0, tiles, ep, c->status, c->num_sms, st,
       what);
 }
@@ -586,6 +637,7 @@ size_t mla_cache_device_bytes(const mla_config* cfg) {
   b += (size_t)(c.n_heads + 1) * kQK * c.hidden * 2;       // Wqcat
   b += (size_t)c.hidden * c.n_heads * kLatent * 2;         // W_OV
   b += 256;                                                // status word
+  b += (size_t)(c.frame_h + c.frame_w) * 16 * 8;           // RoPE h / w tables
   return b;
 }
 
@@ -603,6 +655,7 @@ void mla_cache_destroy(mla_cache* c) {
   cudaFree(c->o_lat);
   cudaFree(c->wqcat);
   cudaFree(c->wov);
+  cudaFree(c->rope_hw);
   cudaFree(c->status);
   delete c;
 }
@@ -626,7 +679,6 @@ mla_status mla_cache_create(const mla_config* cfg, const mla_weights* w, void* s
                          ? cfg->softmax_scale
                          : (float)(1.0 / std::sqrt((double)(cfg->d_nope + cfg->d_rope)));
   c->rope = make_bands(*cfg);
-  c->out_bn = cfg->hidden % 256 == 0 ? 256 : 128;
   cudaGetDevice(&c->device);
   if (cudaDeviceGetAttribute(&c->num_sms, cudaDevAttrMultiProcessorCount, c->device) != cudaSuccess ||
       c->num_sms <= 0)
@@ -654,6 +706,10 @@ mla_status mla_cache_create(const mla_config* cfg, const mla_weights* w, void* s
   MLA_TRY(cudaMalloc(&c->wqcat, (size_t)(k.n_heads + 1) * kQK * k.hidden * 2));
   MLA_TRY(cudaMalloc(&c->wov, (size_t)k.hidden * k.n_heads * kLatent * 2));
   MLA_TRY(cudaMalloc(&c->status, 256));
+  const std::vector<float2> rope_hw = make_rope_hw(k);
+  MLA_TRY(cudaMalloc(&c->rope_hw, rope_hw.size() * sizeof(float2)));
+  MLA_TRY(cudaMemcpyAsync(c->rope_hw, rope_hw.data(), rope_hw.size() * sizeof(float2),
+                          cudaMemcpyHostToDevice, st));
   MLA_TRY(cudaMemsetAsync(c->ckv, 0, ring_rows * kLatent * 2, st));
   MLA_TRY(cudaMemsetAsync(c->krope, 0, ring_rows * kRope * 2, st));
   MLA_TRY(cudaMemsetAsync(c->qp, 0, q_rows * k.n_heads * kQK * 2, st));
@@ -677,13 +733,17 @@ mla_status mla_cache_create(const mla_config* cfg, const mla_weights* w, void* s
                (uint64_t)k.hidden * 2, (uint64_t)(k.n_heads + 1) * kQK * k.hidden * 2, 64, kQK,
                CU_TENSOR_MAP_SWIZZLE_128B);
   if (s != MLA_OK) return cleanup(s);
+  s = make_map(&c->map_wqcat160, c->wqcat, k.hidden, (uint64_t)(k.n_heads + 1) * kQK, 1,
+               (uint64_t)k.hidden * 2, (uint64_t)(k.n_heads + 1) * kQK * k.hidden * 2, 64, 160,
+               CU_TENSOR_MAP_SWIZZLE_128B);
+  if (s != MLA_OK) return cleanup(s);
   s = make_map(&c->map_wqcat32, c->wqcat, k.hidden, (uint64_t)(k.n_heads + 1) * kQK, 1,
                (uint64_t)k.hidden * 2, (uint64_t)(k.n_heads + 1) * kQK * k.hidden * 2, 64, 32,
                CU_TENSOR_MAP_SWIZZLE_128B);
   if (s != MLA_OK) return cleanup(s);
   s = make_map(&c->map_wov, c->wov, (uint64_t)k.n_heads * kLatent, k.hidden, 1,
                (uint64_t)k.n_heads * kLatent * 2, (uint64_t)k.hidden * k.n_heads * kLatent * 2,
-               64, c->out_bn, CU_TENSOR_MAP_SWIZZLE_128B, true);
+               64, kOutBN, CU_TENSOR_MAP_SWIZZLE_128B, true);
   if (s != MLA_OK) return cleanup(s);
 
   static std::once_flag attr_once;
@@ -695,14 +755,14 @@ mla_status mla_cache_create(const mla_config* cfg, const mla_weights* w, void* s
       r = set_smem(mla::tc_gemm_kernel<kQK, kProjWideAStages, kProjWideBStages, mla::kEpiLatent, false, 2>,
                    mla::GemmSmem<kQK, kProjWideAStages, kProjWideBStages, 2>::kBytes);
     if (r == MLA_OK)
+      r = set_smem(mla::tc_gemm_kernel<160, kProjMidAStages, kProjMidBStages, mla::kEpiLatent, false, 2>,
+                   mla::GemmSmem<160, kProjMidAStages, kProjMidBStages, 2>::kBytes);
+    if (r == MLA_OK)
       r = set_smem(mla::tc_gemm_kernel<32, kProjNarrowAStages, kProjNarrowBStages, mla::kEpiLatent, false, 1>,
                    mla::GemmSmem<32, kProjNarrowAStages, kProjNarrowBStages, 1>::kBytes);
     if (r == MLA_OK)
-      r = set_smem(mla::tc_gemm_kernel<256, kOutAStages, kOutBStages, mla::kEpiStore, true, 1>,
-                   mla::GemmSmem<256, kOutAStages, kOutBStages>::kBytes);
-    if (r == MLA_OK)
-      r = set_smem(mla::tc_gemm_kernel<128, kOutAStages, kOutBStages, mla::kEpiStore, true, 1>,
-                   mla::GemmSmem<128, kOutAStages, kOutBStages>::kBytes);
+      r = set_smem(mla::tc_gemm_kernel<kOutBN, kOutAStages, kOutBStages, mla::kEpiStore, true, 1>,
+                   mla::GemmSmem<kOutBN, kOutAStages, kOutBStages>::kBytes);
     if (r == MLA_OK)
       r = set_smem(mla::window_attn_kernel<kAttnStages>,
                    mla::AttnSmem<kAttnStages>::kBytes);
