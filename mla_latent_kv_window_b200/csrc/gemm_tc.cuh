@@ -8,13 +8,16 @@
 //   warp 0      TMA producer of A k-blocks (64 wide) into an A_STAGES-deep ring
 //   warp 2      TMA producer of B k-blocks into a B_STAGES-deep ring
 //   warp 1      TMEM allocator + single-thread tcgen05.mma issuer (M=128, N=BN, K=16 steps)
-//   warps 3..10 epilogue, two warps per TMEM lane quarter: each thread owns one row and one
-//               half of the tile's 32-column chunks.  tcgen05.ld of the accumulator (the next
-//               chunk is loaded while the current one is converted), fused column transform,
-//               16-bit pack into a 32 x 32 staging box per (chunk, quarter), then one TMA tensor
-//               store per box issued by the warp's lane 0.  The boxes use the 64-byte swizzle of
-//               the output tensor maps, which also makes the row-per-thread writes bank-conflict
-//               free; rows past the end of the launch are clipped by the maps' extents.
+//   warps 3..10 epilogue, two warps per TMEM lane quarter: each thread converts one row of
+//               the tile (256-row tiles: one 128-row sub-tile per warp of the pair; 128-row
+//               tiles: half of the 32-column chunks each).  Per chunk: tcgen05.ld of the
+//               accumulator (the next chunk is loaded while the current one is converted),
+//               fused column transform, 16-bit pack into one of the warp's two 32 x 32 staging
+//               boxes, then one TMA tensor store issued by lane 0 right away, so the TMA engine
+//               writes a box while the warp converts the next chunk.  The boxes use the 64-byte
+//               swizzle of the output tensor maps, which also makes the row-per-thread writes
+//               bank-conflict free; rows past the end of the launch are clipped by the maps'
+//               extents.
 // The rings run continuously across tile boundaries.  With M_SUB = 1 the accumulator is
 // double-buffered in TMEM (2 x 256 columns), so the epilogue of tile i overlaps the MMAs of
 // tile i+1.  With M_SUB = 2 a tile is 256 rows: two M=128 accumulators (TMEM columns [0,256)
@@ -71,7 +74,7 @@ struct EpiArgs {
   int32_t frame_w;
   float q_scale;             // softmax_scale * log2(e), applied to the query columns
   RopeBands rope;
-  const float2* rope_hw;     // (cos, sin) tables: [frame_h][16] for h, then [frame_w][16] for w
+  const float2* rope_hw;     // (cos, sin) tables: [16][frame_h] for h, then [16][frame_w] for w
   int32_t frame_h;
 };
 
@@ -80,8 +83,8 @@ struct GemmSmem {
   static constexpr int kABytes = M_SUB * 128 * 64 * 2;
   static constexpr int kBBytes = BN * 64 * 2;
   static constexpr int kBOffset = A_STAGES * kABytes;
-  static constexpr int kStagingOffset = kBOffset + B_STAGES * kBBytes;   // (BN/32) x 4 boxes of 2 KB
-  static constexpr int kBarOffset = kStagingOffset + 128 * BN * 2;
+  static constexpr int kStagingOffset = kBOffset + B_STAGES * kBBytes;   // 8 warps x 2 boxes of 2 KB
+  static constexpr int kBarOffset = kStagingOffset + 8 * 2 * 2048;
   static constexpr int kBytes = kBarOffset + 512 + 1024;    // barriers + alignment slack
   static_assert(kABytes % 1024 == 0 && kBBytes % 1024 == 0, "stage atoms must stay 1 KB aligned");
   static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "column blocks are whole 32-column chunks");
@@ -94,38 +97,52 @@ struct GemmTiles {
   __host__ __device__ int32_t count() const { return m_tiles * n_blocks * batch; }
 };
 
-// Rotate the 16 (re, im) pairs of v: pair p by pos[axis[p]] * freq[p].  The h and w factors
-// (cos, sin) come from tables tab_h / tab_w (16 pairs per position, computed in double on the
-// host and rounded once).  The t factors are formed here: the angle is p + e with
-// p = fl(t * hi), e = (t * hi - p) + t * lo (exact product error by FMA), reduced to [-pi, pi]
-// by Cody-Waite reduction with 2 pi split into two floats (accurate for integer t below
-// 2^24), and evaluated with the hardware sine/cosine.
-__device__ __forceinline__ void rope_rotate32(float* v, int64_t t, const float2* tab_h,
-                                              const float2* tab_w, const RopeBands& rb) {
+// RoPE factors of one token: f[p] = (cos, sin) of pos[axis[p]] * freq[p] for the 16 pairs.
+// The h and w factors come from pair-major tables (computed in double on the host and rounded
+// once): pair p of position h at tab_h[p * h_stride], of position w at tab_w[p * w_stride], so
+// the 32 rows of a warp (consecutive tokens) read consecutive entries.  The t factors are formed here: the angle is p + e
+// with p = fl(t * hi), e = (t * hi - p) + t * lo (exact product error by FMA), reduced to
+// [-pi, pi] by Cody-Waite reduction with 2 pi split into two floats (accurate for integer t
+// below 2^24), and evaluated with the hardware sine/cosine.  The table loads cost an L2 round
+// trip (about a microsecond under a full HBM stream), so the epilogue calls this well before
+// it needs the factors: the loads are issued here in program order, each register is written
+// by exactly one of load or compute, and nothing waits for a load until rope_apply.
+__device__ __forceinline__ void rope_factors(float2* f, int64_t t, const float2* tab_h,
+                                             int h_stride, const float2* tab_w, int w_stride,
+                                             const RopeBands& rb) {
   constexpr float kInv2Pi = 0.15915494309189535f;
   constexpr float kTwoPiHi = 6.28318548202514648f;       // fl(2 pi)
   constexpr float kTwoPiLo = -1.7484556000744e-07f;      // 2 pi - fl(2 pi)
+#pragma unroll
+  for (int p = 0; p < 16; ++p)
+    if (rb.axis[p] != 0)
+      f[p] = ld_nc_f2(rb.axis[p] == 2 ? tab_w + p * w_stride : tab_h + p * h_stride);
   const float tf = (float)t;
 #pragma unroll
   for (int p = 0; p < 16; ++p) {
-    const int ax = rb.axis[p];
-    float sn, cs;
-    if (ax == 0) {
+    if (rb.axis[p] == 0) {
       const float hi = rb.freq_hi[p];
       const float prod = tf * hi;
       const float err = fmaf(tf, hi, -prod) + tf * rb.freq_lo[p];
       const float k = rintf(prod * kInv2Pi);
       float r = fmaf(-k, kTwoPiHi, prod);
       r = fmaf(-k, kTwoPiLo, r) + err;
-      __sincosf(r, &sn, &cs);
-    } else {
-      const float2 f = __ldg((ax == 1 ? tab_h : tab_w) + p);
-      cs = f.x;
-      sn = f.y;
+      __sincosf(r, &f[p].y, &f[p].x);
+      pin_f2(f[p]);
     }
+  }
+}
+
+// Row of a 128-row sub-tile held by TMEM lane quarter q, lane l (32x32b access shape).
+__device__ __forceinline__ int row_in_sub(uint32_t q, uint32_t l) { return (int)(q * 32u + l); }
+
+// Rotate the 16 (re, im) pairs of v by the factors f.
+__device__ __forceinline__ void rope_apply(float* v, const float2* f) {
+#pragma unroll
+  for (int p = 0; p < 16; ++p) {
     const float a = v[2 * p], b = v[2 * p + 1];
-    v[2 * p] = a * cs - b * sn;
-    v[2 * p + 1] = a * sn + b * cs;
+    v[2 * p] = a * f[p].x - b * f[p].y;
+    v[2 * p + 1] = a * f[p].y + b * f[p].x;
   }
 }
 
@@ -273,105 +290,115 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
   } else {
     // ------------------------------------------------------------------ epilogue warps
+    // Each thread converts one row of the tile: with 256-row tiles the two warps of a TMEM lane
+    // quarter take one 128-row sub-tile each; with 128-row tiles they split the columns.
     const uint32_t sub_q = warp & 3u;          // TMEM lane quarter = rows 32*sub_q.. of a sub-tile
-    const int half = (int)(warp - 3) >> 2;     // 0: first half of the chunks, 1: second half
+    const int pair = (int)(warp - 3) >> 2;     // which warp of the quarter's pair
     constexpr int kChunks = BN / 32;
     constexpr int kSplit = (kChunks + 1) / 2;
-    const int c_lo = half ? kSplit : 0;
-    const int c_hi = half ? kChunks : kSplit;
-    const int row = sub_q * 32 + lane;         // row of each 128-row sub-tile owned by this thread
-    // Staging box (chunk c, quarter q) at (c*4 + q) * 2 KB: 32 rows of 64 B; 16-byte unit u of
-    // row r sits at slot u ^ ((r >> 1) & 3), the 64-byte swizzle of the output maps.
-    uint8_t* stage = smem + L::kStagingOffset;
+    constexpr int kMaxChunks = M_SUB == 2 ? kChunks : kSplit;   // chunks per warp and tile
+    const int my_sub = M_SUB == 2 ? pair : 0;
+    const int c_lo = M_SUB == 2 ? 0 : (pair ? kSplit : 0);
+    const int c_hi = M_SUB == 2 ? kChunks : (pair ? kChunks : kSplit);
+    // Two 2 KB staging boxes per warp (32 rows x 64 B); 16-byte unit u of row r sits at slot
+    // u ^ ((r >> 1) & 3), the 64-byte swizzle of the output maps.  A box is rewritten only after
+    // the tensor store issued from it two chunks earlier has read it.
+    uint8_t* stage = smem + L::kStagingOffset + (warp - 3) * 2 * 2048;
     const uint32_t swz = (lane >> 1) & 3u;
+    int issued = 0;                            // tensor stores issued by this warp (lane 0)
+    float2 rf[16];                             // RoPE factors of this thread's row
     for (int i = 0; i < my_tiles; ++i) {
       const int buf = i % kAccBufs;
       int m0t, y, z;
       tile_coords(blockIdx.x + i * gridDim.x, m0t, y, z);
+      const int col_base = b_row0 + y * BN;
+      const int m = m0t + my_sub * 128 + row_in_sub(sub_q, lane);
+      const int row0 = m0t + my_sub * 128 + (int)sub_q * 32;
+      // The RoPE chunk of this warp's columns (at most one: one per 224 columns); its factors
+      // are formed now, while the tile's MMAs still run.
+      int rc = -1;
+      if constexpr (kEpi == kEpiLatent) {
+        for (int c = c_lo; c < c_hi; ++c)
+          if ((col_base + c * 32) % 224 == 192) rc = c;
+        if (rc >= 0) {
+          const int F = ep.tokens_per_frame;
+          const int fi = m / F;                // frame within this launch
+          const int k = m - fi * F;
+          const int hh = k / ep.frame_w;
+          rope_factors(rf, ep.t0 + fi, ep.rope_hw + hh, ep.frame_h,
+                       ep.rope_hw + 16 * ep.frame_h + (k - hh * ep.frame_w), ep.frame_w, ep.rope);
+        }
+      }
       if (!mbar_wait_warp_sleepy(&acc_full[buf], (uint32_t)(i / kAccBufs) & 1u, status)) break;
       tc_fence_after();
-      const int col_base = b_row0 + y * BN;
-#pragma unroll 1
-      for (int sub = 0; sub < M_SUB; ++sub) {
-        const int m = m0t + sub * 128 + row;
-        const uint32_t tbase = tmem + (buf + sub) * 256 + ((sub_q * 32u) << 16);
-        int64_t t = 0;
-        const float2* tab_h = nullptr;
-        const float2* tab_w = nullptr;
+      const uint32_t tbase = tmem + (buf + my_sub) * 256 + ((sub_q * 32u) << 16);
+      // Chunk order: the RoPE chunk first, then the rest in order.
+      auto chunk_at = [&](int cc) {
+        if (rc < 0) return c_lo + cc;
+        if (cc == 0) return rc;
+        const int e = c_lo + cc - 1;
+        return e >= rc ? e + 1 : e;
+      };
+      uint32_t r[2][32];
+      if (c_lo < c_hi) tmem_ld32(tbase + chunk_at(0) * 32, r[0]);   // (BN = 32: one warp owns nothing)
+#pragma unroll
+      for (int cc = 0; cc < kMaxChunks; ++cc) {
+        if (c_lo + cc >= c_hi) break;
+        const int c = chunk_at(cc);
+        uint32_t* cur = r[cc & 1];
+        tmem_ld_wait();
+        tmem_regs_ready(cur);
+        if (c_lo + cc + 1 < c_hi) tmem_ld32(tbase + chunk_at(cc + 1) * 32, r[(cc + 1) & 1]);
+        float v[32];
+#pragma unroll
+        for (int q = 0; q < 32; ++q) v[q] = __uint_as_float(cur[q]);
+        const int col = col_base + c * 32;
         if constexpr (kEpi == kEpiLatent) {
-          const int F = ep.tokens_per_frame;
-          const int fi = m / F;               // frame within this launch
-          const int k = m - fi * F;
-          t = ep.t0 + fi;
-          const int hh = k / ep.frame_w;
-          tab_h = ep.rope_hw + hh * 16;
-          tab_w = ep.rope_hw + (ep.frame_h + k - hh * ep.frame_w) * 16;
+          if (c == rc) rope_apply(v, rf);
+          if (col < ep.latent_col0) {
+#pragma unroll
+            for (int q = 0; q < 32; ++q) v[q] *= ep.q_scale;
+          }
         }
-        // The staging boxes are free once this warp's previous tensor stores have read them.
-        if (lane == 0) bulk_wait_read_all();
+        // Box issued % 2 is free once at most one later store is still reading.
+        if (lane == 0) bulk_wait_read_1();
         __syncwarp();
-        uint32_t r[2][32];
-        if (c_lo < c_hi) tmem_ld32(tbase + c_lo * 32, r[0]);   // (BN = 32: half 1 owns nothing)
+        uint8_t* box_base = stage + (issued & 1) * 2048;
+        uint4* box = reinterpret_cast<uint4*>(box_base + lane * 64);
 #pragma unroll
-        for (int cc = 0; cc < kSplit; ++cc) {
-          const int c = c_lo + cc;
-          if (c >= c_hi) break;
-          uint32_t* cur = r[cc & 1];
-          tmem_ld_wait();
-          tmem_regs_ready(cur);
-          if (c + 1 < c_hi) tmem_ld32(tbase + (c + 1) * 32, r[(cc + 1) & 1]);
-          float v[32];
-#pragma unroll
-          for (int q = 0; q < 32; ++q) v[q] = __uint_as_float(cur[q]);
-          if constexpr (kEpi == kEpiLatent) {
-            const int col = col_base + c * 32;
-            if (col % 224 == 192) rope_rotate32(v, t, tab_h, tab_w, ep.rope);
-            if (col < ep.latent_col0) {
-#pragma unroll
-              for (int q = 0; q < 32; ++q) v[q] *= ep.q_scale;
-            }
-          }
-          uint4* box = reinterpret_cast<uint4*>(stage + (c * 4 + sub_q) * 2048 + lane * 64);
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            uint4 w;
-            if constexpr (kEpi == kEpiLatent)
-              w = make_uint4(pack_f16x2(v[8 * u + 0], v[8 * u + 1]), pack_f16x2(v[8 * u + 2], v[8 * u + 3]),
-                             pack_f16x2(v[8 * u + 4], v[8 * u + 5]), pack_f16x2(v[8 * u + 6], v[8 * u + 7]));
-            else
-              w = make_uint4(pack_bf16x2(v[8 * u + 0], v[8 * u + 1]), pack_bf16x2(v[8 * u + 2], v[8 * u + 3]),
-                             pack_bf16x2(v[8 * u + 4], v[8 * u + 5]), pack_bf16x2(v[8 * u + 6], v[8 * u + 7]));
-            box[u ^ swz] = w;
-          }
-        }
-        if (sub == M_SUB - 1) {
-          // Every accumulator of this tile has been read: the buffer is free for the MMAs.
-          tc_fence_before();
-          mbar_arrive(&acc_empty[buf]);
+        for (int u = 0; u < 4; ++u) {
+          uint4 w;
+          if constexpr (kEpi == kEpiLatent)
+            w = make_uint4(pack_f16x2(v[8 * u + 0], v[8 * u + 1]), pack_f16x2(v[8 * u + 2], v[8 * u + 3]),
+                           pack_f16x2(v[8 * u + 4], v[8 * u + 5]), pack_f16x2(v[8 * u + 6], v[8 * u + 7]));
+          else
+            w = make_uint4(pack_bf16x2(v[8 * u + 0], v[8 * u + 1]), pack_bf16x2(v[8 * u + 2], v[8 * u + 3]),
+                           pack_bf16x2(v[8 * u + 4], v[8 * u + 5]), pack_bf16x2(v[8 * u + 6], v[8 * u + 7]));
+          box[u ^ swz] = w;
         }
         fence_proxy_async_smem();   // staging writes -> visible to the TMA engine
         __syncwarp();
-        const int row0 = m0t + sub * 128 + (int)sub_q * 32;
-        if (lane == 0 && row0 < M) {
-          for (int c = c_lo; c < c_hi; ++c) {
-            const int col = col_base + c * 32;
-            if (col >= ep.n_cols) break;
-            const uint8_t* src = stage + (c * 4 + sub_q) * 2048;
+        if (col < ep.n_cols && row0 < M) {
+          if (lane == 0) {
             if constexpr (kEpi == kEpiLatent) {
               const int j = col - ep.latent_col0;
               if (j < 0)
-                tma_store_3d(&map_o0, src, col, row0, z);
+                tma_store_3d(&map_o0, box_base, col, row0, z);
               else if (j < 192)
-                tma_store_3d(&map_o1, src, j, row0, z);
+                tma_store_3d(&map_o1, box_base, j, row0, z);
               else
-                tma_store_3d(&map_o2, src, j - 192, row0, z);
+                tma_store_3d(&map_o2, box_base, j - 192, row0, z);
             } else {
-              tma_store_3d(&map_o0, src, col, row0, z);
+              tma_store_3d(&map_o0, box_base, col, row0, z);
             }
+            bulk_commit();
           }
-          bulk_commit();
+          ++issued;
         }
       }
+      // This thread has read all its accumulator columns of the tile.
+      tc_fence_before();
+      mbar_arrive(&acc_empty[buf]);
     }
     if (lane == 0) bulk_wait_all();
   }

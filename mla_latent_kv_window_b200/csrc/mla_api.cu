@@ -40,16 +40,16 @@ constexpr int kQK = kLatent + kRope;  // 224
 // Pipeline depths of the launched kernel variants (A = activations, B = weights); each GEMM
 // CTA runs alone on its SM.  The weight ring is deep too: its L2 latency sets the k-block rate
 // when only a few CTAs run.
-constexpr int kProjAStages = 5;     // 5 x 16 KB of hidden states in flight per SM (HBM latency)
+constexpr int kProjAStages = 6;     // 6 x 16 KB of hidden states in flight per SM (HBM latency)
 constexpr int kProjBStages = 3;     // 3 x 28 KB of L2-resident weights
-constexpr int kProjWideAStages = 3; // 256-row tiles: 3 x 32 KB of hidden states
+constexpr int kProjWideAStages = 4; // 256-row tiles: 4 x 32 KB of hidden states
 constexpr int kProjWideBStages = 2;
 constexpr int kProjNarrowAStages = 8;   // 32-column latent blocks: 8 x 16 KB + 4 x 4 KB
 constexpr int kProjNarrowBStages = 4;
-constexpr int kProjMidAStages = 3;      // 256 x 160 tiles: 3 x 32 KB + 3 x 20 KB
+constexpr int kProjMidAStages = 4;      // 256 x 160 tiles: 4 x 32 KB + 3 x 20 KB
 constexpr int kProjMidBStages = 3;
 constexpr int kOutBN = 192;             // output projection column block
-constexpr int kOutAStages = 5;
+constexpr int kOutAStages = 6;
 constexpr int kOutBStages = 3;
 
 // Tile shapes of the projection GEMMs with the steady-state time of one 64-wide k-block in
@@ -258,7 +258,7 @@ struct mla_cache {
   __half* o_lat = nullptr;         // fp16 P . c_kv
   __nv_bfloat16* wqcat = nullptr;  // bf16: multiplies the caller's bf16 hidden states
   __half* wov = nullptr;           // fp16: multiplies o_lat
-  float2* rope_hw = nullptr;       // RoPE (cos, sin) of the h and w bands, [frame_h + frame_w][16]
+  float2* rope_hw = nullptr;       // RoPE (cos, sin) of the h and w bands, [16][frame_h + frame_w]
   int* status = nullptr;
 
   CUtensorMap map_wqcat{};         // B operand of the projections: box 64 x 224
@@ -326,22 +326,22 @@ RopeBands make_bands(const mla_config& cfg) {
 }
 
 // (cos, sin) of the h and w RoPE bands for every h in [0, frame_h) and w in [0, frame_w),
-// evaluated in double and rounded once: rows [0, frame_h) hold h, rows [frame_h, frame_h +
-// frame_w) hold w, 16 pairs each (pairs of the other axes hold (1, 0)).
+// evaluated in double and rounded once, pair-major: [16][frame_h] for h, then [16][frame_w]
+// for w (pairs of the other axes hold (1, 0)).
 std::vector<float2> make_rope_hw(const mla_config& cfg) {
-  std::vector<float2> tab((size_t)(cfg.frame_h + cfg.frame_w) * 16, make_float2(1.f, 0.f));
+  const size_t H = cfg.frame_h, Wd = cfg.frame_w;
+  std::vector<float2> tab(16 * (H + Wd), make_float2(1.f, 0.f));
   int p = 0;
   const int dims[3] = {cfg.rope_t, cfg.rope_h, cfg.rope_w};
   for (int a = 0; a < 3; ++a)
     for (int i = 0; i < dims[a] / 2; ++i, ++p) {
       const double f = std::pow(cfg.rope_base, -2.0 * i / dims[a]);
       if (a == 1)
-        for (int h = 0; h < cfg.frame_h; ++h)
-          tab[(size_t)h * 16 + p] = make_float2((float)std::cos(h * f), (float)std::sin(h * f));
+        for (size_t h = 0; h < H; ++h)
+          tab[p * H + h] = make_float2((float)std::cos(h * f), (float)std::sin(h * f));
       if (a == 2)
-        for (int w = 0; w < cfg.frame_w; ++w)
-          tab[(size_t)(cfg.frame_h + w) * 16 + p] =
-              make_float2((float)std::cos(w * f), (float)std::sin(w * f));
+        for (size_t w = 0; w < Wd; ++w)
+          tab[16 * H + p * Wd + w] = make_float2((float)std::cos(w * f), (float)std::sin(w * f));
     }
   return tab;
 }

@@ -119,6 +119,18 @@ __device__ __forceinline__ void grid_launch_dependents() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
+// Read-only 8-byte load issued at this point of the program (a volatile asm keeps the compiler
+// from sinking it towards its first use, so its latency overlaps whatever runs in between).
+__device__ __forceinline__ float2 ld_nc_f2(const float2* p) {
+  float2 v;
+  asm volatile("ld.global.nc.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "l"(p));
+  return v;
+}
+// Keep a computed value at this point of the program (the compiler may not sink its producer).
+__device__ __forceinline__ void pin_f2(float2& v) {
+  asm volatile("" : "+f"(v.x), "+f"(v.y));
+}
+
 // Named barrier over a subset of warps (id 1..15; id 0 is __syncthreads).
 __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
@@ -179,6 +191,10 @@ __device__ __forceinline__ void bulk_commit() {
 // Wait until this thread's committed bulk copies have finished reading shared memory.
 __device__ __forceinline__ void bulk_wait_read_all() {
   asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// Wait until at most one of this thread's committed bulk copy groups is still reading shared memory.
+__device__ __forceinline__ void bulk_wait_read_1() {
+  asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
 }
 // Wait until this thread's committed bulk copies have completed.
 __device__ __forceinline__ void bulk_wait_all() {
