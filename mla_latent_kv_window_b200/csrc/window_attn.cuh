@@ -30,6 +30,9 @@
 //               fp16 o_lat, staged in shared memory and written by one bulk copy per row.
 //
 // TMEM columns: S [0,128), P [128,192), Q [192,304), O [304,496).
+// Launched with programmatic stream serialization: barrier init, TMEM allocation and the
+// tensor-map prefetch overlap the projection kernel's tail; griddepcontrol.wait precedes the first
+// global access.
 #pragma once
 
 #include "ptx.cuh"
