@@ -110,9 +110,15 @@ def sustained_peak():
 
 
 def kernel_source_hash() -> str:
+    """Hash of the CUDA sources with comments and blank lines removed (a comment edit leaves the
+    kernels, and so the ncu counters taken on them, unchanged)."""
+    import re
     h = hashlib.sha256()
     for f in ("ptx.cuh", "gemm_tc.cuh", "window_attn.cuh", "dense_attn.cuh", "mla_api.cu"):
-        h.update(open(os.path.join(ROOT, "mla_latent_kv_window_b200", "csrc", f), "rb").read())
+        src = open(os.path.join(ROOT, "mla_latent_kv_window_b200", "csrc", f)).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        src = re.sub(r"//[^\n]*", "", src)
+        h.update("\n".join(l.rstrip() for l in src.splitlines() if l.strip()).encode())
     return h.hexdigest()[:16]
 
 
