@@ -22,6 +22,12 @@ DIMS_WAN13B = dict(
     hidden=1536, n_heads=12, d_head=128, d_nope=128, d_latent=192, d_rope=32,
     rope_t=8, rope_h=12, rope_w=12, rope_base=10000.0,
 )
+# The paper's default attention dims ([VideoMLA] §4.1): content key 96 + positional key 32
+# (= the backbone's 128 per head), a low-rank query of width d_q = 768, RoPE (6, 5, 5) pairs.
+DIMS_PAPER = dict(
+    hidden=1536, n_heads=12, d_head=128, d_nope=96, d_latent=192, d_rope=32,
+    rope_t=12, rope_h=10, rope_w=10, rope_base=10000.0, d_q=768,
+)
 
 
 @dataclasses.dataclass(frozen=True)
@@ -39,6 +45,7 @@ class Workload:
     seed: int = 0
     stream_scale: bool = False  # per-stream random scale in [0.5, 2]
     dims: tuple = tuple(sorted(DIMS_WAN13B.items()))
+    sink_frames: int = 0        # first frames kept for good besides the window (App. D.4/D.5)
 
     @property
     def F(self) -> int:
@@ -62,6 +69,16 @@ WORKLOADS = {
                               stream_scale=True),
     "wan_w63_q1": Workload("wan_w63_q1", frame_h=30, frame_w=52, window_frames=63,
                            fill_frames=63, query_frames=1, seed=4000),
+    # Next rows: the paper-default dims, and a sink frame plus a short window.
+    "paper_tiny": Workload("paper_tiny", frame_h=4, frame_w=6, window_frames=2, fill_frames=3,
+                           query_frames=1, seed=5, dims=tuple(sorted(DIMS_PAPER.items()))),
+    "paper_w21_q1": Workload("paper_w21_q1", frame_h=30, frame_w=52, window_frames=21,
+                             fill_frames=21, query_frames=1, seed=5000,
+                             dims=tuple(sorted(DIMS_PAPER.items()))),
+    "sink_tiny": Workload("sink_tiny", frame_h=4, frame_w=6, window_frames=2, fill_frames=5,
+                          query_frames=2, seed=6, sink_frames=1),
+    "sink_w6_q3": Workload("sink_w6_q3", frame_h=30, frame_w=52, window_frames=6,
+                           fill_frames=10, query_frames=3, seed=6000, sink_frames=1),
 }
 
 
@@ -78,22 +95,30 @@ def normal_bf16(shape, std: float, seed: int) -> torch.Tensor:
 
 
 def make_weights(dims: dict, seed: int) -> dict:
-    """All seven projection weights of one layer, bf16, N(0, 1/fan_in)."""
+    """The projection weights of one layer, bf16, N(0, 1/fan_in).
+
+    With a low-rank query (dims["d_q"] > 0) the query projections read the d_q-wide query
+    latent, w_q is [n_h d_nope, d_q], w_qr [n_h d_rope, d_q], and w_dq [d_q, hidden] is added.
+    """
     d = dims["hidden"]
     nh = dims["n_heads"]
     dn = dims["d_nope"]
     dv = dims["d_head"]
     dc = dims["d_latent"]
     dr = dims["d_rope"]
+    dq = dims.get("d_q", 0)
+    q_in = dq if dq else d
     shapes = {
-        "w_q": (nh * dn, d),
-        "w_qr": (nh * dr, d),
+        "w_q": (nh * dn, q_in),
+        "w_qr": (nh * dr, q_in),
         "w_dkv": (dc, d),
         "w_kr": (dr, d),
         "w_uk": (nh * dn, dc),
         "w_uv": (nh * dv, dc),
         "w_o": (d, nh * dv),
     }
+    if dq:
+        shapes["w_dq"] = (dq, d)
     out = {}
     for i, (name, shp) in enumerate(shapes.items()):
         out[name] = normal_bf16(shp, 1.0 / float(shp[1]) ** 0.5, seed * 16 + i)

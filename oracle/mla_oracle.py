@@ -14,15 +14,20 @@ What it computes (the unabsorbed plain definition, in float64, from bf16 inputs)
   head-shared content latent c = x W_DKV^T (d_c) and a head-shared positional
   state r = x W_KR^T (d_rope).  Following [VideoMLA] App. D.5, r is stored
   *before* RoPE and rotated when the window is assembled.
-* Sliding window ([VideoMLA] §1, App. D.4): a FIFO of the last W latent frames.
+* Sliding window ([VideoMLA] §1, App. D.4): a FIFO of the last W latent frames,
+  optionally after `sink_frames` sink frames: the first frames of the video,
+  kept for good (App. D.4/D.5 "sink + local window").
 * Attention ([VideoMLA] §3.3): per head, keys and values are reconstructed
   from the latent, k_h = [c W_UK[h]^T || RoPE3D(r)], v_h = c W_UV[h]^T, the
-  query is q_h = [x W_Q[h]^T || RoPE3D(x W_QR[h]^T)], and textbook softmax
-  attention runs over the window frames plus the chunk's own frames (the query
+  query is q_h = [x W_Q[h]^T || RoPE3D(x W_QR[h]^T)] (with a low-rank query,
+  [VideoMLA] §4.1 d_q = 768, x is first projected to c_q = x W_DQ^T and W_Q, W_QR
+  read c_q), and textbook softmax attention runs over the sink and window frames
+  plus the chunk's own frames (the query
   chunk is the newest, so chunk-causal masking ([VideoMLA] App. D.4) masks
   nothing).  out = concat_h(o_h) W_O^T.
-* Positions ([VideoMLA] App. D.5): the active window frames and the query chunk
-  get window-local temporal coordinates 0, 1, ... and are rotated at use.
+* Positions ([VideoMLA] App. D.5): the active frames (sink frames, then the
+  window frames, oldest first) and the query chunk get window-local temporal
+  coordinates 0, 1, ... and are rotated at use.
 * 3D RoPE ([VideoMLA] §3.2, §4.1, App. C.1): the d_rope channels split into
   temporal / height / width groups of adjacent pairs; axis a with d_a channels
   rotates pair i by angle pos_a * base^(-2 i / d_a) (i = 0 is the highest
@@ -133,9 +138,10 @@ class OracleLayer:
     """One VideoMLA self-attention layer with its sliding-window latent cache, in float64.
 
     dims: hidden, n_heads, d_head, d_nope, d_latent, d_rope, rope_t, rope_h, rope_w,
-    rope_base, plus frame_h, frame_w, window_frames.  weights: w_q [n_h d_nope, d],
-    w_qr [n_h d_rope, d], w_dkv [d_c, d], w_kr [d_rope, d], w_uk [n_h d_nope, d_c],
-    w_uv [n_h d_head, d_c], w_o [d, n_h d_head] (nn.Linear [out, in] layout).
+    rope_base, plus frame_h, frame_w, window_frames and optionally sink_frames.  weights:
+    w_q [n_h d_nope, d], w_qr [n_h d_rope, d], w_dkv [d_c, d], w_kr [d_rope, d],
+    w_uk [n_h d_nope, d_c], w_uv [n_h d_head, d_c], w_o [d, n_h d_head] (nn.Linear [out, in]
+    layout); with a low-rank query also w_dq [d_q, d], and then w_q, w_qr read d_q columns.
     """
 
     def __init__(self, dims: dict, weights: dict, softmax_scale: float | None = None):
@@ -144,7 +150,10 @@ class OracleLayer:
         self.F = self.d["frame_h"] * self.d["frame_w"]
         dn, dr = self.d["d_nope"], self.d["d_rope"]
         self.scale = softmax_scale if softmax_scale else 1.0 / math.sqrt(dn + dr)
-        # FIFO of cached frames, oldest first; each entry is (absolute frame index, c [F,d_c], r [F,d_r]).
+        # Sink frames (the first sink_frames frames appended, kept for good) and the FIFO of the
+        # other cached frames, oldest first; each entry is (absolute frame index, c [F,d_c], r [F,d_r]).
+        self.n_sink = int(self.d.get("sink_frames", 0))
+        self.sink: list[tuple[int, np.ndarray, np.ndarray]] = []
         self.frames: list[tuple[int, np.ndarray, np.ndarray]] = []
         self.frames_appended = 0
 
@@ -156,28 +165,43 @@ class OracleLayer:
         return c, r
 
     def append(self, x) -> None:
-        """Append n whole latent frames of hidden states x [n F, d]; keep the newest W frames."""
+        """Append n whole latent frames of hidden states x [n F, d]: the first sink_frames frames
+        ever appended become the sink, the others go through the FIFO of the newest W frames."""
         x = _f64(x)
         if x.shape[0] % self.F:
             raise ValueError("append takes whole latent frames")
         c, r = self.latent(x)
         for i in range(x.shape[0] // self.F):
             sl = slice(i * self.F, (i + 1) * self.F)
-            self.frames.append((self.frames_appended, c[sl], r[sl]))
+            entry = (self.frames_appended, c[sl], r[sl])
             self.frames_appended += 1
+            if len(self.sink) < self.n_sink:
+                self.sink.append(entry)
+                continue
+            self.frames.append(entry)
             if len(self.frames) > self.d["window_frames"]:
                 self.frames.pop(0)
+
+    def active_frames(self):
+        """The cached frames attention sees, in logical order: sink frames, then the window."""
+        return self.sink + self.frames
+
+    def query_input(self, x: np.ndarray) -> np.ndarray:
+        """What the query projections read: x itself, or with a low-rank query the query latent
+        c_q = x W_DQ^T ([VideoMLA] §4.1: d_q = 768; no norm on c_q, as elsewhere in the block)."""
+        return x @ self.W["w_dq"].T if "w_dq" in self.W else x
 
     def _rope(self, v, t, h, w):
         d = self.d
         return rope3d(v, t, h, w, d["rope_t"], d["rope_h"], d["rope_w"], d["rope_base"])
 
     def cache_contents(self):
-        """What a ring that rotates at append time would hold: per valid frame (oldest first)
-        the absolute frame index, c [F, d_c] and r rotated at the frame's ABSOLUTE index [F, d_r]."""
+        """What a ring that rotates at append time would hold: per valid frame (sink frames first,
+        then the window oldest first) the absolute frame index, c [F, d_c] and r rotated at the
+        frame's ABSOLUTE index [F, d_r]."""
         hh, ww = token_hw(np.arange(self.F), self.d["frame_w"])
         out = []
-        for f, c, r in self.frames:
+        for f, c, r in self.active_frames():
             out.append((f, c.copy(), self._rope(r, f, hh, ww)))
         return out
 
@@ -185,17 +209,19 @@ class OracleLayer:
         """Assemble the attention context: latent keys (window frames oldest first, then the chunk)
         with their positions, and the chunk's query inputs with theirs.
 
-        positions="local" is the App. D.5 re-indexing (window-local temporal coordinates);
-        "absolute" uses absolute frame indices (equal results for a window without a sink).
+        positions="local" is the App. D.5 re-indexing (window-local temporal coordinates: sink
+        frames, window frames and the chunk numbered 0, 1, ... in that order); "absolute" uses
+        absolute frame indices (equal results for a window without a sink).
         """
         x = _f64(x_chunk)
         if x.shape[0] % self.F or x.shape[0] == 0:
             raise ValueError("a query chunk is one or more whole latent frames")
         nq_frames = x.shape[0] // self.F
         c_new, r_new = self.latent(x)
-        frame_ids = [f for f, _, _ in self.frames] + [self.frames_appended + i for i in range(nq_frames)]
-        c_all = np.concatenate([c for _, c, _ in self.frames] + [c_new], axis=0)
-        r_all = np.concatenate([r for _, _, r in self.frames] + [r_new], axis=0)
+        active = self.active_frames()
+        frame_ids = [f for f, _, _ in active] + [self.frames_appended + i for i in range(nq_frames)]
+        c_all = np.concatenate([c for _, c, _ in active] + [c_new], axis=0)
+        r_all = np.concatenate([r for _, _, r in active] + [r_new], axis=0)
         if positions == "local":
             t_of_frame = np.arange(len(frame_ids), dtype=np.float64)
         elif positions == "absolute":
@@ -224,8 +250,9 @@ class OracleLayer:
         k_nope = ctx["c"] @ w_uk.T                          # Eq. 2 (up-projection), keys
         v = ctx["c"] @ w_uv.T                               # Eq. 2 (up-projection), values
         k_rope = self._rope(ctx["r"], ctx["t_key"], ctx["h_key"], ctx["w_key"])   # shared by heads
-        q_nope = x @ self.W["w_q"][h * dn:(h + 1) * dn].T
-        q_rope = self._rope(x @ self.W["w_qr"][h * dr:(h + 1) * dr].T, tq, hq, wq)
+        xq = self.query_input(x)
+        q_nope = xq @ self.W["w_q"][h * dn:(h + 1) * dn].T
+        q_rope = self._rope(xq @ self.W["w_qr"][h * dr:(h + 1) * dr].T, tq, hq, wq)
         K = np.concatenate([k_nope, k_rope], axis=1)
         Q = np.concatenate([q_nope, q_rope], axis=1)
         return Q, K, v
@@ -269,9 +296,10 @@ class OracleLayer:
         dn, dr = d["d_nope"], d["d_rope"]
         ctx = self.keys_and_queries(x_chunk, positions)
         w_uk = self.W["w_uk"][h * dn:(h + 1) * dn]
-        q_nope = ctx["x"] @ self.W["w_q"][h * dn:(h + 1) * dn].T
+        xq = self.query_input(ctx["x"])
+        q_nope = xq @ self.W["w_q"][h * dn:(h + 1) * dn].T
         q_abs = q_nope @ w_uk                                   # [n_q, d_c]
-        q_rope = self._rope(ctx["x"] @ self.W["w_qr"][h * dr:(h + 1) * dr].T, ctx["t_q"], ctx["h_q"], ctx["w_q"])
+        q_rope = self._rope(xq @ self.W["w_qr"][h * dr:(h + 1) * dr].T, ctx["t_q"], ctx["h_q"], ctx["w_q"])
         k_rope = self._rope(ctx["r"], ctx["t_key"], ctx["h_key"], ctx["w_key"])
         return (q_abs @ ctx["c"].T + q_rope @ k_rope.T) * self.scale
 

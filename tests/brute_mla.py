@@ -29,7 +29,10 @@ def rotate(vec, t, h, w, split, base):
 
 
 def attention(dims, W, window_x, chunk_x):
-    """window_x: list of frames (oldest first) of token hidden vectors; chunk_x: the query frames.
+    """window_x: list of cached frames in logical order (sink frames, then the window oldest
+    first) of token hidden vectors; chunk_x: the query frames.  Frames get window-local temporal
+    coordinates 0, 1, ... in that order.  With W["w_dq"] the query projections read the low-rank
+    query latent W_DQ x instead of x.
 
     Returns out[q][d] for every token of the chunk.
     """
@@ -57,7 +60,8 @@ def attention(dims, W, window_x, chunk_x):
                 Wqr = W["w_qr"][hd * dr:(hd + 1) * dr]
                 Wuk = W["w_uk"][hd * dn:(hd + 1) * dn]
                 Wuv = W["w_uv"][hd * dv:(hd + 1) * dv]
-                q = matvec(Wq, x) + rotate(matvec(Wqr, x), q_t0 + qf, k // fw, k % fw, split, base)
+                xq = matvec(W["w_dq"], x) if "w_dq" in W else x
+                q = matvec(Wq, xq) + rotate(matvec(Wqr, xq), q_t0 + qf, k // fw, k % fw, split, base)
                 scores = []
                 vals = []
                 for c, kr in keys:

@@ -300,3 +300,98 @@ def test_ring_slot_matches_fifo_simulation():
             for k in (0, 3, F - 1):
                 assert ring_slot(f, k, W, F) == owner[f] * F + k
     assert appended == 29
+
+
+# ---------------------------------------------------------------------------- next rows: low-rank query, sink
+def test_brute_force_low_rank_query():
+    # [VideoMLA] §4.1's low-rank query (x -> c_q = W_DQ x -> W_Q c_q, W_QR c_q) with the paper's
+    # 96/32-style split and (6,5,5)-style pairs, shrunk: the oracle against the scalar loops.
+    dims = _tiny_dims(d_q=5, d_nope=3, d_rope=12, rope_t=4, rope_h=4, rope_w=4)
+    layer, w, x_fill, x_q = _tiny_run(dims, seed=23, window=2, fill=3, q_frames=1)
+    assert "w_dq" in w and tuple(w["w_q"].shape) == (2 * 3, 5)
+    out = layer.attention(x_q)
+    F = 4
+    Wl = {k: v.double().tolist() for k, v in w.items()}
+    frames = [x_fill[i * F:(i + 1) * F].double().tolist() for i in range(3)][-2:]
+    ref = np.array(brute_mla.attention(dims, Wl, frames, [x_q.double().tolist()]))
+    np.testing.assert_allclose(out, ref, rtol=1e-12, atol=1e-12)
+
+
+def test_low_rank_query_equals_composed_full_rank():
+    # A low-rank query is a full-rank one with W_Q = W_UQ W_DQ and W_QR = W_QR' W_DQ (matrix
+    # associativity): the two code paths of the oracle must agree in fp64.
+    dims = _dims(frame_h=2, frame_w=3, window_frames=2, hidden=64, n_heads=2, d_head=16, d_nope=12,
+                 d_q=24)
+    lr, w, x_fill, x_q = _tiny_run(dims, seed=24, window=2, fill=3, q_frames=1)
+    wf = {k: v.double() for k, v in w.items() if k != "w_dq"}
+    wf["w_q"] = w["w_q"].double() @ w["w_dq"].double()
+    wf["w_qr"] = w["w_qr"].double() @ w["w_dq"].double()
+    fr_dims = dict(dims)
+    fr_dims.pop("d_q")
+    fr = OracleLayer(fr_dims, wf)
+    fr.append(x_fill)
+    np.testing.assert_allclose(lr.attention(x_q), fr.attention(x_q), rtol=1e-11, atol=1e-13)
+
+
+def test_sink_and_window_bookkeeping():
+    # App. D.4/D.5: the first sink_frames frames stay for good; the window keeps the newest W of
+    # the others.  Frame lists after each append, against a direct statement of that rule.
+    dims = _tiny_dims(window_frames=2, sink_frames=1)
+    layer, _ = _layer(dims, 3)
+    x = mla_synth.make_hidden(1, 9 * 4, dims["hidden"], 4)[0]
+    seen = 0
+    for n in (1, 1, 2, 4, 1):
+        layer.append(x[seen * 4:(seen + n) * 4])
+        seen += n
+        assert [f for f, _, _ in layer.sink] == [0]
+        assert [f for f, _, _ in layer.frames] == list(range(max(1, seen - 2), seen))
+        assert [f for f, _, _ in layer.active_frames()] == [0] + list(range(max(1, seen - 2), seen))
+
+
+def test_brute_force_sink():
+    # One sink frame + a 2-frame window after 5 appended frames: the brute force gets the logical
+    # key frames [0, 3, 4] written out by hand, numbered 0, 1, 2 (App. D.5), then the chunk.
+    dims = _tiny_dims(window_frames=2, sink_frames=1)
+    layer, w, x_fill, x_q = _tiny_run(dims, seed=25, window=2, fill=5, q_frames=2)
+    out = layer.attention(x_q)
+    F = 4
+    Wl = {k: v.double().tolist() for k, v in w.items()}
+    fr = [x_fill[i * F:(i + 1) * F].double().tolist() for i in range(5)]
+    chunk = [x_q[i * F:(i + 1) * F].double().tolist() for i in range(2)]
+    ref = np.array(brute_mla.attention(dims, Wl, [fr[0], fr[3], fr[4]], chunk))
+    np.testing.assert_allclose(out, ref, rtol=1e-12, atol=1e-12)
+
+
+def test_sink_changes_the_absolute_reading():
+    # With a sink and a slid window, absolute frame indices no longer differ from the local ones
+    # by one shared offset, so the two readings give different outputs (the GPU must rotate the
+    # query separately for the sink keys).
+    dims = _tiny_dims(window_frames=2, sink_frames=1)
+    layer, _, _, x_q = _tiny_run(dims, seed=26, window=2, fill=6, q_frames=1)
+    a = layer.attention(x_q, positions="local")
+    b = layer.attention(x_q, positions="absolute")
+    assert np.max(np.abs(a - b)) > 1e-6
+
+
+def test_sink_segment_rotation_equals_local():
+    # The GPU keeps keys rotated at their absolute frame index and rotates the query at its
+    # absolute index for window and chunk keys, but at its window-local index for sink keys
+    # (RoPE(a) . RoPE(b) depends on a - b only).  Those scores equal the App. D.5 local ones.
+    dims = _tiny_dims(window_frames=2, sink_frames=1)
+    layer, _, _, x_q = _tiny_run(dims, seed=27, window=2, fill=6, q_frames=2)
+    loc = layer.keys_and_queries(x_q, "local")
+    ab = layer.keys_and_queries(x_q, "absolute")
+    d = dims
+    rope = lambda v, t, h, w: rope3d(v, t, h, w, d["rope_t"], d["rope_h"], d["rope_w"], d["rope_base"])
+    n_sink_keys = layer.n_sink * 4
+    for hd in range(d["n_heads"]):
+        xq = layer.query_input(loc["x"])
+        qr = xq @ layer.W["w_qr"][hd * d["d_rope"]:(hd + 1) * d["d_rope"]].T
+        k_abs = rope(ab["r"], ab["t_key"], ab["h_key"], ab["w_key"])
+        q_abs = rope(qr, ab["t_q"], ab["h_q"], ab["w_q"])
+        q_loc = rope(qr, loc["t_q"], loc["h_q"], loc["w_q"])
+        s_gpu = q_abs @ k_abs.T
+        s_gpu[:, :n_sink_keys] = q_loc @ k_abs[:n_sink_keys].T
+        k_loc = rope(loc["r"], loc["t_key"], loc["h_key"], loc["w_key"])
+        np.testing.assert_allclose(s_gpu, q_loc @ k_loc.T, rtol=1e-10, atol=1e-12)
+
