@@ -73,28 +73,41 @@ typedef struct {
   int32_t max_chunk_frames; /* largest query chunk, in frames (3)                        */
   int32_t batch;            /* B independent streams sharing the weights                 */
   float softmax_scale;      /* 0 -> 1 / sqrt(d_nope + d_rope)                            */
+  int32_t d_q;              /* low-rank query width ([VideoMLA] §4.1 default: 768); 0 -> the
+                               query projections read x directly (full-rank W_Q)           */
+  int32_t sink_frames;      /* first frames of the video kept for good besides the window
+                               ([VideoMLA] App. D.4/D.5 "sink + local window"); 0 -> none   */
 } mla_config;
 
 /* Device bf16 weights, nn.Linear layout [out, in]:
- *  w_q  [n_heads*d_nope, hidden]    w_qr [n_heads*d_rope, hidden]
+ *  w_q  [n_heads*d_nope, q_in]      w_qr [n_heads*d_rope, q_in]
  *  w_dkv[d_latent, hidden]          w_kr [d_rope, hidden]
  *  w_uk [n_heads*d_nope, d_latent]  w_uv [n_heads*d_head, d_latent]
- *  w_o  [hidden, n_heads*d_head]
+ *  w_o  [hidden, n_heads*d_head]    w_dq [d_q, hidden] (only with d_q > 0, else ignored)
+ * q_in = hidden for a full-rank query (d_q == 0); with d_q > 0 the query projections read the
+ * low-rank query latent c_q = x W_DQ^T and q_in = d_q.
  * Read only during mla_cache_create; the caller keeps ownership. */
 typedef struct {
   const void *w_q, *w_qr, *w_dkv, *w_kr, *w_uk, *w_uv, *w_o;
+  const void* w_dq;
 } mla_weights;
 
 /* Validate a configuration on the host (no GPU needed).  MLA_OK, MLA_ERR_INVALID_ARGUMENT
  * for values the method does not allow, MLA_ERR_UNSUPPORTED for values the kernels lack. */
 mla_status mla_config_check(const mla_config* cfg);
 
-/* Physical ring slot of (absolute frame index, token in frame): (frame mod W) * F + token
- * ([VideoMLA] §1, App. D.4: fixed-size sliding window of W latent frames, oldest evicted).
+/* Physical row of (absolute frame index, token in frame) in a stream's latent planes
+ * ([VideoMLA] §1, App. D.4: fixed-size sliding window of W latent frames, oldest evicted):
+ *   no sink:                      (frame mod W) * F + token
+ *   frame < sink_frames:          frame * F + token               (sink frames, kept for good)
+ *   otherwise:                    sink_rows + ((frame - sink_frames) mod W) * F + token
+ * with sink_rows = sink_frames * F rounded up to a multiple of 128 (the sink region ends on a
+ * key-tile boundary; its padding rows are never attended).
  * Host only.  MLA_ERR_INVALID_ARGUMENT for frame < 0 or token outside [0, F). */
 mla_status mla_ring_slot(const mla_config* cfg, int64_t frame, int32_t token, int64_t* slot);
 
-/* Bytes of the latent window itself: batch * W * F * (d_latent + d_rope) * 2 (bf16). */
+/* Bytes of the latent window itself: batch * (sink_frames + W) * F * (d_latent + d_rope) * 2
+ * (16-bit cache). */
 size_t mla_ring_bytes(const mla_config* cfg);
 
 /* Bytes of device memory mla_cache_create allocates for this configuration (ring with its
@@ -102,7 +115,8 @@ size_t mla_ring_bytes(const mla_config* cfg);
 size_t mla_cache_device_bytes(const mla_config* cfg);
 
 /* Create a cache on the current device.  Derives and owns the absorbed weights
- *   W_Qabs[h] = W_UK[h]^T W_Q[h]   (hidden -> d_latent per head, queries)
+ *   W_Qabs[h] = W_UK[h]^T W_Q[h]   (hidden -> d_latent per head, queries; with a low-rank
+ *                                   query W_UK[h]^T W_Q[h] W_DQ, and W_QR W_DQ for the RoPE part)
  *   W_OV[h]   = W_O[:, h] W_UV[h]  (d_latent per head -> hidden, outputs)
  * ([VideoMLA] §3.3 reconstructs per-head K/V from the latent through W_UK/W_UV; folding them
  * into the query and output projections is the standard MLA absorption), the RoPE tables and
@@ -113,16 +127,21 @@ mla_status mla_cache_create(const mla_config* cfg, const mla_weights* w, void* s
 
 /* Append n_frames >= 1 whole latent frames x [batch, n_frames*F, hidden] to every stream's
  * window: c_kv = x W_DKV^T and k_rope = RoPE3D(x W_KR^T) at the frames' own (t, h, w), written
- * to ring slots (t mod W) * F + k ([VideoMLA] §3.1, §3.2).  When n_frames > W only the last W
- * frames are computed (the others would be evicted within the call). */
+ * to the rows mla_ring_slot names ([VideoMLA] §3.1, §3.2): the first sink_frames frames ever
+ * appended to the sink, the others to ring slots.  Frames that would be evicted within the
+ * call (more than W non-sink frames) are not computed. */
 mla_status mla_cache_append(mla_cache* c, const void* x, int32_t n_frames, void* stream);
 
 /* Latent-window attention for one query chunk x_chunk [batch, n_frames*F, hidden],
  * 1 <= n_frames <= max_chunk_frames, writing out [batch, n_frames*F, hidden].
- * The chunk attends to the valid window frames plus all of its own tokens (chunk-causal,
- * [VideoMLA] App. D.4).  The chunk's latents go to a scratch tail, not into the ring: call
- * mla_cache_append with the final hidden states to make them part of the window.
- * With an empty window (nothing appended yet) the chunk attends to itself alone. */
+ * The chunk attends to the sink frames, the valid window frames and all of its own tokens
+ * (chunk-causal, [VideoMLA] App. D.4).  Positions follow the window-local re-indexing of
+ * App. D.5 (sink, window, chunk numbered 0, 1, ...): keys are stored rotated at their absolute
+ * frame index, which differs from the local one by a single offset for window and chunk
+ * frames; for the sink keys the query's temporal RoPE bands are turned back by that offset.
+ * The chunk's latents go to a scratch tail, not into the ring: call mla_cache_append with the
+ * final hidden states to make them part of the window.  With an empty window (nothing
+ * appended yet) the chunk attends to itself alone. */
 mla_status mla_window_attention(mla_cache* c, const void* x_chunk, int32_t n_frames, void* out,
                                 void* stream);
 
@@ -167,22 +186,25 @@ mla_status mla_dense_sync(void* stream);
 /* Free everything the cache owns (synchronises the device first).  NULL-safe. */
 void mla_cache_destroy(mla_cache* c);
 
-/* Frames appended so far and frames currently valid in the window (min(appended, W)). */
+/* Frames appended so far and cached frames attention currently sees: valid sink frames plus
+ * valid window frames (min(appended, sink_frames) + min(max(appended - sink_frames, 0), W)). */
 mla_status mla_cache_state(const mla_cache* c, int64_t* frames_appended, int32_t* valid_frames);
 
 /* Synchronise `stream` and return the device status word: MLA_OK, or the error a kernel
  * recorded (MLA_ERR_DEVICE_TIMEOUT).  Reading clears nothing. */
 mla_status mla_cache_sync(mla_cache* c, void* stream);
 
-/* Copy stream b's ring planes to host memory, in physical slot order: ckv_host receives
- * W*F rows of d_latent fp16, krope_host W*F rows of d_rope fp16 (either may be NULL);
- * *n_valid_rows = valid_frames * F.  Synchronous; diagnostic, not on the hot path. */
+/* Copy stream b's cached planes to host memory, in physical row order (the rows mla_ring_slot
+ * names): ckv_host receives sink_rows + W*F rows of d_latent fp16, krope_host as many rows of
+ * d_rope fp16 (either may be NULL); *n_valid_rows = valid_frames * F (mla_cache_state).
+ * Synchronous; diagnostic, not on the hot path. */
 mla_status mla_cache_read(const mla_cache* c, int32_t b, void* ckv_host, void* krope_host,
                           int64_t* n_valid_rows);
 
 /* Device pointers of the cache's internal planes, for diagnostics and tests. */
 typedef struct {
-  void* ckv;          /* fp16 [batch][rows_per_stream][d_latent]; rows = (W + max_chunk)*F   */
+  void* ckv;          /* fp16 [batch][rows_per_stream][d_latent];
+                         rows = sink_rows + (W + max_chunk)*F                              */
   void* krope;        /* fp16 [batch][rows_per_stream][d_rope]                               */
   void* qp;           /* fp16 [batch][max_chunk*F*n_heads][d_latent + d_rope]: absorbed,
                          rotated queries of the last attention call, times scale * log2(e)   */

@@ -48,11 +48,12 @@ class mla_config(ctypes.Structure):
         ("frame_h", ctypes.c_int32), ("frame_w", ctypes.c_int32),
         ("window_frames", ctypes.c_int32), ("max_chunk_frames", ctypes.c_int32),
         ("batch", ctypes.c_int32), ("softmax_scale", ctypes.c_float),
+        ("d_q", ctypes.c_int32), ("sink_frames", ctypes.c_int32),
     ]
 
 
 class mla_weights(ctypes.Structure):
-    _fields_ = [(n, ctypes.c_void_p) for n in ("w_q", "w_qr", "w_dkv", "w_kr", "w_uk", "w_uv", "w_o")]
+    _fields_ = [(n, ctypes.c_void_p) for n in ("w_q", "w_qr", "w_dkv", "w_kr", "w_uk", "w_uv", "w_o", "w_dq")]
 
 
 class mla_debug_buffers(ctypes.Structure):
@@ -118,13 +119,13 @@ def _check(status: int, where: str) -> None:
 
 
 def make_config(dims: dict, frame_h: int, frame_w: int, window_frames: int, max_chunk_frames: int,
-                batch: int = 1, softmax_scale: float = 0.0) -> mla_config:
+                batch: int = 1, softmax_scale: float = 0.0, sink_frames: int = 0) -> mla_config:
     return mla_config(
         hidden=dims["hidden"], n_heads=dims["n_heads"], d_head=dims["d_head"], d_nope=dims["d_nope"],
         d_latent=dims["d_latent"], d_rope=dims["d_rope"], rope_t=dims["rope_t"], rope_h=dims["rope_h"],
         rope_w=dims["rope_w"], rope_base=float(dims["rope_base"]), frame_h=frame_h, frame_w=frame_w,
         window_frames=window_frames, max_chunk_frames=max_chunk_frames, batch=batch,
-        softmax_scale=softmax_scale)
+        softmax_scale=softmax_scale, d_q=int(dims.get("d_q", 0)), sink_frames=sink_frames)
 
 
 # ---------------------------------------------------------------------------- C names, torch args
@@ -162,6 +163,8 @@ def mla_cache_device_bytes(cfg: mla_config) -> int:
 
 def mla_cache_create(cfg: mla_config, weights: dict, stream=None) -> int:
     w = mla_weights(**{k: _dev_ptr(weights[k], k) for k in ("w_q", "w_qr", "w_dkv", "w_kr", "w_uk", "w_uv", "w_o")})
+    if cfg.d_q > 0:
+        w.w_dq = _dev_ptr(weights["w_dq"], "w_dq")
     h = ctypes.c_void_p()
     _check(load_library().mla_cache_create(ctypes.byref(cfg), ctypes.byref(w), _stream_handle(stream),
                                            ctypes.byref(h)), "mla_cache_create")
@@ -255,8 +258,10 @@ class LatentWindowCache:
     """One layer's latent window on the current CUDA device (owns the C handle)."""
 
     def __init__(self, dims: dict, weights: dict, frame_h: int, frame_w: int, window_frames: int,
-                 max_chunk_frames: int, batch: int = 1, softmax_scale: float = 0.0, stream=None):
-        self.cfg = make_config(dims, frame_h, frame_w, window_frames, max_chunk_frames, batch, softmax_scale)
+                 max_chunk_frames: int, batch: int = 1, softmax_scale: float = 0.0, stream=None,
+                 sink_frames: int = 0):
+        self.cfg = make_config(dims, frame_h, frame_w, window_frames, max_chunk_frames, batch, softmax_scale,
+                               sink_frames)
         self.F = frame_h * frame_w
         self.handle = mla_cache_create(self.cfg, weights, stream)
 
@@ -274,15 +279,20 @@ class LatentWindowCache:
     def state(self):
         return mla_cache_state(self.handle)
 
+    def sink_rows(self) -> int:
+        """Rows of the sink region: sink_frames * F rounded up to a multiple of 128."""
+        return (self.cfg.sink_frames * self.F + 127) // 128 * 128
+
     def sync(self, stream=None) -> None:
         _check(mla_cache_sync(self.handle, stream), "mla_cache_sync")
 
     def read_ring(self, b: int = 0):
-        """(ckv [W*F, 192], krope [W*F, 32]) fp16 of stream b in physical slot order, and the valid row count."""
+        """(ckv [rows, 192], krope [rows, 32]) fp16 of stream b in physical row order (rows =
+        sink rows + W*F, see mla_ring_slot), and the valid row count."""
         import torch
-        W = self.cfg.window_frames
-        ckv = torch.empty(W * self.F, self.cfg.d_latent, dtype=torch.float16)
-        kr = torch.empty(W * self.F, self.cfg.d_rope, dtype=torch.float16)
+        rows = self.sink_rows() + self.cfg.window_frames * self.F
+        ckv = torch.empty(rows, self.cfg.d_latent, dtype=torch.float16)
+        kr = torch.empty(rows, self.cfg.d_rope, dtype=torch.float16)
         n = mla_cache_read(self.handle, b, ckv, kr)
         return ckv, kr, n
 

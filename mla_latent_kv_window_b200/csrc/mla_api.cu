@@ -87,6 +87,14 @@ mla_status fail(mla_status s, const char* fmt, ...) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Rows of the sink region of a stream's planes: sink_frames * F rounded up to whole 128-key
+// tiles, so that no key tile mixes sink keys (attended with their own query rotation) and
+// window keys.
+int64_t sink_rows_of(const mla_config& c) {
+  const int64_t n = (int64_t)c.sink_frames * c.frame_h * c.frame_w;
+  return (n + 127) / 128 * 128;
+}
+
 // ------------------------------------------------------------------------------ tensor maps
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -158,11 +166,15 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 // Create-time derivation of the absorbed weights (fp32 accumulation, one bf16 rounding).
 // Wqcat rows, per head h: [h*224, h*224+192) = W_UK[h]^T W_Q[h], [h*224+192, h*224+224) = W_QR[h];
 // then [n_h*224, n_h*224+192) = W_DKV and [n_h*224+192, (n_h+1)*224) = W_KR.
+// With a low-rank query the head rows come precomposed in fp32: qabs_f32 [n_heads*192][hidden]
+// (W_UK[h]^T W_Q[h] W_DQ) and qr_f32 [n_heads*32][hidden] (W_QR W_DQ); w_q, w_qr, w_uk unused.
 __global__ void build_wqcat_kernel(const __nv_bfloat16* __restrict__ w_q,
                                    const __nv_bfloat16* __restrict__ w_qr,
                                    const __nv_bfloat16* __restrict__ w_dkv,
                                    const __nv_bfloat16* __restrict__ w_kr,
                                    const __nv_bfloat16* __restrict__ w_uk,
+                                   const float* __restrict__ qabs_f32,
+                                   const float* __restrict__ qr_f32,
                                    __nv_bfloat16* __restrict__ wqcat, int hidden, int n_heads,
                                    int d_nope) {
   const int k = blockIdx.x * blockDim.x + threadIdx.x;
@@ -171,7 +183,10 @@ __global__ void build_wqcat_kernel(const __nv_bfloat16* __restrict__ w_q,
   const int h = rowq / kQK;
   const int c = rowq % kQK;
   float acc = 0.f;
-  if (h < n_heads) {
+  if (h < n_heads && qabs_f32) {
+    acc = c < kLatent ? qabs_f32[(size_t)(h * kLatent + c) * hidden + k]
+                      : qr_f32[(size_t)(h * kRope + c - kLatent) * hidden + k];
+  } else if (h < n_heads) {
     if (c < kLatent) {
       for (int j = 0; j < d_nope; ++j) {
         const int r = h * d_nope + j;
@@ -190,6 +205,23 @@ __global__ void build_wqcat_kernel(const __nv_bfloat16* __restrict__ w_q,
 
 // W_OV[o][h*192 + c] = sum_j W_O[o][h*d_head + j] * W_UV[h*d_head + j][c], stored fp16 (it
 // multiplies the fp16 o_lat).
+// Create-time fp32 product for composing low-rank weights: per batch index z,
+//   C[z][m][n] = sum_k A(z, m, k) B(z, k, n),  A(z,m,k) = A[z*a_sz + m*a_sm + k*a_sk] (TA),
+//   B(z,k,n) = B[z*b_sz + k*b_sk + n] (TB), C row-major [M][N] per z at C + z*c_sz.
+template <typename TA, typename TB>
+__global__ void compose_kernel(const TA* __restrict__ A, int64_t a_sz, int64_t a_sm, int64_t a_sk,
+                               const TB* __restrict__ B, int64_t b_sz, int64_t b_sk,
+                               float* __restrict__ C, int64_t c_sz, int M, int N, int K) {
+  const int n = blockIdx.x * blockDim.x + threadIdx.x;
+  const int m = blockIdx.y;
+  const int z = blockIdx.z;
+  if (n >= N || m >= M) return;
+  const TA* a = A + z * a_sz + (int64_t)m * a_sm;
+  const TB* b = B + z * b_sz + n;
+  float acc = 0.f;
+  for (int k = 0; k < K; ++k) acc += (float)a[(int64_t)k * a_sk] * (float)b[(int64_t)k * b_sk];
+  C[z * c_sz + (int64_t)m * N + n] = acc;
+}
 __global__ void build_wov_kernel(const __nv_bfloat16* __restrict__ w_o,
                                  const __nv_bfloat16* __restrict__ w_uv,
                                  __half* __restrict__ wov, int hidden, int n_heads,
@@ -244,7 +276,8 @@ mla_status launch_gemm(const CUtensorMap& ma, const CUtensorMap& mb, const CUten
 struct mla_cache {
   mla_config cfg;
   int F = 0;
-  int64_t rows_per_stream = 0;     // (W + max_chunk) * F
+  int64_t rows_per_stream = 0;     // sink_rows + (W + max_chunk) * F
+  int64_t sink_rows = 0;           // sink region: sink_frames * F rounded up to 128 rows
   int64_t max_q_tokens = 0;        // max_chunk * F
   int64_t frames_appended = 0;
   float softmax_scale = 0.f;
@@ -278,6 +311,14 @@ struct mla_cache {
 };
 
 namespace {
+
+// Valid sink frames (vs) and valid window frames (vw) of a cache: the first sink_frames frames
+// ever appended are the sink, the newest W of the others the window.
+void valid_counts(const mla_cache* c, int64_t& vs, int64_t& vw) {
+  const int64_t A = c->frames_appended, S = c->cfg.sink_frames, W = c->cfg.window_frames;
+  vs = A < S ? A : S;
+  vw = A - vs < W ? A - vs : W;
+}
 
 cudaEvent_t take_event(mla_cache* c) {
   if (!c->pool.empty()) {
@@ -472,6 +513,22 @@ mla_status launch_attention(mla_cache* c, const __half* qp, int64_t qp_batch_str
   a.n_keys = (int32_t)n_keys;
   a.o_lat = o_lat;
   a.o_lat_batch_stride = o_lat_batch_stride;
+  // Sink keys (rows [0, sink_rows), valid below vs * F) are stored rotated at their absolute
+  // frame index, which is also their window-local one; the queries (rotated at absolute t) must
+  // meet them at their local t = absolute t + delta, delta = (vs + vw) - frames_appended: turn
+  // the temporal RoPE bands by delta (computed in double, rounded once).
+  int64_t vs, vw;
+  valid_counts(c, vs, vw);
+  a.sink_tiles = (int32_t)(c->sink_rows / 128);
+  a.sink_keys = (int32_t)(vs * c->F);
+  {
+    const double delta = (double)(vs + vw) - (double)c->frames_appended;
+    for (int p = 0; p < 16; ++p) a.sink_rot[p] = make_float2(1.f, 0.f);
+    for (int i = 0; i < cfg.rope_t / 2; ++i) {
+      const double ang = delta * std::pow(cfg.rope_base, -2.0 * i / cfg.rope_t);
+      a.sink_rot[i] = make_float2((float)std::cos(ang), (float)std::sin(ang));
+    }
+  }
   using Sm = mla::AttnSmem<kAttnStages>;
   dim3 grid((unsigned)((R + 127) / 128), (unsigned)cfg.batch);
   ProfScope p(c, MLA_KERNEL_ATTENTION, st, profile);
@@ -590,8 +647,12 @@ mla_status mla_config_check(const mla_config* cfg) {
     return fail(MLA_ERR_INVALID_ARGUMENT, "frame grid, window, chunk and batch must be >= 1");
   if (!(c.softmax_scale >= 0.f) || !std::isfinite(c.softmax_scale))
     return fail(MLA_ERR_INVALID_ARGUMENT, "softmax_scale must be finite and >= 0");
+  if (c.d_q < 0 || c.sink_frames < 0)
+    return fail(MLA_ERR_INVALID_ARGUMENT, "d_q and sink_frames must be >= 0");
+  if (c.sink_frames > (1 << 20))
+    return fail(MLA_ERR_INVALID_ARGUMENT, "sink_frames too large");
   const int64_t F = (int64_t)c.frame_h * c.frame_w;
-  const int64_t rows = (int64_t)(c.window_frames + (int64_t)c.max_chunk_frames) * F;
+  const int64_t rows = sink_rows_of(c) + (int64_t)(c.window_frames + (int64_t)c.max_chunk_frames) * F;
   if (rows > (int64_t)1 << 30 || (int64_t)c.max_chunk_frames * F * c.n_heads > (int64_t)1 << 30)
     return fail(MLA_ERR_INVALID_ARGUMENT, "window or chunk too large (row index overflow)");
   if ((int64_t)c.batch * rows * kQK > ((int64_t)1 << 40))
@@ -612,23 +673,27 @@ mla_status mla_ring_slot(const mla_config* cfg, int64_t frame, int32_t token, in
   const int64_t F = (int64_t)cfg->frame_h * cfg->frame_w;
   if (frame < 0 || token < 0 || token >= F)
     return fail(MLA_ERR_INVALID_ARGUMENT, "frame must be >= 0 and token in [0, F)");
-  *slot = (frame % cfg->window_frames) * F + token;
+  if (cfg->sink_frames < 0) return fail(MLA_ERR_INVALID_ARGUMENT, "sink_frames must be >= 0");
+  if (frame < cfg->sink_frames)
+    *slot = frame * F + token;
+  else
+    *slot = sink_rows_of(*cfg) + ((frame - cfg->sink_frames) % cfg->window_frames) * F + token;
   return MLA_OK;
 }
 
 size_t mla_ring_bytes(const mla_config* cfg) {
   if (!cfg || cfg->batch <= 0 || cfg->window_frames <= 0 || cfg->frame_h <= 0 ||
-      cfg->frame_w <= 0 || cfg->d_latent <= 0 || cfg->d_rope < 0)
+      cfg->frame_w <= 0 || cfg->d_latent <= 0 || cfg->d_rope < 0 || cfg->sink_frames < 0)
     return 0;
-  return (size_t)cfg->batch * cfg->window_frames * cfg->frame_h * cfg->frame_w *
-         (size_t)(cfg->d_latent + cfg->d_rope) * 2;
+  return (size_t)cfg->batch * (size_t)(cfg->sink_frames + cfg->window_frames) * cfg->frame_h *
+         cfg->frame_w * (size_t)(cfg->d_latent + cfg->d_rope) * 2;
 }
 
 size_t mla_cache_device_bytes(const mla_config* cfg) {
   if (mla_config_check(cfg) != MLA_OK) return 0;
   const mla_config& c = *cfg;
   const size_t F = (size_t)c.frame_h * c.frame_w;
-  const size_t rows = (size_t)(c.window_frames + c.max_chunk_frames) * F;
+  const size_t rows = (size_t)sink_rows_of(c) + (size_t)(c.window_frames + c.max_chunk_frames) * F;
   const size_t q = (size_t)c.max_chunk_frames * F;
   size_t b = 0;
   b += (size_t)c.batch * rows * kQK * 2;                   // ckv + krope (ring + chunk tail)
@@ -668,12 +733,15 @@ mla_status mla_cache_create(const mla_config* cfg, const mla_weights* w, void* s
   if (s != MLA_OK) return s;
   if (!w || !w->w_q || !w->w_qr || !w->w_dkv || !w->w_kr || !w->w_uk || !w->w_uv || !w->w_o)
     return fail(MLA_ERR_INVALID_ARGUMENT, "a weight pointer is NULL");
+  if (cfg->d_q > 0 && !w->w_dq)
+    return fail(MLA_ERR_INVALID_ARGUMENT, "d_q > 0 needs w_dq");
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
 
   mla_cache* c = new mla_cache();
   c->cfg = *cfg;
   c->F = cfg->frame_h * cfg->frame_w;
-  c->rows_per_stream = (int64_t)(cfg->window_frames + cfg->max_chunk_frames) * c->F;
+  c->sink_rows = sink_rows_of(*cfg);
+  c->rows_per_stream = c->sink_rows + (int64_t)(cfg->window_frames + cfg->max_chunk_frames) * c->F;
   c->max_q_tokens = (int64_t)cfg->max_chunk_frames * c->F;
   c->softmax_scale = cfg->softmax_scale > 0.f
                          ? cfg->softmax_scale
@@ -716,12 +784,44 @@ mla_status mla_cache_create(const mla_config* cfg, const mla_weights* w, void* s
   MLA_TRY(cudaMemsetAsync(c->o_lat, 0, q_rows * k.n_heads * kLatent * 2, st));
   MLA_TRY(cudaMemsetAsync(c->status, 0, 256, st));
 
+  // fp32 temporaries of the low-rank query composition, freed on every exit (after the
+  // stream synchronisation below on success).
+  struct DevTmp {
+    float* p = nullptr;
+    ~DevTmp() {
+      if (p) cudaFree(p);
+    }
+  } t_f32, qabs_f32, qr_f32;
   {
+    const __nv_bfloat16* w_q = (const __nv_bfloat16*)w->w_q;
+    const __nv_bfloat16* w_qr = (const __nv_bfloat16*)w->w_qr;
+    const __nv_bfloat16* w_uk = (const __nv_bfloat16*)w->w_uk;
+    if (k.d_q > 0) {
+      // Low-rank query ([VideoMLA] §4.1): the query projections read c_q = x W_DQ^T, so
+      // W_Qabs[h] = (W_UK[h]^T W_Q[h]) W_DQ and W_QR,eff = W_QR W_DQ, composed in fp32.
+      const __nv_bfloat16* w_dq = (const __nv_bfloat16*)w->w_dq;
+      const int dn = k.d_nope, dq = k.d_q, nh = k.n_heads;
+      MLA_TRY(cudaMalloc(&t_f32.p, (size_t)nh * kLatent * dq * 4));
+      MLA_TRY(cudaMalloc(&qabs_f32.p, (size_t)nh * kLatent * k.hidden * 4));
+      MLA_TRY(cudaMalloc(&qr_f32.p, (size_t)nh * kRope * k.hidden * 4));
+      // T[h][c][j] = sum_n W_UK[h*dn + n][c] W_Q[h*dn + n][j]
+      compose_kernel<__nv_bfloat16, __nv_bfloat16><<<dim3((dq + 255) / 256, kLatent, nh), 256, 0, st>>>(
+          w_uk, (int64_t)dn * kLatent, 1, kLatent, w_q, (int64_t)dn * dq, dq, t_f32.p,
+          (int64_t)kLatent * dq, kLatent, dq, dn);
+      MLA_TRY(cudaGetLastError());
+      // W_Qabs[h*192 + c][i] = sum_j T[h][c][j] W_DQ[j][i]
+      compose_kernel<float, __nv_bfloat16><<<dim3((k.hidden + 255) / 256, nh * kLatent, 1), 256, 0, st>>>(
+          t_f32.p, 0, dq, 1, w_dq, 0, k.hidden, qabs_f32.p, 0, nh * kLatent, k.hidden, dq);
+      MLA_TRY(cudaGetLastError());
+      // W_QR,eff[r][i] = sum_j W_QR[r][j] W_DQ[j][i]
+      compose_kernel<__nv_bfloat16, __nv_bfloat16><<<dim3((k.hidden + 255) / 256, nh * kRope, 1), 256, 0, st>>>(
+          w_qr, 0, dq, 1, w_dq, 0, k.hidden, qr_f32.p, 0, nh * kRope, k.hidden, dq);
+      MLA_TRY(cudaGetLastError());
+    }
     dim3 g((k.hidden + 255) / 256, (k.n_heads + 1) * kQK);
-    build_wqcat_kernel<<<g, 256, 0, st>>>(
-        (const __nv_bfloat16*)w->w_q, (const __nv_bfloat16*)w->w_qr,
-        (const __nv_bfloat16*)w->w_dkv, (const __nv_bfloat16*)w->w_kr,
-        (const __nv_bfloat16*)w->w_uk, c->wqcat, k.hidden, k.n_heads, k.d_nope);
+    build_wqcat_kernel<<<g, 256, 0, st>>>(w_q, w_qr, (const __nv_bfloat16*)w->w_dkv,
+                                          (const __nv_bfloat16*)w->w_kr, w_uk, qabs_f32.p,
+                                          qr_f32.p, c->wqcat, k.hidden, k.n_heads, k.d_nope);
     MLA_TRY(cudaGetLastError());
     dim3 g2((k.n_heads * kLatent + 255) / 256, k.hidden);
     build_wov_kernel<<<g2, 256, 0, st>>>((const __nv_bfloat16*)w->w_o,
@@ -784,21 +884,36 @@ mla_status mla_cache_append(mla_cache* c, const void* x, int32_t n_frames, void*
     return fail(MLA_ERR_INVALID_ARGUMENT, "too many frames in one append");
   const mla_config& cfg = c->cfg;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  // Only the last W frames of a long append survive in the ring.
-  const int skip = n_frames > cfg.window_frames ? n_frames - cfg.window_frames : 0;
+  const int64_t S = cfg.sink_frames, W = cfg.window_frames;
   const int64_t x_batch_rows = (int64_t)n_frames * c->F;
+  const int64_t frame_elems = c->F * (int64_t)cfg.hidden;
+  const __nv_bfloat16* xp = static_cast<const __nv_bfloat16*>(x);
+  int64_t t = c->frames_appended;   // absolute index of the next frame
+  int64_t left = n_frames;
   mla_status s = MLA_OK;
   {
     ProfScope p(c, MLA_KERNEL_APPEND, st);
-    // Frames t go to slots (t mod W): one launch per run of consecutive slots.
-    int64_t t = c->frames_appended + skip;
-    int64_t left = n_frames - skip;
-    const __nv_bfloat16* xp = static_cast<const __nv_bfloat16*>(x) + (int64_t)skip * c->F * cfg.hidden;
+    // 1. Frames that are still sink frames go to rows t * F of the sink region.
+    if (t < S) {
+      const int64_t nf = left < S - t ? left : S - t;
+      s = launch_latent_gemm(c, xp, nf * c->F, x_batch_rows, false, t, t * c->F, st);
+      xp += nf * frame_elems;
+      t += nf;
+      left -= nf;
+    }
+    // 2. Of the rest, only the last W frames survive in the ring.
+    if (left > W) {
+      xp += (left - W) * frame_elems;
+      t += left - W;
+      left = W;
+    }
+    // 3. Window frames go to ring slots ((t - S) mod W): one launch per run of consecutive slots.
     while (left > 0 && s == MLA_OK) {
-      const int64_t slot = t % cfg.window_frames;
-      const int64_t nf = left < cfg.window_frames - slot ? left : cfg.window_frames - slot;
-      s = launch_latent_gemm(c, xp, nf * c->F, x_batch_rows, false, t, slot * c->F, st);
-      xp += nf * c->F * cfg.hidden;
+      const int64_t slot = (t - S) % W;
+      const int64_t nf = left < W - slot ? left : W - slot;
+      s = launch_latent_gemm(c, xp, nf * c->F, x_batch_rows, false, t,
+                             c->sink_rows + slot * c->F, st);
+      xp += nf * frame_elems;
       t += nf;
       left -= nf;
     }
@@ -819,9 +934,9 @@ mla_status mla_window_attention(mla_cache* c, const void* x_chunk, int32_t n_fra
     return fail(MLA_ERR_INVALID_ARGUMENT, "x_chunk and out must be 16-byte aligned");
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const int64_t nq = (int64_t)n_frames * c->F;
-  const int64_t valid = c->frames_appended < cfg.window_frames ? c->frames_appended
-                                                               : cfg.window_frames;
-  const int64_t base_row = valid * c->F;
+  int64_t vs, vw;
+  valid_counts(c, vs, vw);
+  const int64_t base_row = c->sink_rows + vw * c->F;   // chunk latents go right after the window
   const int64_t n_keys = base_row + nq;
   mla_status s;
 
@@ -879,9 +994,9 @@ mla_status mla_window_attention_noalloc(mla_cache* c, const void* x_chunk, int32
   __half* o_lat = reinterpret_cast<__half*>(static_cast<unsigned char*>(scratch) + qp_bytes);
 
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const int64_t valid = c->frames_appended < cfg.window_frames ? c->frames_appended
-                                                               : cfg.window_frames;
-  const int64_t base_row = valid * c->F;
+  int64_t vs, vw;
+  valid_counts(c, vs, vw);
+  const int64_t base_row = c->sink_rows + vw * c->F;
   const int64_t n_keys = base_row + nq;
 
   // 1. absorbed queries (into the scratch) + chunk latents (into the cache's chunk tail)
@@ -950,9 +1065,11 @@ mla_status mla_dense_sync(void* stream) {
 mla_status mla_cache_state(const mla_cache* c, int64_t* frames_appended, int32_t* valid) {
   if (!c) return fail(MLA_ERR_INVALID_ARGUMENT, "NULL cache");
   if (frames_appended) *frames_appended = c->frames_appended;
-  if (valid)
-    *valid = (int32_t)(c->frames_appended < c->cfg.window_frames ? c->frames_appended
-                                                                 : c->cfg.window_frames);
+  if (valid) {
+    int64_t vs, vw;
+    valid_counts(c, vs, vw);
+    *valid = (int32_t)(vs + vw);
+  }
   return MLA_OK;
 }
 
@@ -969,7 +1086,7 @@ mla_status mla_cache_read(const mla_cache* c, int32_t b, void* ckv_host, void* k
                           int64_t* n_valid_rows) {
   if (!c) return fail(MLA_ERR_INVALID_ARGUMENT, "NULL cache");
   if (b < 0 || b >= c->cfg.batch) return fail(MLA_ERR_INVALID_ARGUMENT, "stream index out of range");
-  const int64_t ring = (int64_t)c->cfg.window_frames * c->F;
+  const int64_t ring = c->sink_rows + (int64_t)c->cfg.window_frames * c->F;
   if (ckv_host)
     MLA_CUDA(cudaMemcpy(ckv_host, c->ckv + (int64_t)b * c->rows_per_stream * kLatent,
                         ring * kLatent * 2, cudaMemcpyDeviceToHost));
@@ -977,9 +1094,9 @@ mla_status mla_cache_read(const mla_cache* c, int32_t b, void* ckv_host, void* k
     MLA_CUDA(cudaMemcpy(krope_host, c->krope + (int64_t)b * c->rows_per_stream * kRope,
                         ring * kRope * 2, cudaMemcpyDeviceToHost));
   if (n_valid_rows) {
-    const int64_t v = c->frames_appended < c->cfg.window_frames ? c->frames_appended
-                                                                : c->cfg.window_frames;
-    *n_valid_rows = v * c->F;
+    int64_t vs, vw;
+    valid_counts(c, vs, vw);
+    *n_valid_rows = (vs + vw) * c->F;
   }
   return MLA_OK;
 }

@@ -29,7 +29,13 @@
 //               only when the max grows by > 2^8), ex2, P_j as fp16 into TMEM; finally O / l ->
 //               fp16 o_lat, staged in shared memory and written by one bulk copy per row.
 //
-// TMEM columns: S [0,128), P [128,192), Q [192,304), O [304,496).
+// TMEM columns: S [0,128), P [128,192), Q [192,304), O [304,496), QS [496,512).
+//
+// Sink keys ([VideoMLA] App. D.4/D.5 "sink + local window"): the first sink_tiles key tiles
+// hold the sink frames (rows past sink_keys are padding and are masked).  Their k_rope was
+// rotated at the sink frame's absolute index, which is also its window-local one, while Qp
+// was rotated at the query's absolute index; so for sink tiles the two RoPE k-steps of S take
+// QS, the query's RoPE part turned by the temporal offset between the two (sink_rot).
 // Launched with programmatic stream serialization: barrier init, TMEM allocation and the
 // tensor-map prefetch overlap the projection kernel's tail; griddepcontrol.wait precedes the first
 // global access.
@@ -61,6 +67,7 @@ constexpr uint32_t kTmemS = 0;
 constexpr uint32_t kTmemP = 128;
 constexpr uint32_t kTmemQ = 192;
 constexpr uint32_t kTmemO = 304;
+constexpr uint32_t kTmemQS = 496;   // RoPE part of Q turned for the sink keys (2 k-steps)
 
 struct AttnArgs {
   const __half* qp;            // [batch][qp_rows][224] fp16
@@ -69,6 +76,9 @@ struct AttnArgs {
   int32_t n_keys;              // keys per stream (window + chunk)
   __half* o_lat;               // fp16
   int64_t o_lat_batch_stride;  // elements
+  int32_t sink_tiles;          // leading key tiles that hold sink frames (0: no sink)
+  int32_t sink_keys;           // valid sink keys; keys [sink_keys, 128 * sink_tiles) are padding
+  float2 sink_rot[16];         // (cos, sin) turning each RoPE pair of Q for the sink keys
 };
 
 template <int KV_STAGES>
@@ -158,16 +168,20 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         if (j >= 1 && !mbar_wait(s_free, (uint32_t)(j - 1) & 1u, status)) break;
         tc_fence_after();
         const uint32_t kv_base = smem_u32(smem + L::kKV + st * L::kTileBytes);
+        const bool sink_tile = (j + rot) % nt < args.sink_tiles;
 #pragma unroll
         for (int kk = 0; kk < 14; ++kk) {
           // A = Q from TMEM: 16 fp16 of K per step = 8 packed columns.
           uint64_t db;
-          if (kk < 12)
+          uint32_t qa = tmem + kTmemQ + kk * 8;
+          if (kk < 12) {
             db = smem_desc(kv_base + (kk >> 2) * L::kAtomC + (kk & 3) * 32, 16, 1024,
                            kSwizzle128B);
-          else
+          } else {
             db = smem_desc(kv_base + 3 * L::kAtomC + (kk - 12) * 32, 16, 512, kSwizzle64B);
-          umma_ts(tmem + kTmemS, tmem + kTmemQ + kk * 8, db, idesc_s, kk > 0 ? 1u : 0u);
+            if (sink_tile) qa = tmem + kTmemQS + (kk - 12) * 8;
+          }
+          umma_ts(tmem + kTmemS, qa, db, idesc_s, kk > 0 ? 1u : 0u);
         }
         tc_commit(s_full);
       }
@@ -220,10 +234,21 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           q[4 * i + 2] = v.z;
           q[4 * i + 3] = v.w;
         }
-        if (c < 3)
+        if (c < 3) {
           tmem_st32(tmem + kTmemQ + lane_off + c * 32, q);
-        else
+        } else {
           tmem_st16(tmem + kTmemQ + lane_off + 96, q);      // columns [96, 112)
+          if (args.sink_tiles > 0) {
+            // QS: pair p of the RoPE part (packed column p) turned by sink_rot[p].
+#pragma unroll
+            for (int p = 0; p < 16; ++p) {
+              const float2 v = __half22float2(*reinterpret_cast<const __half2*>(&q[p]));
+              const float2 r = args.sink_rot[p];
+              q[p] = pack_f16x2(v.x * r.x - v.y * r.y, v.x * r.y + v.y * r.x);
+            }
+            tmem_st16(tmem + kTmemQS + lane_off, q);
+          }
+        }
       }
       tmem_st_wait();
       tc_fence_before();
@@ -246,7 +271,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       tc_fence_before();
       mbar_arrive(s_free);
 
-      const int valid = n_keys - ((j + rot) % nt) * kTileKeys;   // keys of this tile that exist
+      // Keys of this tile that exist: below n_keys, and for a sink tile below sink_keys.
+      const int tile = (j + rot) % nt;
+      const int valid = (tile < args.sink_tiles ? args.sink_keys : n_keys) - tile * kTileKeys;
       if (valid < kTileKeys) {
 #pragma unroll
         for (int i = 0; i < kTileKeys; ++i)
@@ -263,7 +290,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       float alpha = 1.f;
       bool rescale = false;
       if (j == 0) {
-        m_used = mx;
+        m_used = fmaxf(mx, -1e30f);   // finite even if the first tile is all padding
       } else if (mx > m_used + kRescaleThreshold) {
         alpha = ex2_approx(m_used - mx);
         m_used = mx;

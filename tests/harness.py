@@ -37,7 +37,8 @@ def assert_close(gpu, ref, what: str, rel_tol: float = REL_L2, max_tol: float = 
 
 def dims_of(w: mla_synth.Workload) -> dict:
     d = dict(w.dims)
-    d.update(frame_h=w.frame_h, frame_w=w.frame_w, window_frames=w.window_frames)
+    d.update(frame_h=w.frame_h, frame_w=w.frame_w, window_frames=w.window_frames,
+             sink_frames=w.sink_frames)
     return d
 
 
@@ -53,7 +54,8 @@ class Pair:
         self.weights = weights if weights is not None else mla_synth.make_weights(dict(w.dims), mla_synth.weight_seed(w, layer))
         dev_w = {k: v.cuda() for k, v in self.weights.items()}
         self.gpu = LatentWindowCache(dict(w.dims), dev_w, w.frame_h, w.frame_w, w.window_frames,
-                                     max_chunk_frames or w.query_frames, batch=w.batch)
+                                     max_chunk_frames or w.query_frames, batch=w.batch,
+                                     sink_frames=w.sink_frames)
         self.oracles = [OracleLayer(self.dims, self.weights) for _ in range(w.batch)]
         self.scales = mla_synth.stream_scales(w.batch, w.seed) if w.stream_scale else None
 

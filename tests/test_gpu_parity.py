@@ -26,15 +26,17 @@ def small(frame_h=4, frame_w=6, window=2, fill=2, q=1, batch=1, seed=0, scale=Fa
 
 
 def check_ring(pair: Pair, what: str):
-    """Every valid frame f sits at slots (f mod W) F + k with the oracle's c_kv and k_rope."""
+    """Every valid frame f sits at slots (f mod W) F + k with the oracle's c_kv and k_rope (with
+    a sink: at the rows mla_ring_slot names, which the host tests pin against a FIFO simulation)."""
     W, F = pair.w.window_frames, pair.F
     for b, orc in enumerate(pair.oracles):
         ckv, kr, n_valid = pair.gpu.read_ring(b)
         contents = orc.cache_contents()
         assert n_valid == len(contents) * F
         for f, c, r in contents:
-            s0 = ring_slot(f, 0, W, F)
-            assert s0 == pair.gpu_slot(f, 0)
+            s0 = pair.gpu_slot(f, 0)
+            if not pair.w.sink_frames:
+                assert s0 == ring_slot(f, 0, W, F)
             assert_close(ckv[s0:s0 + F], c, f"{what}: c_kv of frame {f} (stream {b})")
             assert_close(kr[s0:s0 + F], r, f"{what}: k_rope of frame {f} (stream {b})")
 
@@ -45,11 +47,12 @@ def oracle_qp(pair: Pair, x_chunk, b: int):
     d = pair.dims
     ctx = orc.keys_and_queries(x_chunk, positions="absolute")
     rows = []
+    xq = orc.query_input(ctx["x"])
     for h in range(d["n_heads"]):
         dn, dr = d["d_nope"], d["d_rope"]
-        q_nope = ctx["x"] @ orc.W["w_q"][h * dn:(h + 1) * dn].T
+        q_nope = xq @ orc.W["w_q"][h * dn:(h + 1) * dn].T
         q_abs = q_nope @ orc.W["w_uk"][h * dn:(h + 1) * dn]
-        q_rope = rope3d(ctx["x"] @ orc.W["w_qr"][h * dr:(h + 1) * dr].T, ctx["t_q"], ctx["h_q"], ctx["w_q"],
+        q_rope = rope3d(xq @ orc.W["w_qr"][h * dr:(h + 1) * dr].T, ctx["t_q"], ctx["h_q"], ctx["w_q"],
                         d["rope_t"], d["rope_h"], d["rope_w"], d["rope_base"])
         rows.append(np.concatenate([q_abs, q_rope], axis=1) * orc.scale * LOG2E)
     return np.stack(rows, axis=1).reshape(-1, 224)
@@ -238,3 +241,65 @@ def test_wan_30_layers_4_steps_wrapped():
             assert_close(kr[s0:s0 + w.F], r, "appended chunk k_rope")
         p.check_status()
         p.gpu.close()
+
+
+# ---------------------------------------------------------------------------- next rows
+def test_paper_dims_tiny():
+    # [VideoMLA] §4.1 defaults: 96/32 key split (scale 1/sqrt(128)), low-rank query d_q = 768,
+    # RoPE (6,5,5) pairs; every element against the oracle's low-rank path.
+    w = mla_synth.WORKLOADS["paper_tiny"]
+    p = Pair(w)
+    p.append(p.hidden(w.fill_frames, mla_synth.fill_seed(w, 0)))
+    check_ring(p, "paper dims")
+    full_check(p, p.hidden(w.query_frames, mla_synth.chunk_seed(w, 0, 0)), "paper dims")
+
+
+def test_paper_dims_w21_full_size():
+    w = mla_synth.WORKLOADS["paper_w21_q1"]
+    p = Pair(w)
+    p.append(p.hidden(w.fill_frames, mla_synth.fill_seed(w, 0)))
+    sampled_check(p, p.hidden(1, mla_synth.chunk_seed(w, 0, 0)), "paper dims, 21-frame window", 64, 5)
+
+
+def test_sink_tiny_through_wraps():
+    # 1 sink frame + a 2-frame window: appends of 1, 1, 3 and 1 frames (the window slides and
+    # wraps while frame 0 stays); every element checked after each stage, including a chunk that
+    # sees the sink, the window and itself at App. D.5 window-local positions.
+    w = mla_synth.WORKLOADS["sink_tiny"]
+    p = Pair(w, max_chunk_frames=2)
+    seed = 700
+    for n in (1, 1, 3, 1):
+        p.append(p.hidden(n, seed))
+        seed += 1
+        check_ring(p, f"sink: after append of {n}")
+        full_check(p, p.hidden(2, seed), f"sink: chunk after append of {n}")
+        seed += 1
+    assert p.gpu.state() == (6, 3)
+
+
+def test_sink_ragged_tiles():
+    # F = 200 (sink region padded from 200 to 256 rows), window of 3, 2-frame chunks.
+    w = mla_synth.Workload("sink_ragged", frame_h=10, frame_w=20, window_frames=3, fill_frames=6,
+                           query_frames=2, seed=19, sink_frames=1)
+    p = Pair(w, max_chunk_frames=2)
+    p.append(p.hidden(6, 720))
+    check_ring(p, "sink ragged")
+    full_check(p, p.hidden(2, 721), "sink ragged")
+
+
+def test_sink_w6_q3_full_size():
+    # The long-rollout configuration: 1 sink frame + 6 recent frames (10,920 cached keys) and a
+    # 3-frame chunk, after 10 appended frames (the window has wrapped).
+    w = mla_synth.WORKLOADS["sink_w6_q3"]
+    p = Pair(w)
+    p.append(p.hidden(w.fill_frames, mla_synth.fill_seed(w, 0)))
+    assert p.gpu.state() == (10, 7)
+    ckv, kr, n = p.gpu.read_ring(0)
+    contents = p.oracles[0].cache_contents()
+    assert [f for f, _, _ in contents] == [0, 4, 5, 6, 7, 8, 9]
+    for f, c, r in (contents[0], contents[1], contents[-1]):
+        s0 = p.gpu_slot(f, 0)
+        assert_close(ckv[s0:s0 + w.F], c, f"c_kv frame {f}")
+        assert_close(kr[s0:s0 + w.F], r, f"k_rope frame {f}")
+    sampled_check(p, p.hidden(3, mla_synth.chunk_seed(w, 0, 0)), "sink + 6-frame window", 64, 6)
+

@@ -17,7 +17,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 def cfg(**over):
     d = dict(mla_synth.DIMS_WAN13B)
-    kw = dict(frame_h=30, frame_w=52, window_frames=21, max_chunk_frames=3, batch=1)
+    kw = dict(frame_h=30, frame_w=52, window_frames=21, max_chunk_frames=3, batch=1, sink_frames=0)
     kw.update({k: over.pop(k) for k in list(over) if k in kw})
     d.update(over)
     return B.make_config(d, **kw)
@@ -46,8 +46,12 @@ def test_config_check():
     assert B.mla_config_check(cfg(d_latent=128)) == B.MLA_ERR_UNSUPPORTED
     assert b"d_latent" in B.load_library().mla_last_error()
     assert B.mla_config_check(cfg(hidden=1600)) == B.MLA_ERR_UNSUPPORTED
-    # the paper's default (6,5,5)-pair split is valid
+    # the paper's default (6,5,5)-pair split, 96/32 split and d_q = 768 are valid, and a sink
     assert B.mla_config_check(cfg(rope_t=12, rope_h=10, rope_w=10)) == B.MLA_OK
+    assert B.mla_config_check(cfg(d_nope=96, d_q=768)) == B.MLA_OK
+    assert B.mla_config_check(cfg(sink_frames=1, window_frames=6)) == B.MLA_OK
+    for over in (dict(d_q=-1), dict(sink_frames=-1)):
+        assert B.mla_config_check(cfg(**over)) == B.MLA_ERR_INVALID_ARGUMENT, over
 
 
 def test_ring_slot_matches_oracle_exactly():
@@ -61,6 +65,33 @@ def test_ring_slot_matches_oracle_exactly():
         B.mla_ring_slot(cfg(), -1, 0)
     with pytest.raises(B.MLAError):
         B.mla_ring_slot(cfg(), 0, 1560)
+
+
+def test_ring_slot_with_sink_matches_fifo_simulation():
+    # Sink frames keep their own buffer for good (rows f*F of a sink region rounded up to whole
+    # 128-row key tiles); the other frames cycle through W window buffers like a FIFO.  The
+    # closed form of mla_ring_slot must name the same row as this simulation.
+    from collections import deque
+    for S, W, fh, fw in ((1, 6, 30, 52), (1, 2, 4, 6), (2, 3, 3, 5), (3, 1, 1, 1)):
+        F = fh * fw
+        sink_rows = -(-S * F // 128) * 128
+        c = cfg(window_frames=W, frame_h=fh, frame_w=fw, sink_frames=S)
+        fifo, owner, fresh = deque(), {}, 0
+        for f in range(S + 3 * W + 2):
+            if f < S:
+                owner[f] = ("sink", f)
+            else:
+                if len(fifo) == W:
+                    buf = owner.pop(fifo.popleft())[1]
+                else:
+                    buf, fresh = fresh, fresh + 1
+                owner[f] = ("win", buf)
+                fifo.append(f)
+            for g, (kind, buf) in owner.items():
+                row0 = buf * F if kind == "sink" else sink_rows + buf * F
+                for k in sorted({0, F // 2, F - 1}):
+                    assert B.mla_ring_slot(c, g, k) == row0 + k, (S, W, g, k)
+        assert B.mla_ring_bytes(c) == (S + W) * F * 224 * 2
 
 
 def test_ring_bytes_reproduce_printed_accounting():
