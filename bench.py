@@ -337,6 +337,7 @@ def run_ours(args, rank, local, world):
 
     status_ok = all(B.mla_cache_sync(c.handle) == 0 for c in caches)
     layout = layout_baseline(B, w, dims, dev, stream, attn_ms, attn_flop) if rank == 0 else None
+    nxt = next_rows(B, dev) if rank == 0 else None
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -390,6 +391,8 @@ def run_ours(args, rank, local, world):
         }
         if layout is not None:
             line["layout_baseline"] = layout
+        if nxt is not None:
+            line["next_rows"] = nxt
         if cpu is not None:
             line["cpu_baseline"] = cpu
         print(json.dumps(line), flush=True)
@@ -467,6 +470,54 @@ def layout_baseline(B, w, dims, dev, stream, latent_ms, latent_flop):
             "cache_bytes_per_layer": cache_bytes(224, 63), "status_ok": ok63},
         "note": "dense counts 512 flop per (query, head, key); latent 832 (absorbed scores + P.c_kv)",
     }
+
+
+def next_rows(B, dev):
+    """Per-launch times of the rows after the main path: the paper-default dims (96/32 split,
+    d_q = 768, RoPE (6,5,5) pairs) on the 21-frame one-frame step, and 1 sink frame + a 6-frame
+    window with 3-frame chunks (the long-rollout configuration)."""
+    import torch
+
+    import mla_synth
+    res = {}
+    for name, chunk_frames in (("paper_w21_q1", 1), ("sink_w6_q3", 3)):
+        w = mla_synth.WORKLOADS[name]
+        dims = dict(w.dims)
+        F = w.F
+        wts = {k: v.to(dev) for k, v in mla_synth.make_weights(dims, mla_synth.weight_seed(w, 0)).items()}
+        c = B.LatentWindowCache(dims, wts, w.frame_h, w.frame_w, w.window_frames, chunk_frames,
+                                sink_frames=w.sink_frames)
+        c.append(mla_synth.make_hidden(1, w.fill_frames * F, dims["hidden"], mla_synth.fill_seed(w, 0)).to(dev))
+        x = mla_synth.make_hidden(1, chunk_frames * F, dims["hidden"], mla_synth.chunk_seed(w, 0, 0)).to(dev)
+        out = torch.empty_like(x)
+        B.mla_cache_profile_enable(c.handle, True)
+        for _ in range(3):
+            c.attention(x, out)
+        torch.cuda.synchronize()
+        B.mla_cache_profile_read(c.handle)
+        reps = 10
+        for _ in range(reps):
+            c.attention(x, out)
+        torch.cuda.synchronize()
+        prof = B.mla_cache_profile_read(c.handle)
+        ok = B.mla_cache_sync(c.handle) == 0
+        _, valid = c.state()
+        c.close()
+        nq = chunk_frames * F
+        keys = valid * F + nq
+        a_ms = prof["attention"][0] / max(prof["attention"][1], 1)
+        call_ms = sum(t for t, _ in prof.values()) / reps
+        flop = FLOP_PER_QHK * nq * dims["n_heads"] * keys
+        res[name] = {
+            "keys": keys, "query_tokens": nq,
+            "attention_ms": round(a_ms, 4), "attention_tflops": round(flop / (a_ms / 1e3) / 1e12, 1),
+            "call_ms": round(call_ms, 4), "query_tokens_per_s": round(nq / (call_ms / 1e3), 1),
+            "kernel_ms_per_launch": {k: round(t / max(n, 1), 5) for k, (t, n) in prof.items() if n},
+            "status_ok": ok,
+        }
+    res["note"] = ("attention TFLOP/s at 832 flop per (query, head, key) over the valid keys (sink "
+                   "padding rows excluded); call = query projection + attention + output projection")
+    return res
 
 
 # ---------------------------------------------------------------------------- the oracle on CPU
