@@ -111,7 +111,9 @@ mla_status mla_ring_slot(const mla_config* cfg, int64_t frame, int32_t token, in
 size_t mla_ring_bytes(const mla_config* cfg);
 
 /* Bytes of device memory mla_cache_create allocates for this configuration (ring with its
- * chunk tail, absorbed weights, per-call scratch, status word).  0 for an invalid config. */
+ * chunk tail, absorbed weights, per-call scratch, status word, RoPE tables, and the per-head
+ * weights of mla_window_attention_reconstruct when the configuration allows that call).
+ * 0 for an invalid config. */
 size_t mla_cache_device_bytes(const mla_config* cfg);
 
 /* Create a cache on the current device.  Derives and owns the absorbed weights
@@ -166,6 +168,21 @@ mla_status mla_window_attention(mla_cache* c, const void* x_chunk, int32_t n_fra
  *  - Arguments, layouts, stream ordering and errors otherwise as mla_window_attention. */
 mla_status mla_window_attention_noalloc(mla_cache* c, const void* x_chunk, int32_t n_frames,
                                         void* out, void* stream);
+
+/* The same attention call computed the training-time way ([VideoMLA] §3.3): per-head keys
+ * K_h = [c W_UK[h]^T | k_rope] and values V_h = c W_UV[h]^T are materialised for every key of
+ * the window and the chunk, the per-head queries [q_nope | RoPE3D(q_rope)] are projected, dense
+ * per-head softmax attention runs over them, and out = concat_h(o_h) W_O^T.  Same arguments and
+ * the same result (up to rounding) as mla_window_attention; it exists to measure where
+ * reconstruct-then-dense beats the absorbed kernel (per (query, head, key) it needs 512 flop
+ * instead of 832, plus the reconstruction of every key for every call).
+ *  - Needs d_nope + d_rope == 128, d_head == 128 (the paper's default dims), d_nope a multiple
+ *    of 32, and sink_frames == 0; otherwise MLA_ERR_UNSUPPORTED.
+ *  - The first call allocates the dense per-call buffers (per-head K and V of the largest
+ *    window: 2 x batch x (W + max_chunk_frames) x F x n_heads x 256 bytes, plus the per-head
+ *    queries and outputs of one chunk); they live until mla_cache_destroy. */
+mla_status mla_window_attention_reconstruct(mla_cache* c, const void* x_chunk, int32_t n_frames,
+                                            void* out, void* stream);
 
 /* Dense per-head attention, the layout VideoMLA replaces ([VideoMLA] §1: every cached token
  * keeps 12 x 128 keys and 12 x 128 values, 3,072 scalars): the measurement baseline of the

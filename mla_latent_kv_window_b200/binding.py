@@ -27,6 +27,7 @@ KERNEL_NAMES = ("append", "qproj", "attention", "oproj")
 EXPORTED = (
     "mla_config_check", "mla_ring_slot", "mla_ring_bytes", "mla_cache_device_bytes",
     "mla_cache_create", "mla_cache_append", "mla_window_attention", "mla_window_attention_noalloc",
+    "mla_window_attention_reconstruct",
     "mla_cache_destroy", "mla_dense_attention", "mla_dense_sync",
     "mla_cache_state", "mla_cache_sync", "mla_cache_read", "mla_cache_debug_buffers", "mla_cache_copy_buffer",
     "mla_cache_profile_enable", "mla_cache_profile_read", "mla_status_string", "mla_last_error",
@@ -86,6 +87,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "mla_cache_append": (I32, [VP, VP, I32, VP]),
         "mla_window_attention": (I32, [VP, VP, I32, VP, VP]),
         "mla_window_attention_noalloc": (I32, [VP, VP, I32, VP, VP]),
+        "mla_window_attention_reconstruct": (I32, [VP, VP, I32, VP, VP]),
         "mla_dense_attention": (I32, [VP, VP, VP, VP, I32, I32, I32, I32, I32, ctypes.c_float, VP]),
         "mla_dense_sync": (I32, [VP]),
         "mla_cache_destroy": (None, [VP]),
@@ -190,6 +192,13 @@ def mla_window_attention_noalloc(cache: int, x_chunk, n_frames: int, out, stream
            "mla_window_attention_noalloc")
 
 
+def mla_window_attention_reconstruct(cache: int, x_chunk, n_frames: int, out, stream=None) -> None:
+    """mla_window_attention computed as reconstruct-then-dense (per-head K/V materialised)."""
+    _check(load_library().mla_window_attention_reconstruct(cache, _dev_ptr(x_chunk, "x_chunk"), n_frames,
+                                                           _dev_ptr(out, "out"), _stream_handle(stream)),
+           "mla_window_attention_reconstruct")
+
+
 def mla_dense_attention(q, k, v, out, softmax_scale: float = 0.0, stream=None) -> None:
     """Dense per-head attention baseline: q [B, n_q, H, 128], k/v [B, n_kv, H, 128], out like q (bf16)."""
     B, nq, H, D = q.shape
@@ -274,6 +283,13 @@ class LatentWindowCache:
         if out is None:
             out = torch.empty_like(x_chunk)
         mla_window_attention(self.handle, x_chunk, x_chunk.shape[-2] // self.F, out, stream)
+        return out
+
+    def attention_reconstruct(self, x_chunk, out=None, stream=None):
+        import torch
+        if out is None:
+            out = torch.empty_like(x_chunk)
+        mla_window_attention_reconstruct(self.handle, x_chunk, x_chunk.shape[-2] // self.F, out, stream)
         return out
 
     def state(self):

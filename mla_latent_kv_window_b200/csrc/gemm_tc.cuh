@@ -42,6 +42,10 @@
 //               contiguous row range per stream).  The latent path is 16-bit like the paper's
 //               cache; fp16 keeps three more mantissa bits than bf16 for the same bytes.
 //   RoPE applies to the chunks with col mod 224 == 192 (every 224-column block is 192 + 32).
+//   kEpiDense   bf16 to map_o0 at column (col / head_in) * head_out + col % head_in (identity
+//               when head_in == 0), with RoPE on the chunks where col mod rope_period ==
+//               rope_period - 32 (none when rope_period == 0): the per-head Q, K and V of the
+//               reconstruct-then-dense form (head-interleaved [n_h][128] rows).
 //
 // The latent epilogue is the fused "append" of the VideoMLA paper page: c_kv = x W_DKV^T and
 // the decoupled positional key k_R = RoPE3D(x W_KR^T) (§3.1, §3.2), one head-shared copy per
@@ -54,6 +58,7 @@ namespace mla {
 
 constexpr int kEpiStore = 0;
 constexpr int kEpiLatent = 1;
+constexpr int kEpiDense = 2;
 constexpr int kGemmThreads = 352;
 constexpr int kEpiWarps = 8;       // two per TMEM lane quarter, each owning half of every row
 
@@ -76,6 +81,8 @@ struct EpiArgs {
   RopeBands rope;
   const float2* rope_hw;     // (cos, sin) tables: [16][frame_h] for h, then [16][frame_w] for w
   int32_t frame_h;
+  int32_t head_in, head_out; // kEpiDense: output column remap (0: identity)
+  int32_t rope_period;       // kEpiDense: RoPE on chunks with col % rope_period == rope_period - 32
 };
 
 template <int BN, int A_STAGES, int B_STAGES, int M_SUB = 1>
@@ -317,9 +324,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       // The RoPE chunk of this warp's columns (at most one: one per 224 columns); its factors
       // are formed now, while the tile's MMAs still run.
       int rc = -1;
-      if constexpr (kEpi == kEpiLatent) {
-        for (int c = c_lo; c < c_hi; ++c)
-          if ((col_base + c * 32) % 224 == 192) rc = c;
+      if constexpr (kEpi == kEpiLatent || kEpi == kEpiDense) {
+        const int rp = kEpi == kEpiLatent ? 224 : ep.rope_period;
+        if (rp > 0)
+          for (int c = c_lo; c < c_hi; ++c)
+            if ((col_base + c * 32) % rp == rp - 32) rc = c;
         if (rc >= 0) {
           const int F = ep.tokens_per_frame;
           const int fi = m / F;                // frame within this launch
@@ -353,6 +362,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
         for (int q = 0; q < 32; ++q) v[q] = __uint_as_float(cur[q]);
         const int col = col_base + c * 32;
+        if constexpr (kEpi == kEpiDense) {
+          if (c == rc) rope_apply(v, rf);
+        }
         if constexpr (kEpi == kEpiLatent) {
           if (c == rc) rope_apply(v, rf);
           if (col < ep.latent_col0) {
@@ -388,6 +400,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 tma_store_3d(&map_o1, box_base, j, row0, z);
               else
                 tma_store_3d(&map_o2, box_base, j - 192, row0, z);
+            } else if constexpr (kEpi == kEpiDense) {
+              const int x = ep.head_in ? (col / ep.head_in) * ep.head_out + col % ep.head_in : col;
+              tma_store_3d(&map_o0, box_base, x, row0, z);
             } else {
               tma_store_3d(&map_o0, box_base, col, row0, z);
             }

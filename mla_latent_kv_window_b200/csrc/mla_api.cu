@@ -48,7 +48,7 @@ constexpr int kProjNarrowAStages = 8;   // 32-column latent blocks: 8 x 16 KB + 
 constexpr int kProjNarrowBStages = 4;
 constexpr int kProjMidAStages = 4;      // 256 x 160 tiles: 4 x 32 KB + 3 x 20 KB
 constexpr int kProjMidBStages = 3;
-constexpr int kOutBN = 192;             // output projection column block
+constexpr int kOutBN = 192;             // output projection column block (also the dense form's GEMMs)
 constexpr int kOutAStages = 6;
 constexpr int kOutBStages = 3;
 
@@ -247,6 +247,46 @@ mla_status set_smem(K kernel, int bytes) {
   return MLA_OK;
 }
 
+// Per-head query weight of the dense form: rows h*128 + j = W_Q[h*d_nope + j] (j < d_nope),
+// W_QR[h*32 + j - d_nope] (j >= d_nope); with a low-rank query the fp32 compositions with W_DQ.
+__global__ void build_wqd_kernel(const __nv_bfloat16* __restrict__ w_q,
+                                 const __nv_bfloat16* __restrict__ w_qr,
+                                 const float* __restrict__ qeff_f32, const float* __restrict__ qreff_f32,
+                                 __nv_bfloat16* __restrict__ wqd, int hidden, int n_heads, int d_nope) {
+  const int k = blockIdx.x * blockDim.x + threadIdx.x;
+  const int row = blockIdx.y;  // h*128 + j
+  if (k >= hidden) return;
+  const int h = row / 128, j = row % 128;
+  float v;
+  if (j < d_nope) {
+    const size_t r = (size_t)(h * d_nope + j) * hidden + k;
+    v = qeff_f32 ? qeff_f32[r] : __bfloat162float(w_q[r]);
+  } else {
+    const size_t r = (size_t)(h * kRope + j - d_nope) * hidden + k;
+    v = qreff_f32 ? qreff_f32[r] : __bfloat162float(w_qr[r]);
+  }
+  wqd[(size_t)row * hidden + k] = __float2bfloat16_rn(v);
+}
+__global__ void bf16_to_f16_kernel(const __nv_bfloat16* __restrict__ in, __half* __restrict__ out,
+                                   int64_t n) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) out[i] = __float2half_rn(__bfloat162float(in[i]));
+}
+// k_rope of every key into the RoPE channels [d_nope, 128) of every head of the dense K:
+// kd[z][n][h][d_nope + r] = krope[z][n][r].
+__global__ void krope_broadcast_kernel(const __half* __restrict__ krope, int64_t krope_stream_rows,
+                                       __nv_bfloat16* __restrict__ kd, int n_keys, int n_heads,
+                                       int d_nope) {
+  const int n = blockIdx.x;
+  const int z = blockIdx.y;
+  const __half* src = krope + ((int64_t)z * krope_stream_rows + n) * kRope;
+  __nv_bfloat16* dst = kd + ((int64_t)z * n_keys + n) * n_heads * 128 + d_nope;
+  for (int i = threadIdx.x; i < n_heads * kRope; i += blockDim.x) {
+    const int h = i / kRope, r = i % kRope;
+    dst[h * 128 + r] = __float2bfloat16_rn(__half2float(src[r]));
+  }
+}
+
 mla_status check_launch(const char* what) {
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return fail(MLA_ERR_CUDA, "%s launch failed: %s", what, cudaGetErrorString(e));
@@ -292,6 +332,20 @@ struct mla_cache {
   __nv_bfloat16* wqcat = nullptr;  // bf16: multiplies the caller's bf16 hidden states
   __half* wov = nullptr;           // fp16: multiplies o_lat
   float2* rope_hw = nullptr;       // RoPE (cos, sin) of the h and w bands, [16][frame_h + frame_w]
+
+  // Reconstruct-then-dense form (mla_window_attention_reconstruct), when d_nope + d_rope == 128,
+  // d_head == 128 and there is no sink: per-head weights, built at creation, and per-call
+  // buffers allocated on first use.
+  bool dense_ok = false;
+  __nv_bfloat16* wqd = nullptr;    // [n_h*128][hidden]: per head [W_Q (d_nope) | W_QR (32)]
+  __half* wukh = nullptr;          // [n_h*d_nope][192] W_UK (fp16: multiplies the fp16 cache)
+  __half* wuvh = nullptr;          // [n_h*128][192] W_UV
+  __nv_bfloat16* wo = nullptr;     // [hidden][n_h*128] W_O
+  CUtensorMap map_wqd{}, map_wukh{}, map_wuvh{}, map_wo{};
+  __nv_bfloat16* qd = nullptr;     // [B][n_q][n_h][128]   per call, compact
+  __nv_bfloat16* kd = nullptr;     // [B][n_keys][n_h][128] per call, compact
+  __nv_bfloat16* vd = nullptr;     // [B][n_keys][n_h][128]
+  __nv_bfloat16* od = nullptr;     // [B][n_q][n_h][128]
   int* status = nullptr;
 
   CUtensorMap map_wqcat{};         // B operand of the projections: box 64 x 224
@@ -611,6 +665,33 @@ mla_status dense_status_word(int** out) {
   return MLA_OK;
 }
 
+// Dense per-head attention over compact q [B][n_q][H][128], k, v [B][n_kv][H][128] (bf16).
+mla_status launch_dense(const void* q, const void* k, const void* v, void* out, int batch,
+                        int n_q, int n_kv, int n_heads, float scale, int* status, cudaStream_t st) {
+  const uint64_t row = (uint64_t)n_heads * 128;
+  CUtensorMap mq, mk, mv;
+  mla_status s;
+  if ((s = make_map(&mq, q, row, n_q, batch, row * 2, row * n_q * 2, 64, 128,
+                    CU_TENSOR_MAP_SWIZZLE_128B)) != MLA_OK)
+    return s;
+  if ((s = make_map(&mk, k, row, n_kv, batch, row * 2, row * n_kv * 2, 64, 128,
+                    CU_TENSOR_MAP_SWIZZLE_128B)) != MLA_OK)
+    return s;
+  if ((s = make_map(&mv, v, row, n_kv, batch, row * 2, row * n_kv * 2, 64, 128,
+                    CU_TENSOR_MAP_SWIZZLE_128B)) != MLA_OK)
+    return s;
+  mla::DenseArgs a{};
+  a.n_q = n_q;
+  a.n_kv = n_kv;
+  a.n_heads = n_heads;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.out = static_cast<__nv_bfloat16*>(out);
+  dim3 grid((unsigned)((n_q + 127) / 128), (unsigned)n_heads, (unsigned)batch);
+  mla::dense_attn_kernel<kDenseStages>
+      <<<grid, mla::kDenseThreads, mla::DenseSmem<kDenseStages>::kBytes, st>>>(mq, mk, mv, a, status);
+  return check_launch("dense attention");
+}
+
 }  // namespace
 
 extern "C" {
@@ -703,6 +784,9 @@ size_t mla_cache_device_bytes(const mla_config* cfg) {
   b += (size_t)c.hidden * c.n_heads * kLatent * 2;         // W_OV
   b += 256;                                                // status word
   b += (size_t)(c.frame_h + c.frame_w) * 16 * 8;           // RoPE h / w tables
+  if (c.d_nope + c.d_rope == 128 && c.d_head == 128 && c.d_nope % 32 == 0 && c.sink_frames == 0)
+    b += (size_t)c.n_heads * 128 * (2 * (size_t)c.hidden + 2 * kLatent) +
+         (size_t)c.n_heads * c.d_nope * kLatent * 2;      // dense-form weights (W_Qd, W_O, W_UV, W_UK)
   return b;
 }
 
@@ -721,6 +805,14 @@ void mla_cache_destroy(mla_cache* c) {
   cudaFree(c->wqcat);
   cudaFree(c->wov);
   cudaFree(c->rope_hw);
+  cudaFree(c->wqd);
+  cudaFree(c->wukh);
+  cudaFree(c->wuvh);
+  cudaFree(c->wo);
+  cudaFree(c->qd);
+  cudaFree(c->kd);
+  cudaFree(c->vd);
+  cudaFree(c->od);
   cudaFree(c->status);
   delete c;
 }
@@ -829,6 +921,48 @@ mla_status mla_cache_create(const mla_config* cfg, const mla_weights* w, void* s
                                          k.n_heads, k.d_head);
     MLA_TRY(cudaGetLastError());
   }
+  // Weights of the reconstruct-then-dense form (training-time layout, [VideoMLA] §3.3).
+  c->dense_ok = k.d_nope + k.d_rope == 128 && k.d_head == 128 && k.d_nope % 32 == 0 &&
+                k.sink_frames == 0;
+  DevTmp qeff_f32;
+  if (c->dense_ok) {
+    const int nh = k.n_heads, dn = k.d_nope;
+    MLA_TRY(cudaMalloc(&c->wqd, (size_t)nh * 128 * k.hidden * 2));
+    MLA_TRY(cudaMalloc(&c->wukh, (size_t)nh * dn * kLatent * 2));
+    MLA_TRY(cudaMalloc(&c->wuvh, (size_t)nh * 128 * kLatent * 2));
+    MLA_TRY(cudaMalloc(&c->wo, (size_t)k.hidden * nh * 128 * 2));
+    if (k.d_q > 0) {
+      // W_Q W_DQ in fp32 (W_QR W_DQ is qr_f32 above).
+      MLA_TRY(cudaMalloc(&qeff_f32.p, (size_t)nh * dn * k.hidden * 4));
+      compose_kernel<__nv_bfloat16, __nv_bfloat16><<<dim3((k.hidden + 255) / 256, nh * dn, 1), 256, 0, st>>>(
+          (const __nv_bfloat16*)w->w_q, 0, k.d_q, 1, (const __nv_bfloat16*)w->w_dq, 0, k.hidden,
+          qeff_f32.p, 0, nh * dn, k.hidden, k.d_q);
+      MLA_TRY(cudaGetLastError());
+    }
+    build_wqd_kernel<<<dim3((k.hidden + 255) / 256, nh * 128), 256, 0, st>>>(
+        (const __nv_bfloat16*)w->w_q, (const __nv_bfloat16*)w->w_qr, qeff_f32.p, qr_f32.p, c->wqd,
+        k.hidden, nh, dn);
+    MLA_TRY(cudaGetLastError());
+    const int64_t n_uk = (int64_t)nh * dn * kLatent, n_uv = (int64_t)nh * 128 * kLatent;
+    bf16_to_f16_kernel<<<(unsigned)((n_uk + 255) / 256), 256, 0, st>>>(
+        (const __nv_bfloat16*)w->w_uk, c->wukh, n_uk);
+    bf16_to_f16_kernel<<<(unsigned)((n_uv + 255) / 256), 256, 0, st>>>(
+        (const __nv_bfloat16*)w->w_uv, c->wuvh, n_uv);
+    MLA_TRY(cudaGetLastError());
+    MLA_TRY(cudaMemcpyAsync(c->wo, w->w_o, (size_t)k.hidden * nh * 128 * 2,
+                            cudaMemcpyDeviceToDevice, st));
+    const uint64_t qd_cols = (uint64_t)nh * 128;
+    if ((s = make_map(&c->map_wqd, c->wqd, k.hidden, qd_cols, 1, (uint64_t)k.hidden * 2,
+                      qd_cols * k.hidden * 2, 64, kOutBN, CU_TENSOR_MAP_SWIZZLE_128B)) != MLA_OK ||
+        (s = make_map(&c->map_wukh, c->wukh, kLatent, (uint64_t)nh * dn, 1, kLatent * 2,
+                      (uint64_t)nh * dn * kLatent * 2, 64, kOutBN, CU_TENSOR_MAP_SWIZZLE_128B,
+                      true)) != MLA_OK ||
+        (s = make_map(&c->map_wuvh, c->wuvh, kLatent, qd_cols, 1, kLatent * 2,
+                      qd_cols * kLatent * 2, 64, kOutBN, CU_TENSOR_MAP_SWIZZLE_128B, true)) != MLA_OK ||
+        (s = make_map(&c->map_wo, c->wo, qd_cols, k.hidden, 1, qd_cols * 2,
+                      qd_cols * k.hidden * 2, 64, kOutBN, CU_TENSOR_MAP_SWIZZLE_128B)) != MLA_OK)
+      return cleanup(s);
+  }
   s = make_map(&c->map_wqcat, c->wqcat, k.hidden, (uint64_t)(k.n_heads + 1) * kQK, 1,
                (uint64_t)k.hidden * 2, (uint64_t)(k.n_heads + 1) * kQK * k.hidden * 2, 64, kQK,
                CU_TENSOR_MAP_SWIZZLE_128B);
@@ -863,6 +997,17 @@ mla_status mla_cache_create(const mla_config* cfg, const mla_weights* w, void* s
     if (r == MLA_OK)
       r = set_smem(mla::tc_gemm_kernel<kOutBN, kOutAStages, kOutBStages, mla::kEpiStore, true, 1>,
                    mla::GemmSmem<kOutBN, kOutAStages, kOutBStages>::kBytes);
+    if (r == MLA_OK)
+      r = set_smem(mla::tc_gemm_kernel<kOutBN, kOutAStages, kOutBStages, mla::kEpiDense, false, 1>,
+                   mla::GemmSmem<kOutBN, kOutAStages, kOutBStages>::kBytes);
+    if (r == MLA_OK)
+      r = set_smem(mla::tc_gemm_kernel<kOutBN, kOutAStages, kOutBStages, mla::kEpiDense, true, 1>,
+                   mla::GemmSmem<kOutBN, kOutAStages, kOutBStages>::kBytes);
+    if (r == MLA_OK)
+      r = set_smem(mla::tc_gemm_kernel<kOutBN, kOutAStages, kOutBStages, mla::kEpiStore, false, 1>,
+                   mla::GemmSmem<kOutBN, kOutAStages, kOutBStages>::kBytes);
+    if (r == MLA_OK)
+      r = set_smem(mla::dense_attn_kernel<kDenseStages>, mla::DenseSmem<kDenseStages>::kBytes);
     if (r == MLA_OK)
       r = set_smem(mla::window_attn_kernel<kAttnStages>,
                    mla::AttnSmem<kAttnStages>::kBytes);
@@ -1010,6 +1155,114 @@ mla_status mla_window_attention_noalloc(mla_cache* c, const void* x_chunk, int32
   return launch_out_proj(c, o_lat, nq, nq, out, st, "no-alloc output projection");
 }
 
+mla_status mla_window_attention_reconstruct(mla_cache* c, const void* x_chunk, int32_t n_frames,
+                                            void* out, void* stream) {
+  if (!c || !x_chunk || !out) return fail(MLA_ERR_INVALID_ARGUMENT, "NULL argument");
+  const mla_config& cfg = c->cfg;
+  if (!c->dense_ok)
+    return fail(MLA_ERR_UNSUPPORTED,
+                "the dense form needs d_nope + d_rope == 128, d_head == 128, d_nope a multiple "
+                "of 32 and no sink frames");
+  if (n_frames < 1 || n_frames > cfg.max_chunk_frames)
+    return fail(MLA_ERR_INVALID_ARGUMENT, "n_frames must be in [1, max_chunk_frames=%d]",
+                cfg.max_chunk_frames);
+  if (!aligned16(x_chunk) || !aligned16(out))
+    return fail(MLA_ERR_INVALID_ARGUMENT, "x_chunk and out must be 16-byte aligned");
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int nh = cfg.n_heads, dn = cfg.d_nope;
+  const uint64_t hd = (uint64_t)nh * 128;                 // dense row: n_h heads x 128
+  if (!c->qd) {
+    // Per-call dense buffers, allocated once: the per-head K and V of the largest window are the
+    // dense cache the latent layout avoids (B x rows x n_h x 128 x 2 bytes each).
+    MLA_CUDA(cudaMalloc(&c->qd, (size_t)cfg.batch * c->max_q_tokens * hd * 2));
+    MLA_CUDA(cudaMalloc(&c->od, (size_t)cfg.batch * c->max_q_tokens * hd * 2));
+    MLA_CUDA(cudaMalloc(&c->kd, (size_t)cfg.batch * c->rows_per_stream * hd * 2));
+    MLA_CUDA(cudaMalloc(&c->vd, (size_t)cfg.batch * c->rows_per_stream * hd * 2));
+  }
+  const int64_t nq = (int64_t)n_frames * c->F;
+  int64_t vs, vw;
+  valid_counts(c, vs, vw);
+  const int64_t base_row = c->sink_rows + vw * c->F;
+  const int64_t n_keys = base_row + nq;
+  mla_status s;
+
+  // 1. the chunk's latents into the chunk tail (as the absorbed path does)
+  if ((s = launch_latent_gemm(c, x_chunk, nq, nq, false, c->frames_appended, base_row, st)) != MLA_OK)
+    return s;
+  // 2. per-head queries [q_nope | RoPE3D(q_rope)] at the chunk's absolute positions
+  {
+    CUtensorMap ma, mo;
+    if ((s = make_map(&ma, x_chunk, cfg.hidden, nq, cfg.batch, (uint64_t)cfg.hidden * 2,
+                      (uint64_t)nq * cfg.hidden * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B)) != MLA_OK ||
+        (s = make_out_map(&mo, c->qd, hd, nq, cfg.batch, hd * 2, hd * nq * 2, false)) != MLA_OK)
+      return s;
+    EpiArgs ep{};
+    ep.n_cols = (int)hd;
+    ep.rope_period = 128;
+    ep.t0 = c->frames_appended;
+    ep.tokens_per_frame = c->F;
+    ep.frame_w = cfg.frame_w;
+    ep.rope = c->rope;
+    ep.rope_hw = c->rope_hw;
+    ep.frame_h = cfg.frame_h;
+    const mla::GemmTiles tiles{(int32_t)((nq + 127) / 128), (int32_t)((hd + kOutBN - 1) / kOutBN), cfg.batch};
+    if ((s = launch_gemm<kOutBN, kOutAStages, kOutBStages, mla::kEpiDense, false>(
+             ma, c->map_wqd, mo, mo, mo, (int)nq, cfg.hidden, 0, tiles, ep, c->status, c->num_sms,
+             st, "dense query projection")) != MLA_OK)
+      return s;
+  }
+  // 3. per-head keys and values of every key from the latent: K_h = [c W_UK[h]^T | k_rope],
+  //    V_h = c W_UV[h]^T ([VideoMLA] §3.3)
+  {
+    CUtensorMap ma, mk, mv;
+    if ((s = make_map(&ma, c->ckv, kLatent, n_keys, cfg.batch, kLatent * 2,
+                      (uint64_t)c->rows_per_stream * kLatent * 2, 64, 128,
+                      CU_TENSOR_MAP_SWIZZLE_128B, true)) != MLA_OK ||
+        (s = make_out_map(&mk, c->kd, hd, n_keys, cfg.batch, hd * 2, hd * n_keys * 2, false)) != MLA_OK ||
+        (s = make_out_map(&mv, c->vd, hd, n_keys, cfg.batch, hd * 2, hd * n_keys * 2, false)) != MLA_OK)
+      return s;
+    const int32_t m_tiles = (int32_t)((n_keys + 127) / 128);
+    EpiArgs ek{};
+    ek.n_cols = nh * dn;
+    ek.head_in = dn;
+    ek.head_out = 128;
+    if ((s = launch_gemm<kOutBN, kOutAStages, kOutBStages, mla::kEpiDense, true>(
+             ma, c->map_wukh, mk, mk, mk, (int)n_keys, kLatent, 0,
+             mla::GemmTiles{m_tiles, (nh * dn + kOutBN - 1) / kOutBN, cfg.batch}, ek, c->status,
+             c->num_sms, st, "key reconstruction")) != MLA_OK)
+      return s;
+    krope_broadcast_kernel<<<dim3((unsigned)n_keys, (unsigned)cfg.batch), 128, 0, st>>>(
+        c->krope, c->rows_per_stream, c->kd, (int)n_keys, nh, dn);
+    if ((s = check_launch("k_rope broadcast")) != MLA_OK) return s;
+    EpiArgs ev{};
+    ev.n_cols = (int)hd;
+    if ((s = launch_gemm<kOutBN, kOutAStages, kOutBStages, mla::kEpiDense, true>(
+             ma, c->map_wuvh, mv, mv, mv, (int)n_keys, kLatent, 0,
+             mla::GemmTiles{m_tiles, (int32_t)((hd + kOutBN - 1) / kOutBN), cfg.batch}, ev,
+             c->status, c->num_sms, st, "value reconstruction")) != MLA_OK)
+      return s;
+  }
+  // 4. dense per-head attention
+  if ((s = launch_dense(c->qd, c->kd, c->vd, c->od, cfg.batch, (int)nq, (int)n_keys, nh,
+                        c->softmax_scale, c->status, st)) != MLA_OK)
+    return s;
+  // 5. out = concat_h(o_h) W_O^T
+  {
+    CUtensorMap ma, mo;
+    if ((s = make_map(&ma, c->od, hd, nq, cfg.batch, hd * 2, hd * nq * 2, 64, 128,
+                      CU_TENSOR_MAP_SWIZZLE_128B)) != MLA_OK ||
+        (s = make_out_map(&mo, out, cfg.hidden, nq, cfg.batch, (uint64_t)cfg.hidden * 2,
+                          (uint64_t)nq * cfg.hidden * 2, false)) != MLA_OK)
+      return s;
+    EpiArgs ep{};
+    ep.n_cols = cfg.hidden;
+    const mla::GemmTiles tiles{(int32_t)((nq + 127) / 128), (cfg.hidden + kOutBN - 1) / kOutBN, cfg.batch};
+    return launch_gemm<kOutBN, kOutAStages, kOutBStages, mla::kEpiStore, false>(
+        ma, c->map_wo, mo, mo, mo, (int)nq, (int)hd, 0, tiles, ep, c->status, c->num_sms, st,
+        "dense output projection");
+  }
+}
+
 mla_status mla_dense_attention(const void* q, const void* k, const void* v, void* out,
                                int32_t batch, int32_t n_q, int32_t n_kv, int32_t n_heads,
                                int32_t d_head, float softmax_scale, void* stream) {
@@ -1026,29 +1279,9 @@ mla_status mla_dense_attention(const void* q, const void* k, const void* v, void
   int* status = nullptr;
   mla_status s = dense_status_word(&status);
   if (s != MLA_OK) return s;
-  const uint64_t row = (uint64_t)n_heads * 128;
-  CUtensorMap mq, mk, mv;
-  if ((s = make_map(&mq, q, row, n_q, batch, row * 2, row * n_q * 2, 64, 128,
-                    CU_TENSOR_MAP_SWIZZLE_128B)) != MLA_OK)
-    return s;
-  if ((s = make_map(&mk, k, row, n_kv, batch, row * 2, row * n_kv * 2, 64, 128,
-                    CU_TENSOR_MAP_SWIZZLE_128B)) != MLA_OK)
-    return s;
-  if ((s = make_map(&mv, v, row, n_kv, batch, row * 2, row * n_kv * 2, 64, 128,
-                    CU_TENSOR_MAP_SWIZZLE_128B)) != MLA_OK)
-    return s;
-  mla::DenseArgs a{};
-  a.n_q = n_q;
-  a.n_kv = n_kv;
-  a.n_heads = n_heads;
   const float scale = softmax_scale > 0.f ? softmax_scale : (float)(1.0 / std::sqrt(128.0));
-  a.scale_log2 = scale * 1.4426950408889634f;
-  a.out = static_cast<__nv_bfloat16*>(out);
-  dim3 grid((unsigned)((n_q + 127) / 128), (unsigned)n_heads, (unsigned)batch);
-  mla::dense_attn_kernel<kDenseStages>
-      <<<grid, mla::kDenseThreads, mla::DenseSmem<kDenseStages>::kBytes,
-         reinterpret_cast<cudaStream_t>(stream)>>>(mq, mk, mv, a, status);
-  return check_launch("dense attention");
+  return launch_dense(q, k, v, out, batch, n_q, n_kv, n_heads, scale, status,
+                      reinterpret_cast<cudaStream_t>(stream));
 }
 
 mla_status mla_dense_sync(void* stream) {

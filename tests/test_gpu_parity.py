@@ -303,3 +303,58 @@ def test_sink_w6_q3_full_size():
         assert_close(kr[s0:s0 + w.F], r, f"k_rope frame {f}")
     sampled_check(p, p.hidden(3, mla_synth.chunk_seed(w, 0, 0)), "sink + 6-frame window", 64, 6)
 
+
+
+# ---------------------------------------------------------------------------- reconstruct-then-dense
+def reconstruct_check(pair: Pair, x_chunk, what: str, rows=None):
+    out = pair.gpu.attention_reconstruct(x_chunk.cuda())
+    torch.cuda.synchronize()
+    out = out.cpu()
+    for b, orc in enumerate(pair.oracles):
+        if rows is None:
+            assert_close(out[b], orc.attention(x_chunk[b]), f"{what}: out (stream {b})")
+        else:
+            assert_close(out[b][rows], orc.attention(x_chunk[b], rows=rows), f"{what}: out rows (stream {b})")
+    pair.check_status()
+    return out
+
+
+def test_reconstruct_dense_paper_tiny():
+    # The training-time form ([VideoMLA] §3.3): per-head K/V materialised from the latent, dense
+    # attention, W_O.  Every element against the oracle, and against the absorbed path.
+    w = mla_synth.WORKLOADS["paper_tiny"]
+    p = Pair(w)
+    p.append(p.hidden(w.fill_frames, mla_synth.fill_seed(w, 0)))
+    x = p.hidden(w.query_frames, mla_synth.chunk_seed(w, 0, 0))
+    dense = reconstruct_check(p, x, "reconstruct (paper tiny)")
+    absorbed = p.attention(x)
+    assert_close(dense, absorbed.float().numpy(), "reconstruct vs absorbed")
+
+
+def test_reconstruct_dense_ragged_batched():
+    # F = 200 tokens: 600 + 400 keys (ragged 128-key tiles), 400 query rows, 2 streams.
+    w = mla_synth.Workload("paper_ragged", frame_h=10, frame_w=20, window_frames=3, fill_frames=4,
+                           query_frames=2, batch=2, seed=29,
+                           dims=tuple(sorted(mla_synth.DIMS_PAPER.items())))
+    p = Pair(w, max_chunk_frames=2)
+    p.append(p.hidden(4, 730))
+    reconstruct_check(p, p.hidden(2, 731), "reconstruct (ragged, batched)")
+
+
+def test_reconstruct_dense_paper_w21_full_size():
+    w = mla_synth.WORKLOADS["paper_w21_q1"]
+    p = Pair(w)
+    p.append(p.hidden(w.fill_frames, mla_synth.fill_seed(w, 0)))
+    rows = np.sort(np.random.default_rng(7).choice(w.F, size=48, replace=False))
+    reconstruct_check(p, p.hidden(1, mla_synth.chunk_seed(w, 0, 0)), "reconstruct (21-frame window)", rows)
+
+
+def test_reconstruct_dense_unsupported_configs():
+    from mla_latent_kv_window_b200 import MLAError
+    for w in (small(window=2, q=1, seed=30),                       # d_nope + d_rope = 160
+              mla_synth.WORKLOADS["sink_tiny"]):                    # sink frames
+        p = Pair(w, max_chunk_frames=1)
+        p.append(p.hidden(2, 740))
+        with pytest.raises(MLAError, match="UNSUPPORTED"):
+            p.gpu.attention_reconstruct(p.hidden(1, 741).cuda())
+        p.check_status()
