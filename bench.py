@@ -517,7 +517,50 @@ def next_rows(B, dev):
         }
     res["note"] = ("attention TFLOP/s at 832 flop per (query, head, key) over the valid keys (sink "
                    "padding rows excluded); call = query projection + attention + output projection")
+    res["reconstruct_vs_absorbed"] = reconstruct_crossover(B, dev)
     return res
+
+
+def reconstruct_crossover(B, dev):
+    """Absorbed kernel vs reconstruct-then-dense on the paper-default dims over the 21-frame
+    window, for 1-, 2- and 3-frame chunks (whole calls, CUDA events).  The dense form pays a
+    per-call reconstruction of every key and then 512 flop per (query, head, key) instead of 832;
+    a straight-line fit of both call times in the query count gives where they cross."""
+    import numpy as np
+    import torch
+
+    import mla_synth
+    w = mla_synth.WORKLOADS["paper_w21_q1"]
+    dims = dict(w.dims)
+    F = w.F
+    wts = {k: v.to(dev) for k, v in mla_synth.make_weights(dims, mla_synth.weight_seed(w, 0)).items()}
+    c = B.LatentWindowCache(dims, wts, w.frame_h, w.frame_w, w.window_frames, 3)
+    c.append(mla_synth.make_hidden(1, w.fill_frames * F, dims["hidden"], mla_synth.fill_seed(w, 0)).to(dev))
+    stream = torch.cuda.current_stream()
+    rows = []
+    for nf in (1, 2, 3):
+        x = mla_synth.make_hidden(1, nf * F, dims["hidden"], mla_synth.chunk_seed(w, 0, nf)).to(dev)
+        out = torch.empty_like(x)
+        t_abs = _event_ms(lambda: c.attention(x, out), stream)
+        t_rec = _event_ms(lambda: c.attention_reconstruct(x, out), stream)
+        rows.append({"query_tokens": nf * F, "keys": w.window_frames * F + nf * F,
+                     "absorbed_ms": round(t_abs, 4), "reconstruct_dense_ms": round(t_rec, 4)})
+    ok = B.mla_cache_sync(c.handle) == 0
+    c.close()
+    n = np.array([r["query_tokens"] for r in rows], dtype=np.float64)
+    ta = np.array([r["absorbed_ms"] for r in rows])
+    tr = np.array([r["reconstruct_dense_ms"] for r in rows])
+    (ba, aa), (br, ar) = np.polyfit(n, ta, 1), np.polyfit(n, tr, 1)
+    cross = (ar - aa) / (ba - br) if ba != br else None
+    return {"workload": "paper dims (96 + 32 per head, d_q = 768, RoPE (6,5,5)), 21-frame window",
+            "calls": rows, "status_ok": ok,
+            "fit_ms": {"absorbed": [round(aa, 4), round(ba * 1e3, 5)],
+                       "reconstruct_dense": [round(ar, 4), round(br * 1e3, 5)],
+                       "form": "[intercept ms, ms per 1000 query tokens]"},
+            "crossover_query_tokens": (round(float(cross), 1) if cross is not None else None),
+            "note": "reconstruct-then-dense is faster above the crossover when the crossover is "
+                    "positive and its slope is smaller; the window's keys are reconstructed "
+                    "every call"}
 
 
 # ---------------------------------------------------------------------------- the oracle on CPU
