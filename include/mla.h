@@ -200,6 +200,16 @@ mla_status mla_dense_attention(const void* q, const void* k, const void* v, void
  * MLA_ERR_DEVICE_TIMEOUT). */
 mla_status mla_dense_sync(void* stream);
 
+/* Diagnostic self-test of the library's bounded device waits: launches one thread that waits on
+ * a barrier phase nothing will complete, using the same wait as every kernel of the library.
+ * The wait gives up after its limit (2 s), records MLA_ERR_DEVICE_TIMEOUT in the cache's status
+ * word and the kernel returns, so the GPU context stays usable.  Synchronises `stream`;
+ * *gave_up receives 1 when the wait ran out.  Afterwards mla_cache_sync reports the timeout,
+ * and the status word stays set (kernels launched later on this cache stop waiting at once):
+ * use a fresh cache for further work.  Not part of the method; exists to test failure
+ * reporting without faulting a GPU. */
+mla_status mla_cache_selftest_timeout(mla_cache* c, void* stream, int32_t* gave_up);
+
 /* Free everything the cache owns (synchronises the device first).  NULL-safe. */
 void mla_cache_destroy(mla_cache* c);
 

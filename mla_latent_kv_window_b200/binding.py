@@ -27,7 +27,7 @@ KERNEL_NAMES = ("append", "qproj", "attention", "oproj")
 EXPORTED = (
     "mla_config_check", "mla_ring_slot", "mla_ring_bytes", "mla_cache_device_bytes",
     "mla_cache_create", "mla_cache_append", "mla_window_attention", "mla_window_attention_noalloc",
-    "mla_window_attention_reconstruct",
+    "mla_window_attention_reconstruct", "mla_cache_selftest_timeout",
     "mla_cache_destroy", "mla_dense_attention", "mla_dense_sync",
     "mla_cache_state", "mla_cache_sync", "mla_cache_read", "mla_cache_debug_buffers", "mla_cache_copy_buffer",
     "mla_cache_profile_enable", "mla_cache_profile_read", "mla_status_string", "mla_last_error",
@@ -88,6 +88,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "mla_window_attention": (I32, [VP, VP, I32, VP, VP]),
         "mla_window_attention_noalloc": (I32, [VP, VP, I32, VP, VP]),
         "mla_window_attention_reconstruct": (I32, [VP, VP, I32, VP, VP]),
+        "mla_cache_selftest_timeout": (I32, [VP, VP, P(I32)]),
         "mla_dense_attention": (I32, [VP, VP, VP, VP, I32, I32, I32, I32, I32, ctypes.c_float, VP]),
         "mla_dense_sync": (I32, [VP]),
         "mla_cache_destroy": (None, [VP]),
@@ -197,6 +198,14 @@ def mla_window_attention_reconstruct(cache: int, x_chunk, n_frames: int, out, st
     _check(load_library().mla_window_attention_reconstruct(cache, _dev_ptr(x_chunk, "x_chunk"), n_frames,
                                                            _dev_ptr(out, "out"), _stream_handle(stream)),
            "mla_window_attention_reconstruct")
+
+
+def mla_cache_selftest_timeout(cache: int, stream=None) -> bool:
+    """Run the bounded-wait self-test (about 2 s); True when the device wait gave up."""
+    flag = ctypes.c_int32()
+    _check(load_library().mla_cache_selftest_timeout(cache, _stream_handle(stream), ctypes.byref(flag)),
+           "mla_cache_selftest_timeout")
+    return flag.value == 1
 
 
 def mla_dense_attention(q, k, v, out, softmax_scale: float = 0.0, stream=None) -> None:

@@ -57,7 +57,8 @@ __global__ void __launch_bounds__(kDenseThreads, 1)
   uint64_t* s_free = s_full + 2;
   uint64_t* p_full = s_free + 2;
   uint64_t* pv_done = p_full + 1;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(pv_done + 1);
+  uint64_t* quiesce = pv_done + 1;               // all MMAs of this CTA have completed
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(quiesce + 1);
 
   const uint32_t warp = warp_id();
   const uint32_t lane = lane_id();
@@ -80,6 +81,7 @@ __global__ void __launch_bounds__(kDenseThreads, 1)
     }
     mbar_init(p_full, 128);
     mbar_init(pv_done, 1);
+    mbar_init(quiesce, 1);
     fence_mbar_init();
     tma_prefetch(&map_q);
     tma_prefetch(&map_k);
@@ -117,9 +119,10 @@ __global__ void __launch_bounds__(kDenseThreads, 1)
         }
         issued = j + 1;
       }
+      // Drain: no copy may still land in shared memory when the CTA exits (also after an error).
       for (int j = issued > KV_STAGES ? issued - KV_STAGES : 0; j < issued; ++j)
-        mbar_wait(&kv_full[j % KV_STAGES], (uint32_t)(j / KV_STAGES) & 1u, status);
-      mbar_wait(q_full, 0, status);
+        mbar_wait_quiesce(&kv_full[j % KV_STAGES], (uint32_t)(j / KV_STAGES) & 1u, status);
+      mbar_wait_quiesce(q_full, 0, status);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -158,6 +161,9 @@ __global__ void __launch_bounds__(kDenseThreads, 1)
           tc_commit(&kv_empty[st]);
         }
       }
+      // The CTA frees shared and tensor memory only after every issued MMA has completed.
+      tc_commit(quiesce);
+      mbar_wait_quiesce(quiesce, 0, status);
     }
   } else {
     const uint32_t sub = warp & 3u;

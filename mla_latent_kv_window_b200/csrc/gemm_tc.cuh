@@ -175,7 +175,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint64_t* b_empty = b_full + B_STAGES;
   uint64_t* acc_full = b_empty + B_STAGES;     // [2]
   uint64_t* acc_empty = acc_full + 2;          // [2]
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(acc_empty + 2);
+  uint64_t* mma_quiesce = acc_empty + 2;       // all of this CTA's MMAs have completed
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(mma_quiesce + 1);
 
   const uint32_t warp = warp_id();
   const uint32_t lane = lane_id();
@@ -198,6 +199,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       mbar_init(&acc_full[s], 1);
       mbar_init(&acc_empty[s], kEpiWarps * 32);
     }
+    mbar_init(mma_quiesce, 1);
     fence_mbar_init();
     tma_prefetch(&map_a);
     tma_prefetch(&map_b);
@@ -254,9 +256,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                              b_row0 + y * BN, 0, policy);
         }
       }
-      // Drain: never leave the CTA with a copy still landing in its shared memory.
+      // Drain: never leave the CTA with a copy still landing in its shared memory (also when
+      // the loop above stopped on an error).
       for (int q = g > stages ? g - stages : 0; q < g; ++q)
-        mbar_wait(&full[q % stages], (uint32_t)(q / stages) & 1u, status);
+        mbar_wait_quiesce(&full[q % stages], (uint32_t)(q / stages) & 1u, status);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
@@ -294,6 +297,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         tc_commit(&acc_full[buf]);
       }
+      // Every MMA issued above has finished reading shared memory and writing TMEM before the
+      // CTA may free either (also when the loop stopped on an error).
+      tc_commit(mma_quiesce);
+      mbar_wait_quiesce(mma_quiesce, 0, status);
     }
   } else {
     // ------------------------------------------------------------------ epilogue warps

@@ -287,6 +287,18 @@ __global__ void krope_broadcast_kernel(const __half* __restrict__ krope, int64_t
   }
 }
 
+// Self-test of the bounded device wait: one thread waits on an mbarrier phase that nothing
+// completes; mbar_wait gives up after its limit and records MLA_ERR_DEVICE_TIMEOUT.
+__global__ void selftest_wait_kernel(int* status, int* gave_up) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    mla::mbar_init(&bar, 1);
+    mla::fence_mbar_init();
+    const bool ok = mla::mbar_wait(&bar, 0, status);
+    *gave_up = ok ? 0 : 1;
+  }
+}
+
 mla_status check_launch(const char* what) {
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return fail(MLA_ERR_CUDA, "%s launch failed: %s", what, cudaGetErrorString(e));
@@ -1261,6 +1273,21 @@ mla_status mla_window_attention_reconstruct(mla_cache* c, const void* x_chunk, i
         ma, c->map_wo, mo, mo, mo, (int)nq, (int)hd, 0, tiles, ep, c->status, c->num_sms, st,
         "dense output projection");
   }
+}
+
+mla_status mla_cache_selftest_timeout(mla_cache* c, void* stream, int32_t* gave_up) {
+  if (!c || !gave_up) return fail(MLA_ERR_INVALID_ARGUMENT, "NULL argument");
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  int* flag = c->status + 1;   // second word of the 256-byte status block
+  MLA_CUDA(cudaMemsetAsync(flag, 0, sizeof(int), st));
+  selftest_wait_kernel<<<1, 32, 0, st>>>(c->status, flag);
+  mla_status s = check_launch("self-test wait");
+  if (s != MLA_OK) return s;
+  MLA_CUDA(cudaStreamSynchronize(st));
+  int h = 0;
+  MLA_CUDA(cudaMemcpy(&h, flag, sizeof(int), cudaMemcpyDeviceToHost));
+  *gave_up = h;
+  return MLA_OK;
 }
 
 mla_status mla_dense_attention(const void* q, const void* k, const void* v, void* out,

@@ -76,6 +76,21 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* s
   }
 }
 
+// Wait for a phase that is certain to complete (copies or MMAs this CTA has already issued),
+// even after another CTA has recorded an error: a CTA must not exit, nor free its tensor memory,
+// while its own asynchronous work may still land.  Bounded like mbar_wait.
+__device__ __forceinline__ bool mbar_wait_quiesce(uint64_t* bar, uint32_t parity, int* status) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t n = 1;; ++n) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((n & 127u) == 0u && global_timer_ns() - t0 > kWaitLimitNs) {
+      atomicCAS(status, 0, kStatusTimeout);
+      return false;
+    }
+  }
+}
+
 // Whole-warp wait for a phase that may take many microseconds (e.g. an epilogue waiting for a
 // tile's MMAs): only lane 0 polls, with a growing __nanosleep back-off, so that 32 threads do
 // not hammer the barrier's shared-memory word (and the status word's L2 line) while the

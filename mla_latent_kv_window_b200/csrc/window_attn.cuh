@@ -97,7 +97,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   uint64_t* s_free = s_full + 1;
   uint64_t* p_full = s_free + 1;
   uint64_t* pv_done = p_full + 1;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(pv_done + 1);
+  uint64_t* quiesce_s = pv_done + 1;             // all S MMAs of this CTA have completed
+  uint64_t* quiesce_pv = quiesce_s + 1;          // all PV MMAs of this CTA have completed
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(quiesce_pv + 1);
 
   const uint32_t warp = warp_id();
   const uint32_t lane = lane_id();
@@ -120,6 +122,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     mbar_init(s_free, 128);
     mbar_init(p_full, 128);
     mbar_init(pv_done, 1);
+    mbar_init(quiesce_s, 1);
+    mbar_init(quiesce_pv, 1);
     fence_mbar_init();
     tma_prefetch(&map_kc);
     tma_prefetch(&map_kr);
@@ -152,9 +156,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         tma_load_3d_hint(kv + 3 * L::kAtomC, &map_kr, &kv_full[st], 0, key0, z, keep);
         issued = j + 1;
       }
-      // Drain: never leave the CTA with a copy still landing in its shared memory.
+      // Drain: never leave the CTA with a copy still landing in its shared memory (also when
+      // the loop above stopped on an error).
       for (int j = issued > KV_STAGES ? issued - KV_STAGES : 0; j < issued; ++j)
-        mbar_wait(&kv_full[j % KV_STAGES], (uint32_t)(j / KV_STAGES) & 1u, status);
+        mbar_wait_quiesce(&kv_full[j % KV_STAGES], (uint32_t)(j / KV_STAGES) & 1u, status);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ S issuer
@@ -185,6 +190,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
         tc_commit(s_full);
       }
+      // The CTA frees shared and tensor memory only after every issued MMA has completed.
+      tc_commit(quiesce_s);
+      mbar_wait_quiesce(quiesce_s, 0, status);
     }
   } else if (warp == 6) {
     // ------------------------------------------------------------------ PV issuer
@@ -209,6 +217,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         tc_commit(pv_done);
         tc_commit(&kv_empty[st]);
       }
+      tc_commit(quiesce_pv);
+      mbar_wait_quiesce(quiesce_pv, 0, status);
     }
   } else {
     // ------------------------------------------------------------------ softmax warps
