@@ -1185,11 +1185,26 @@ mla_status mla_window_attention_reconstruct(mla_cache* c, const void* x_chunk, i
   const uint64_t hd = (uint64_t)nh * 128;                 // dense row: n_h heads x 128
   if (!c->qd) {
     // Per-call dense buffers, allocated once: the per-head K and V of the largest window are the
-    // dense cache the latent layout avoids (B x rows x n_h x 128 x 2 bytes each).
-    MLA_CUDA(cudaMalloc(&c->qd, (size_t)cfg.batch * c->max_q_tokens * hd * 2));
-    MLA_CUDA(cudaMalloc(&c->od, (size_t)cfg.batch * c->max_q_tokens * hd * 2));
-    MLA_CUDA(cudaMalloc(&c->kd, (size_t)cfg.batch * c->rows_per_stream * hd * 2));
-    MLA_CUDA(cudaMalloc(&c->vd, (size_t)cfg.batch * c->rows_per_stream * hd * 2));
+    // dense cache the latent layout avoids (B x rows x n_h x 128 x 2 bytes each).  All four or
+    // none: a failed allocation leaves the cache as it was.
+    void* p[4] = {nullptr, nullptr, nullptr, nullptr};
+    const size_t bytes[4] = {(size_t)cfg.batch * c->max_q_tokens * hd * 2,
+                             (size_t)cfg.batch * c->max_q_tokens * hd * 2,
+                             (size_t)cfg.batch * c->rows_per_stream * hd * 2,
+                             (size_t)cfg.batch * c->rows_per_stream * hd * 2};
+    for (int i = 0; i < 4; ++i) {
+      const cudaError_t e = cudaMalloc(&p[i], bytes[i]);
+      if (e != cudaSuccess) {
+        for (int k = 0; k < i; ++k) cudaFree(p[k]);
+        return fail(e == cudaErrorMemoryAllocation ? MLA_ERR_OUT_OF_MEMORY : MLA_ERR_CUDA,
+                    "dense-form buffers: cudaMalloc of %zu bytes failed: %s", bytes[i],
+                    cudaGetErrorString(e));
+      }
+    }
+    c->qd = static_cast<__nv_bfloat16*>(p[0]);
+    c->od = static_cast<__nv_bfloat16*>(p[1]);
+    c->kd = static_cast<__nv_bfloat16*>(p[2]);
+    c->vd = static_cast<__nv_bfloat16*>(p[3]);
   }
   const int64_t nq = (int64_t)n_frames * c->F;
   int64_t vs, vw;
