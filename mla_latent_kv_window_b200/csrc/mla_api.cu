@@ -2,13 +2,16 @@
 // cache state, absorbed-weight derivation, tensor maps and kernel launches.
 //
 // Path of one attention call (VideoMLA paper page, §3.1-§3.3, App. D.4):
-//   1. tc_gemm<224, kEpiLatent>   x_chunk x [W_Qabs|W_QR per head ; W_DKV|W_KR]^T
+//   1. tc_gemm<kEpiLatent>   x_chunk x [W_Qabs|W_QR per head ; W_DKV|W_KR]^T (tile shape per
+//                            launch from TileShape: 256 x 160 tiles for a one-frame chunk)
 //        heads  -> Qp[(q,h)] = [W_UK[h]^T q_nope | RoPE3D(q_rope)] * scale * log2 e
 //        latent -> chunk tail rows (c_kv, RoPE3D k_rope)
-//   2. window_attn_kernel          o_lat[(q,h)] = softmax(Qp . [c_kv|k_rope]^T) c_kv
-//   3. tc_gemm<256, kEpiStore>    out = o_lat x W_OV^T,  W_OV[h] = W_O[:, h] W_UV[h]
-// An append is step 1's latent block alone, written to ring slots (t mod W) * F + k: one launch
-// per contiguous run of slots (two when the frames wrap around the end of the ring).
+//   2. window_attn_kernel     o_lat[(q,h)] = softmax(Qp . [c_kv|k_rope]^T) c_kv
+//   3. tc_gemm<192, kEpiStore>  out = o_lat x W_OV^T,  W_OV[h] = W_O[:, h] W_UV[h]
+// An append is step 1's latent block alone, written to the rows mla_ring_slot names (sink frames
+// first, then ring slots): one launch per contiguous run of rows (two when the frames wrap
+// around the end of the ring).  mla_window_attention_reconstruct is the training-time form of
+// the same call (per-head K/V materialised, dense attention), kept for comparison.
 // Every kernel of the path is launched with programmatic stream serialization, so its
 // prologue overlaps the tail of the kernel before it.
 #include <cuda.h>
@@ -797,8 +800,8 @@ size_t mla_cache_device_bytes(const mla_config* cfg) {
   b += 256;                                                // status word
   b += (size_t)(c.frame_h + c.frame_w) * 16 * 8;           // RoPE h / w tables
   if (c.d_nope + c.d_rope == 128 && c.d_head == 128 && c.d_nope % 32 == 0 && c.sink_frames == 0)
-    b += (size_t)c.n_heads * 128 * (2 * (size_t)c.hidden + 2 * kLatent) +
-         (size_t)c.n_heads * c.d_nope * kLatent * 2;      // dense-form weights (W_Qd, W_O, W_UV, W_UK)
+    b += (size_t)c.n_heads * 128 * ((size_t)c.hidden * 2 * 2 + kLatent * 2) +   // W_Qd, W_O; W_UV
+         (size_t)c.n_heads * c.d_nope * kLatent * 2;                           // W_UK
   return b;
 }
 

@@ -106,6 +106,13 @@ def test_ring_bytes_reproduce_printed_accounting():
     assert B.mla_ring_bytes(cfg(batch=4)) == 4 * per_layer
     assert B.mla_cache_device_bytes(cfg()) > per_layer
     assert B.mla_cache_device_bytes(cfg(d_latent=128)) == 0
+    # The paper's 96 + 32 split enables the reconstruct-then-dense call, whose per-head weights
+    # (W_Qd and W_O: 1536 x 1536 bf16 each, W_UV: 1536 x 192 and W_UK: 1152 x 192 fp16) come on top.
+    wan = B.mla_cache_device_bytes(cfg(d_nope=128))
+    paper = B.mla_cache_device_bytes(cfg(d_nope=96))
+    assert paper - wan == 2 * 1536 * 1536 * 2 + 1536 * 192 * 2 + 1152 * 192 * 2
+    # A sink frame adds its padded region (1560 -> 1664 rows) to the planes.
+    assert B.mla_cache_device_bytes(cfg(sink_frames=1)) - B.mla_cache_device_bytes(cfg()) == 1664 * 224 * 2
 
 
 def test_calls_validate_before_any_device_work():
