@@ -110,15 +110,19 @@ def sustained_peak():
 
 
 def kernel_source_hash() -> str:
-    """Hash of the CUDA sources with comments and blank lines removed (a comment edit leaves the
-    kernels, and so the ncu counters taken on them, unchanged)."""
+    """Hash of what decides the profiled kernels: the device sources, and the launch constants of
+    the host file (stage counts, tile shapes), with comments and blank lines removed, so that a
+    comment or a host-only edit leaves the kernels, and the ncu counters taken on them, valid."""
     import re
     h = hashlib.sha256()
     for f in ("ptx.cuh", "gemm_tc.cuh", "window_attn.cuh", "dense_attn.cuh", "mla_api.cu"):
         src = open(os.path.join(ROOT, "mla_latent_kv_window_b200", "csrc", f)).read()
         src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
         src = re.sub(r"//[^\n]*", "", src)
-        h.update("\n".join(l.rstrip() for l in src.splitlines() if l.strip()).encode())
+        lines = [l.rstrip() for l in src.splitlines() if l.strip()]
+        if f.endswith(".cu"):
+            lines = [l for l in lines if l.lstrip().startswith("constexpr")]
+        h.update("\n".join(lines).encode())
     return h.hexdigest()[:16]
 
 
