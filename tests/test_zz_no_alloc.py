@@ -20,14 +20,15 @@ def _cache(w: mla_synth.Workload, max_chunk: int):
     import mla_latent_kv_window_b200 as M
     dims = dict(w.dims)
     wts = {k: v.cuda() for k, v in mla_synth.make_weights(dims, mla_synth.weight_seed(w, 0)).items()}
-    cfg = M.make_config(dims, w.frame_h, w.frame_w, w.window_frames, max_chunk, batch=w.batch)
+    cfg = M.make_config(dims, w.frame_h, w.frame_w, w.window_frames, max_chunk, batch=w.batch,
+                        sink_frames=w.sink_frames)
     h = M.mla_cache_create(cfg, wts)
     fill = mla_synth.make_hidden(w.batch, w.fill_frames * w.F, dims["hidden"], mla_synth.fill_seed(w, 0)).cuda()
     M.mla_cache_append(h, fill, w.fill_frames)
     return M, h, dims
 
 
-@pytest.mark.parametrize("name", ["tiny", "wan_w21_q1"])
+@pytest.mark.parametrize("name", ["tiny", "wan_w21_q1", "paper_tiny", "sink_tiny"])
 def test_noalloc_matches_regular_entry_point_twice(name):
     w = mla_synth.WORKLOADS[name]
     M, h, dims = _cache(w, w.query_frames)
