@@ -90,7 +90,8 @@ struct GemmSmem {
   static constexpr int kABytes = M_SUB * 128 * 64 * 2;
   static constexpr int kBBytes = BN * 64 * 2;
   static constexpr int kBOffset = A_STAGES * kABytes;
-  static constexpr int kStagingOffset = kBOffset + B_STAGES * kBBytes;   // 8 warps x 2 boxes of 2 KB
+  static constexpr int kBSlots = B_STAGES ? B_STAGES : A_STAGES;   // B_STAGES == 0: shared ring
+  static constexpr int kStagingOffset = kBOffset + kBSlots * kBBytes;   // 8 warps x 2 boxes of 2 KB
   static constexpr int kBarOffset = kStagingOffset + 8 * 2 * 2048;
   static constexpr int kBytes = kBarOffset + 512 + 1024;    // barriers + alignment slack
   static_assert(kABytes % 1024 == 0 && kBBytes % 1024 == 0, "stage atoms must stay 1 KB aligned");
@@ -162,6 +163,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                    const __grid_constant__ CUtensorMap map_o2, int32_t M, int32_t K,
                    int32_t b_row0, GemmTiles tiles, EpiArgs ep, int* status) {
   using L = GemmSmem<BN, A_STAGES, B_STAGES, M_SUB>;
+  // B_STAGES == 0: one ring for A and B (one producer, one full/empty barrier pair per stage,
+  // one wait and one commit per k-block); otherwise separate rings with their own producers.
+  constexpr bool kShared = B_STAGES == 0;
   static_assert(M_SUB == 1 || M_SUB == 2, "tiles are 128 or 256 rows");
   constexpr int kAccBufs = M_SUB == 1 ? 2 : 1;   // accumulator buffers in 512 TMEM columns
   constexpr int kTileRows = 128 * M_SUB;
@@ -229,9 +233,36 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     m0 = (r - y * tiles.m_tiles) * kTileRows;
   };
 
-  if (warp == 0 || warp == 2) {
-    // ------------------------------------------------------------------ TMA producers
+  if (kShared && warp == 0) {
+    // ------------------------------------------------------------------ TMA producer (shared ring)
     if (lane == 0) {
+      const uint64_t pa = l2_policy_evict_first(), pb = l2_policy_evict_last();
+      int g = 0;
+      bool ok = true;
+      for (int i = 0; i < my_tiles && ok; ++i) {
+        int m0, y, z;
+        tile_coords(blockIdx.x + i * gridDim.x, m0, y, z);
+        const int rot = (int)((blockIdx.x + i * gridDim.x) * 7u % (unsigned)num_kb);
+        for (int kb = 0; kb < num_kb; ++kb, ++g) {
+          const int s = g % A_STAGES;
+          if (!mbar_wait(&a_empty[s], ((uint32_t)(g / A_STAGES) & 1u) ^ 1u, status)) { ok = false; break; }
+          const int kx = ((kb + rot) % num_kb) * 64;
+          mbar_arrive_expect_tx(&a_full[s], L::kABytes + L::kBBytes);
+          tma_load_3d_hint(smem + s * L::kABytes, &map_a, &a_full[s], kx, m0, z, pa);
+          tma_load_3d_hint(smem + L::kBOffset + s * L::kBBytes, &map_b, &a_full[s], kx,
+                           b_row0 + y * BN, 0, pb);
+        }
+      }
+      // Drain: never leave the CTA with a copy still landing in its shared memory (also when
+      // the loop above stopped on an error).
+      for (int q = g > A_STAGES ? g - A_STAGES : 0; q < g; ++q)
+        mbar_wait_quiesce(&a_full[q % A_STAGES], (uint32_t)(q / A_STAGES) & 1u, status);
+    }
+  } else if (kShared && warp == 2) {
+    // idle with a shared ring
+  } else if (warp == 0 || warp == 2) {
+    // ------------------------------------------------------------------ TMA producers
+    if constexpr (!kShared) if (lane == 0) {
       const bool is_a = warp == 0;
       const int stages = is_a ? A_STAGES : B_STAGES;
       uint64_t* full = is_a ? a_full : b_full;
@@ -274,9 +305,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const uint32_t acc = tmem + buf * 256;
         for (int kb = 0; kb < num_kb; ++kb, ++g) {
           const int sa = g % A_STAGES;
-          const int sb = g % B_STAGES;
+          const int sb = kShared ? sa : g % L::kBSlots;
           if (!mbar_wait(&a_full[sa], (uint32_t)(g / A_STAGES) & 1u, status) ||
-              !mbar_wait(&b_full[sb], (uint32_t)(g / B_STAGES) & 1u, status)) {
+              (!kShared && !mbar_wait(&b_full[sb], (uint32_t)(g / L::kBSlots) & 1u, status))) {
             ok = false;
             break;
           }
@@ -293,7 +324,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             }
           }
           tc_commit(&a_empty[sa]);
-          tc_commit(&b_empty[sb]);
+          if (!kShared) tc_commit(&b_empty[sb]);
         }
         tc_commit(&acc_full[buf]);
       }

@@ -43,29 +43,29 @@ constexpr int kQK = kLatent + kRope;  // 224
 // Pipeline depths of the launched kernel variants (A = activations, B = weights); each GEMM
 // CTA runs alone on its SM.  The weight ring is deep too: its L2 latency sets the k-block rate
 // when only a few CTAs run.
-constexpr int kProjAStages = 6;     // 6 x 16 KB of hidden states in flight per SM (HBM latency)
-constexpr int kProjBStages = 3;     // 3 x 28 KB of L2-resident weights
-constexpr int kProjWideAStages = 4; // 256-row tiles: 4 x 32 KB of hidden states
-constexpr int kProjWideBStages = 2;
-constexpr int kProjNarrowAStages = 8;   // 32-column latent blocks: 8 x 16 KB + 4 x 4 KB
-constexpr int kProjNarrowBStages = 4;
-constexpr int kProjMidAStages = 4;      // 256 x 160 tiles: 4 x 32 KB + 3 x 20 KB
-constexpr int kProjMidBStages = 3;
+constexpr int kProjAStages = 4;     // 128 x 224 tiles: shared ring, 4 x (16 + 28) KB
+constexpr int kProjBStages = 0;     // (B_STAGES = 0: B shares A's ring)
+constexpr int kProjWideAStages = 4; // 256 x 224 tiles (the HBM-bound fill): 4 x 32 KB of
+constexpr int kProjWideBStages = 2; //   activations in flight, weights in their own ring
+constexpr int kProjNarrowAStages = 8;   // 128 x 32 latent blocks: shared ring, 8 x (16 + 4) KB
+constexpr int kProjNarrowBStages = 0;
+constexpr int kProjMidAStages = 3;      // 256 x 160 tiles: shared ring, 3 x (32 + 20) KB
+constexpr int kProjMidBStages = 0;
 constexpr int kOutBN = 192;             // output projection column block (also the dense form's GEMMs)
-constexpr int kOutAStages = 6;
-constexpr int kOutBStages = 3;
+constexpr int kOutAStages = 4;          // shared ring, 4 x (16 + 24) KB
+constexpr int kOutBStages = 0;
 
 // Tile shapes of the projection GEMMs with the steady-state time of one 64-wide k-block in
-// microseconds, measured on B200 for one CTA per SM.  A 128-row tile is held back by the
-// per-SM rate of its activation stream, so its k-block time barely depends on BN; a 256-row
+// microseconds, measured on B200 for one CTA per SM.  A 128-row tile's k-block time barely
+// depends on BN (the per-k-block latency of loads, waits and commits dominates); a 256-row
 // tile moves twice the activations per k-block.  A launch picks the shape with the smallest
 // (waves of tiles) x (k-blocks) x (k-block time).
 struct TileShape {
   int bn, m_sub;
   double kb_us;
 };
-constexpr TileShape kShapeQ224{224, 1, 0.39}, kShapeQ160W{160, 2, 0.534},
-    kShapeQ224W{224, 2, 0.597}, kShapeL32{32, 1, 0.375};
+constexpr TileShape kShapeQ224{224, 1, 0.333}, kShapeQ160W{160, 2, 0.468},
+    kShapeQ224W{224, 2, 0.597}, kShapeL32{32, 1, 0.318};
 constexpr int kAttnStages = 4;      // 4 key tiles in flight (Q and P live in tensor memory)
 
 thread_local std::string g_last_error;
