@@ -73,13 +73,14 @@ def full_check(pair: Pair, x_chunk, what: str, intermediates: bool = True):
         ref, parts = orc.attention(x_chunk[b], return_parts=True)
         assert_close(out[b], ref, f"{what}: out (stream {b})")
         if intermediates:
-            qp = pair.gpu.copy_buffer(0, (pair.w.batch, pair.gpu.cfg.max_chunk_frames * pair.F * 12, 224))
-            assert_close(qp[b, :nq * 12], oracle_qp(pair, x_chunk[b], b), f"{what}: Qp (stream {b})")
-            ol = pair.gpu.copy_buffer(1, (pair.w.batch, pair.gpu.cfg.max_chunk_frames * pair.F * 12, 192))
+            nh = pair.dims["n_heads"]
+            qp = pair.gpu.copy_buffer(0, (pair.w.batch, pair.gpu.cfg.max_chunk_frames * pair.F * nh, 224))
+            assert_close(qp[b, :nq * nh], oracle_qp(pair, x_chunk[b], b), f"{what}: Qp (stream {b})")
+            ol = pair.gpu.copy_buffer(1, (pair.w.batch, pair.gpu.cfg.max_chunk_frames * pair.F * nh, 192))
             # o_lat is an internal bf16 intermediate, not an output: its RMS is well below its
             # peaks (rows that attend sharply copy one latent), so bf16 rounding of the queries
             # shows up as a larger max-abs/RMS than in the projected output.  Same L2 bar.
-            assert_close(ol[b, :nq * 12], parts["Pc"].reshape(-1, 192), f"{what}: o_lat (stream {b})",
+            assert_close(ol[b, :nq * nh], parts["Pc"].reshape(-1, 192), f"{what}: o_lat (stream {b})",
                          max_tol=1e-1)
     pair.check_status()
     return out
@@ -358,3 +359,28 @@ def test_reconstruct_dense_unsupported_configs():
         with pytest.raises(MLAError, match="UNSUPPORTED"):
             p.gpu.attention_reconstruct(p.hidden(1, 741).cuda())
         p.check_status()
+
+
+# ---------------------------------------------------------------------------- degenerate and other shapes
+def test_single_token_frames_single_key():
+    # F = 1 (a 1 x 1 frame grid) and an empty window: one query attends to exactly one key, its own
+    # latent, so the output is the value projection of that latent (the oracle's single-key case).
+    w = mla_synth.Workload("one_token", frame_h=1, frame_w=1, window_frames=1, fill_frames=0,
+                           query_frames=1, seed=31)
+    p = Pair(w)
+    full_check(p, p.hidden(1, 760), "one key")
+    p.append(p.hidden(1, 761))
+    check_ring(p, "one-token frame")
+    full_check(p, p.hidden(1, 762), "two keys")
+
+
+def test_narrower_model_four_heads():
+    # hidden 512 = 4 heads x 128: other column-block counts in the projections (4 + 1 blocks of
+    # 224, 512 / 192 output blocks with a ragged last one) and 4-head query rows.
+    dims = dict(mla_synth.DIMS_WAN13B, hidden=512, n_heads=4)
+    w = mla_synth.Workload("narrow_model", frame_h=6, frame_w=10, window_frames=3, fill_frames=4,
+                           query_frames=2, seed=32, dims=tuple(sorted(dims.items())))
+    p = Pair(w, max_chunk_frames=2)
+    p.append(p.hidden(4, 763))
+    check_ring(p, "4 heads")
+    full_check(p, p.hidden(2, 764), "4 heads")
