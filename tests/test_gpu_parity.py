@@ -384,3 +384,21 @@ def test_narrower_model_four_heads():
     p.append(p.hidden(4, 763))
     check_ring(p, "4 heads")
     full_check(p, p.hidden(2, 764), "4 heads")
+
+
+def test_two_sink_frames_partly_filled_then_sliding():
+    # sink_frames = 2 with F = 200: the sink region is 400 rows padded to 512 (4 key tiles).
+    # After one append only one sink frame exists, so two whole key tiles are padding (every key
+    # masked; CTAs that start their key walk there must not produce NaN); then the sink fills, the
+    # window (W = 2) fills and slides, and the query's temporal bands turn for the sink keys.
+    w = mla_synth.Workload("two_sinks", frame_h=10, frame_w=20, window_frames=2, fill_frames=1,
+                           query_frames=1, seed=33, sink_frames=2)
+    p = Pair(w)
+    seed = 770
+    for n in (1, 2, 2):
+        p.append(p.hidden(n, seed))
+        seed += 1
+        check_ring(p, f"two sinks: after append of {n}")
+        full_check(p, p.hidden(1, seed), f"two sinks: chunk after append of {n}")
+        seed += 1
+    assert p.gpu.state() == (5, 4)
