@@ -51,3 +51,23 @@ def test_two_gloo_ranks():
     assert res[0][1] == [0, 1] and res[1][1] == [2, 3]
     assert res[0][2] == res[1][2] == 2.5
     assert res[0][3] == res[1][3] == 4
+
+
+def test_reference_arm_under_torchrun_prints_once():
+    # The reference arm (the oracle on host cores) launched like the driver launches N > 1: rank 0
+    # alone works and prints one JSON line; the other rank exits 0 without work.  CPU only.
+    import json
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+           "--master-addr", "127.0.0.1", "--master-port", str(_free_port()),
+           os.path.join(root, "bench.py"), "--impl", "reference", "--gpus", "2", "--steps", "1",
+           "--warmup", "3"]
+    r = subprocess.run(cmd, capture_output=True, text=True, timeout=600, cwd=root)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1, r.stdout
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["value"] > 0 and d["cpu_baseline"]["kind"] == "oracle"
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["steps"] == 1 and d["warmup"] == 3
