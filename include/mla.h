@@ -179,10 +179,17 @@ mla_status mla_window_attention_noalloc(mla_cache* c, const void* x_chunk, int32
  *  - Needs d_nope + d_rope == 128, d_head == 128 (the paper's default dims), d_nope a multiple
  *    of 32, and sink_frames == 0; otherwise MLA_ERR_UNSUPPORTED.
  *  - The first call allocates the dense per-call buffers (per-head K and V of the largest
- *    window: 2 x batch x (W + max_chunk_frames) x F x n_heads x 256 bytes, plus the per-head
- *    queries and outputs of one chunk); they live until mla_cache_destroy. */
+ *    window: 2 x batch x (W + max_chunk_frames) x F x n_heads x 256 bytes, the per-head
+ *    queries and outputs of one chunk, and the fp32 split-key partials of the dense attention,
+ *    up to 8 x batch x max_chunk_frames x F x n_heads x 520 bytes); they live until
+ *    mla_cache_destroy. */
 mla_status mla_window_attention_reconstruct(mla_cache* c, const void* x_chunk, int32_t n_frames,
                                             void* out, void* stream);
+
+/* Bytes of device workspace with which mla_dense_attention splits the keys of each
+ * (128-query tile, head, stream) item into ranges on the current device: 0 when one pass is
+ * best for this shape (enough items to fill the GPU evenly, or too few keys to split). */
+size_t mla_dense_workspace_bytes(int32_t batch, int32_t n_q, int32_t n_kv, int32_t n_heads);
 
 /* Dense per-head attention, the layout VideoMLA replaces ([VideoMLA] §1: every cached token
  * keeps 12 x 128 keys and 12 x 128 values, 3,072 scalars): the measurement baseline of the
@@ -190,11 +197,17 @@ mla_status mla_window_attention_reconstruct(mla_cache* c, const void* x_chunk, i
  *   q   [batch][n_q][n_heads][d_head]  bf16      k, v [batch][n_kv][n_heads][d_head]  bf16
  *   out [batch][n_q][n_heads][d_head]  bf16      out = softmax(scale q k^T) v per head
  * softmax_scale 0 -> 1/sqrt(d_head).  Built for d_head == 128 (MLA_ERR_UNSUPPORTED otherwise).
- * Every query attends to all n_kv keys (no mask).  Device waits are bounded; a timeout is
- * reported by mla_dense_sync (one status word per device, shared by all dense calls). */
+ * Every query attends to all n_kv keys (no mask).
+ * workspace: NULL (or workspace_bytes 0) runs one pass per item.  Otherwise a caller-owned,
+ * 256-byte aligned device buffer of workspace_bytes bytes, in use until the call's work on
+ * `stream` completes; with mla_dense_workspace_bytes(...) bytes or more the keys are split
+ * into ranges whose fp32 partials a second kernel merges (fewer ranges if it is smaller).
+ * Device waits are bounded; a timeout is reported by mla_dense_sync (one status word per
+ * device, shared by all dense calls). */
 mla_status mla_dense_attention(const void* q, const void* k, const void* v, void* out,
                                int32_t batch, int32_t n_q, int32_t n_kv, int32_t n_heads,
-                               int32_t d_head, float softmax_scale, void* stream);
+                               int32_t d_head, float softmax_scale, void* workspace,
+                               size_t workspace_bytes, void* stream);
 
 /* Synchronise `stream` and return the dense kernels' device status word (MLA_OK or
  * MLA_ERR_DEVICE_TIMEOUT). */

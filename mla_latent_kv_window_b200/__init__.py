@@ -9,4 +9,5 @@ from .binding import (  # noqa: F401
     mla_cache_device_bytes, mla_cache_profile_enable, mla_cache_profile_read, mla_cache_read,
     mla_cache_state, mla_cache_sync, mla_config, mla_config_check, mla_ring_bytes, mla_ring_slot,
     mla_window_attention, mla_window_attention_noalloc, mla_dense_attention, mla_dense_sync,
+    mla_dense_workspace_bytes,
 )

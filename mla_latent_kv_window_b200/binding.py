@@ -28,7 +28,7 @@ EXPORTED = (
     "mla_config_check", "mla_ring_slot", "mla_ring_bytes", "mla_cache_device_bytes",
     "mla_cache_create", "mla_cache_append", "mla_window_attention", "mla_window_attention_noalloc",
     "mla_window_attention_reconstruct", "mla_cache_selftest_timeout",
-    "mla_cache_destroy", "mla_dense_attention", "mla_dense_sync",
+    "mla_cache_destroy", "mla_dense_workspace_bytes", "mla_dense_attention", "mla_dense_sync",
     "mla_cache_state", "mla_cache_sync", "mla_cache_read", "mla_cache_debug_buffers", "mla_cache_copy_buffer",
     "mla_cache_profile_enable", "mla_cache_profile_read", "mla_status_string", "mla_last_error",
 )
@@ -89,7 +89,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "mla_window_attention_noalloc": (I32, [VP, VP, I32, VP, VP]),
         "mla_window_attention_reconstruct": (I32, [VP, VP, I32, VP, VP]),
         "mla_cache_selftest_timeout": (I32, [VP, VP, P(I32)]),
-        "mla_dense_attention": (I32, [VP, VP, VP, VP, I32, I32, I32, I32, I32, ctypes.c_float, VP]),
+        "mla_dense_workspace_bytes": (ctypes.c_size_t, [I32, I32, I32, I32]),
+        "mla_dense_attention": (I32, [VP, VP, VP, VP, I32, I32, I32, I32, I32, ctypes.c_float, VP,
+                                      ctypes.c_size_t, VP]),
         "mla_dense_sync": (I32, [VP]),
         "mla_cache_destroy": (None, [VP]),
         "mla_cache_state": (I32, [VP, P(I64), P(I32)]),
@@ -208,12 +210,23 @@ def mla_cache_selftest_timeout(cache: int, stream=None) -> bool:
     return flag.value == 1
 
 
-def mla_dense_attention(q, k, v, out, softmax_scale: float = 0.0, stream=None) -> None:
-    """Dense per-head attention baseline: q [B, n_q, H, 128], k/v [B, n_kv, H, 128], out like q (bf16)."""
+def mla_dense_workspace_bytes(batch: int, n_q: int, n_kv: int, n_heads: int) -> int:
+    return int(load_library().mla_dense_workspace_bytes(batch, n_q, n_kv, n_heads))
+
+
+def mla_dense_attention(q, k, v, out, softmax_scale: float = 0.0, stream=None, workspace=None) -> None:
+    """Dense per-head attention baseline: q [B, n_q, H, 128], k/v [B, n_kv, H, 128], out like q (bf16).
+    workspace: None runs one pass per item; otherwise a uint8 device tensor (see
+    mla_dense_workspace_bytes) that holds the split-key partials."""
     B, nq, H, D = q.shape
+    ws, ws_bytes = None, 0
+    if workspace is not None and workspace.numel() > 0:
+        if not (workspace.is_cuda and workspace.is_contiguous()):
+            raise ValueError("workspace must be a contiguous CUDA tensor")
+        ws, ws_bytes = int(workspace.data_ptr()), workspace.numel() * workspace.element_size()
     _check(load_library().mla_dense_attention(_dev_ptr(q, "q"), _dev_ptr(k, "k"), _dev_ptr(v, "v"),
                                               _dev_ptr(out, "out"), B, nq, k.shape[1], H, D,
-                                              float(softmax_scale), _stream_handle(stream)),
+                                              float(softmax_scale), ws, ws_bytes, _stream_handle(stream)),
            "mla_dense_attention")
 
 

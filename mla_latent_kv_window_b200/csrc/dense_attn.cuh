@@ -12,6 +12,12 @@
 //                 O  += P_j V_j   M=128 N=128 K=128 (8 k-steps, V read MN-major, P from TMEM)
 //   warps 2..5  softmax (one row per thread, base 2, lazy O rescale), then O / l -> bf16 out.
 // TMEM columns: S0 [0,128), S1 [128,256), O [256,384), P [384,448).
+//
+// Split keys: when there are too few (query tile, head, stream) items to fill the GPU evenly
+// (1,560 queries x 12 heads = 156 items on 148 SMs would take two full waves), blockIdx.z also
+// selects one of `splits` key ranges; each CTA then writes its unnormalised O, running max and
+// sum in fp32, and dense_combine_kernel merges the ranges: out = sum_s 2^(m_s - M) O_s /
+// sum_s 2^(m_s - M) l_s.
 #pragma once
 
 #include "ptx.cuh"
@@ -38,6 +44,10 @@ struct DenseArgs {
   int32_t n_heads;
   float scale_log2;    // softmax_scale * log2(e)
   __nv_bfloat16* out;  // [B][n_q][n_heads][128]
+  int32_t splits;      // key ranges per (query tile, head, stream); 1 -> out directly
+  int32_t kv_per_split;  // keys per range (a multiple of 128)
+  float* o_part;       // splits > 1: [splits][B][n_q][n_heads][128] unnormalised O
+  float2* ml_part;     // splits > 1: [splits][B][n_q][n_heads] (max in log2 units, sum)
 };
 
 template <int KV_STAGES>
@@ -64,8 +74,11 @@ __global__ void __launch_bounds__(kDenseThreads, 1)
   const uint32_t lane = lane_id();
   const int m0 = blockIdx.x * 128;
   const int h = blockIdx.y;
-  const int z = blockIdx.z;
-  const int n_kv = args.n_kv;
+  const int z = (int)blockIdx.z / args.splits;
+  const int sp = (int)blockIdx.z - z * args.splits;   // key range of this CTA
+  const int kv0 = sp * args.kv_per_split;
+  const int kv_end = args.n_kv < kv0 + args.kv_per_split ? args.n_kv : kv0 + args.kv_per_split;
+  const int n_kv = kv_end - kv0;                      // keys of this CTA (>= 1)
   const int nt = (n_kv + 127) / 128;
   const int col0 = h * 128;  // this head's columns in the [tokens][n_heads * 128] views
 
@@ -113,8 +126,9 @@ __global__ void __launch_bounds__(kDenseThreads, 1)
         uint8_t* kv = smem + L::kKV + st * L::kStage;
         mbar_arrive_expect_tx(&kv_full[st], L::kStage);
         for (int a = 0; a < 2; ++a) {
-          tma_load_3d_hint(kv + a * L::kAtom, &map_k, &kv_full[st], col0 + a * 64, j * 128, z, keep);
-          tma_load_3d_hint(kv + (2 + a) * L::kAtom, &map_v, &kv_full[st], col0 + a * 64, j * 128, z,
+          tma_load_3d_hint(kv + a * L::kAtom, &map_k, &kv_full[st], col0 + a * 64, kv0 + j * 128, z,
+                           keep);
+          tma_load_3d_hint(kv + (2 + a) * L::kAtom, &map_v, &kv_full[st], col0 + a * 64, kv0 + j * 128, z,
                            keep);
         }
         issued = j + 1;
@@ -241,7 +255,27 @@ __global__ void __launch_bounds__(kDenseThreads, 1)
       tc_fence_before();
       mbar_arrive(p_full);
     }
-    if (ok && mbar_wait(pv_done, (uint32_t)(nt - 1) & 1u, status)) {
+    if (ok && args.splits > 1 && mbar_wait(pv_done, (uint32_t)(nt - 1) & 1u, status)) {
+      // Partial of one key range: unnormalised O, the max in log2 units and the sum, in fp32.
+      tc_fence_after();
+      const int q = m0 + row;
+      const int64_t prow = (((int64_t)sp * (gridDim.z / args.splits) + z) * args.n_q + q) * args.n_heads + h;
+#pragma unroll 1
+      for (int cq = 0; cq < 4; ++cq) {
+        uint32_t o[32];
+        tmem_ld32(tmem_o + lane_off + cq * 32, o);
+        tmem_ld_wait();
+        tmem_regs_ready(o);
+        if (q < args.n_q) {
+          float4* dst = reinterpret_cast<float4*>(args.o_part + prow * 128 + cq * 32);
+#pragma unroll
+          for (int v4 = 0; v4 < 8; ++v4)
+            dst[v4] = make_float4(__uint_as_float(o[4 * v4]), __uint_as_float(o[4 * v4 + 1]),
+                                  __uint_as_float(o[4 * v4 + 2]), __uint_as_float(o[4 * v4 + 3]));
+        }
+      }
+      if (q < args.n_q) args.ml_part[prow] = make_float2(m_used * c, l_sum);
+    } else if (ok && mbar_wait(pv_done, (uint32_t)(nt - 1) & 1u, status)) {
       tc_fence_after();
       const float inv_l = 1.f / l_sum;
       constexpr int kStride = 272;  // 256 bytes of bf16 + 16 padding
@@ -281,6 +315,34 @@ __global__ void __launch_bounds__(kDenseThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
+}
+
+// Merge of the key ranges of the split dense attention: one warp per (stream, query, head),
+// four of the 128 channels per lane.
+__global__ void dense_combine_kernel(const float* __restrict__ o_part,
+                                     const float2* __restrict__ ml_part, int splits, int batch,
+                                     int n_q, int n_heads, __nv_bfloat16* __restrict__ out) {
+  const int64_t rows = (int64_t)batch * n_q * n_heads;
+  const int64_t r = (int64_t)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (r >= rows) return;
+  float mmax = -INFINITY;
+  for (int s = 0; s < splits; ++s) mmax = fmaxf(mmax, ml_part[(int64_t)s * rows + r].x);
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  float lsum = 0.f;
+  for (int s = 0; s < splits; ++s) {
+    const float2 ml = ml_part[(int64_t)s * rows + r];
+    const float wgt = ex2_approx(ml.x - mmax);
+    lsum += wgt * ml.y;
+    const float4 o = reinterpret_cast<const float4*>(o_part + ((int64_t)s * rows + r) * 128)[lane];
+    acc.x += wgt * o.x;
+    acc.y += wgt * o.y;
+    acc.z += wgt * o.z;
+    acc.w += wgt * o.w;
+  }
+  const float inv = 1.f / lsum;
+  uint2 packed = make_uint2(pack_bf16x2(acc.x * inv, acc.y * inv), pack_bf16x2(acc.z * inv, acc.w * inv));
+  reinterpret_cast<uint2*>(out + r * 128)[lane] = packed;
 }
 
 }  // namespace mla

@@ -361,6 +361,8 @@ struct mla_cache {
   __nv_bfloat16* kd = nullptr;     // [B][n_keys][n_h][128] per call, compact
   __nv_bfloat16* vd = nullptr;     // [B][n_keys][n_h][128]
   __nv_bfloat16* od = nullptr;     // [B][n_q][n_h][128]
+  void* dws = nullptr;             // split-key partials of the dense attention
+  size_t dws_bytes = 0;
   int* status = nullptr;
 
   CUtensorMap map_wqcat{};         // B operand of the projections: box 64 x 224
@@ -680,9 +682,43 @@ mla_status dense_status_word(int** out) {
   return MLA_OK;
 }
 
+constexpr int kDenseMaxSplits = 8;
+
+// Bytes of the split-key partials for `splits` ranges: fp32 O rows, then (max, sum) pairs.
+size_t dense_ws_bytes(int splits, int batch, int n_q, int n_heads) {
+  if (splits <= 1) return 0;
+  const size_t rows = (size_t)batch * n_q * n_heads;
+  return align256((size_t)splits * rows * 128 * 4) + (size_t)splits * rows * 8;
+}
+
+// Key ranges per (query tile, head, stream) item.  Cost model in units of one 128-key tile step
+// of a full wave: the waves the CTAs take, each as long as its range plus about two tiles of
+// fixed cost (the Q tile, pipeline fill, epilogue); every split adds fp32 partial traffic of
+// about 0.018 tile steps per item (128 rows x 128 channels x 4 bytes, written and read once).
+int dense_splits(int batch, int n_q, int n_kv, int n_heads, int num_sms) {
+  const int64_t items = (int64_t)((n_q + 127) / 128) * n_heads * batch;
+  const int nt = (n_kv + 127) / 128;
+  int best = 1;
+  double best_cost = 0.0;
+  for (int s = 1; s <= kDenseMaxSplits && s <= nt; ++s) {
+    const int per = (nt + s - 1) / s;              // tiles per range
+    if ((int64_t)(s - 1) * per >= nt) break;       // the last range would be empty
+    const double waves = (double)((items * s + num_sms - 1) / num_sms);
+    const double cost = waves * (per + 2.0) + (s > 1 ? 0.018 * (double)items * (s + 1) : 0.0);
+    if (s == 1 || cost < best_cost) {
+      best = s;
+      best_cost = cost;
+    }
+  }
+  return best;
+}
+
 // Dense per-head attention over compact q [B][n_q][H][128], k, v [B][n_kv][H][128] (bf16).
+// With a workspace of dense_ws_bytes(s, ...) bytes the keys are split into s ranges (the count
+// dense_splits chooses, or fewer when the workspace holds fewer) and merged by a second kernel.
 mla_status launch_dense(const void* q, const void* k, const void* v, void* out, int batch,
-                        int n_q, int n_kv, int n_heads, float scale, int* status, cudaStream_t st) {
+                        int n_q, int n_kv, int n_heads, float scale, int* status, void* ws,
+                        size_t ws_bytes, int num_sms, cudaStream_t st) {
   const uint64_t row = (uint64_t)n_heads * 128;
   CUtensorMap mq, mk, mv;
   mla_status s;
@@ -701,10 +737,30 @@ mla_status launch_dense(const void* q, const void* k, const void* v, void* out, 
   a.n_heads = n_heads;
   a.scale_log2 = scale * 1.4426950408889634f;
   a.out = static_cast<__nv_bfloat16*>(out);
-  dim3 grid((unsigned)((n_q + 127) / 128), (unsigned)n_heads, (unsigned)batch);
+  const int nt = (n_kv + 127) / 128;
+  int splits = ws ? dense_splits(batch, n_q, n_kv, n_heads, num_sms) : 1;
+  while (splits > 1 && (dense_ws_bytes(splits, batch, n_q, n_heads) > ws_bytes ||
+                        (int64_t)batch * splits > 65535 ||
+                        (splits - 1) * ((nt + splits - 1) / splits) >= nt))
+    --splits;
+  const int per = (nt + splits - 1) / splits;
+  a.splits = splits;
+  a.kv_per_split = splits > 1 ? per * 128 : n_kv;
+  if (splits > 1) {
+    const size_t rows = (size_t)batch * n_q * n_heads;
+    a.o_part = static_cast<float*>(ws);
+    a.ml_part = reinterpret_cast<float2*>(static_cast<uint8_t*>(ws) +
+                                          align256((size_t)splits * rows * 128 * 4));
+  }
+  dim3 grid((unsigned)((n_q + 127) / 128), (unsigned)n_heads, (unsigned)(batch * splits));
   mla::dense_attn_kernel<kDenseStages>
       <<<grid, mla::kDenseThreads, mla::DenseSmem<kDenseStages>::kBytes, st>>>(mq, mk, mv, a, status);
-  return check_launch("dense attention");
+  mla_status s2 = check_launch("dense attention");
+  if (s2 != MLA_OK || splits == 1) return s2;
+  const int64_t rows = (int64_t)batch * n_q * n_heads;
+  mla::dense_combine_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(
+      a.o_part, a.ml_part, splits, batch, n_q, n_heads, static_cast<__nv_bfloat16*>(out));
+  return check_launch("dense split combine");
 }
 
 }  // namespace
@@ -828,6 +884,7 @@ void mla_cache_destroy(mla_cache* c) {
   cudaFree(c->kd);
   cudaFree(c->vd);
   cudaFree(c->od);
+  cudaFree(c->dws);
   cudaFree(c->status);
   delete c;
 }
@@ -1190,12 +1247,14 @@ mla_status mla_window_attention_reconstruct(mla_cache* c, const void* x_chunk, i
     // Per-call dense buffers, allocated once: the per-head K and V of the largest window are the
     // dense cache the latent layout avoids (B x rows x n_h x 128 x 2 bytes each).  All four or
     // none: a failed allocation leaves the cache as it was.
-    void* p[4] = {nullptr, nullptr, nullptr, nullptr};
-    const size_t bytes[4] = {(size_t)cfg.batch * c->max_q_tokens * hd * 2,
+    void* p[5] = {nullptr, nullptr, nullptr, nullptr, nullptr};
+    const size_t bytes[5] = {(size_t)cfg.batch * c->max_q_tokens * hd * 2,
                              (size_t)cfg.batch * c->max_q_tokens * hd * 2,
                              (size_t)cfg.batch * c->rows_per_stream * hd * 2,
-                             (size_t)cfg.batch * c->rows_per_stream * hd * 2};
-    for (int i = 0; i < 4; ++i) {
+                             (size_t)cfg.batch * c->rows_per_stream * hd * 2,
+                             dense_ws_bytes(kDenseMaxSplits, cfg.batch, (int)c->max_q_tokens, nh)};
+    for (int i = 0; i < 5; ++i) {
+      if (bytes[i] == 0) continue;
       const cudaError_t e = cudaMalloc(&p[i], bytes[i]);
       if (e != cudaSuccess) {
         for (int k = 0; k < i; ++k) cudaFree(p[k]);
@@ -1208,6 +1267,8 @@ mla_status mla_window_attention_reconstruct(mla_cache* c, const void* x_chunk, i
     c->od = static_cast<__nv_bfloat16*>(p[1]);
     c->kd = static_cast<__nv_bfloat16*>(p[2]);
     c->vd = static_cast<__nv_bfloat16*>(p[3]);
+    c->dws = p[4];
+    c->dws_bytes = bytes[4];
   }
   const int64_t nq = (int64_t)n_frames * c->F;
   int64_t vs, vw;
@@ -1274,7 +1335,7 @@ mla_status mla_window_attention_reconstruct(mla_cache* c, const void* x_chunk, i
   }
   // 4. dense per-head attention
   if ((s = launch_dense(c->qd, c->kd, c->vd, c->od, cfg.batch, (int)nq, (int)n_keys, nh,
-                        c->softmax_scale, c->status, st)) != MLA_OK)
+                        c->softmax_scale, c->status, c->dws, c->dws_bytes, c->num_sms, st)) != MLA_OK)
     return s;
   // 5. out = concat_h(o_h) W_O^T
   {
@@ -1308,9 +1369,19 @@ mla_status mla_cache_selftest_timeout(mla_cache* c, void* stream, int32_t* gave_
   return MLA_OK;
 }
 
+size_t mla_dense_workspace_bytes(int32_t batch, int32_t n_q, int32_t n_kv, int32_t n_heads) {
+  if (batch < 1 || n_q < 1 || n_kv < 1 || n_heads < 1) return 0;
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1)
+    return 0;
+  return dense_ws_bytes(dense_splits(batch, n_q, n_kv, n_heads, sms), batch, n_q, n_heads);
+}
+
 mla_status mla_dense_attention(const void* q, const void* k, const void* v, void* out,
                                int32_t batch, int32_t n_q, int32_t n_kv, int32_t n_heads,
-                               int32_t d_head, float softmax_scale, void* stream) {
+                               int32_t d_head, float softmax_scale, void* workspace,
+                               size_t workspace_bytes, void* stream) {
   if (!q || !k || !v || !out) return fail(MLA_ERR_INVALID_ARGUMENT, "NULL argument");
   if (batch < 1 || n_q < 1 || n_kv < 1 || n_heads < 1)
     return fail(MLA_ERR_INVALID_ARGUMENT, "batch, n_q, n_kv and n_heads must be >= 1");
@@ -1319,13 +1390,19 @@ mla_status mla_dense_attention(const void* q, const void* k, const void* v, void
     return fail(MLA_ERR_INVALID_ARGUMENT, "softmax_scale must be finite and >= 0");
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
     return fail(MLA_ERR_INVALID_ARGUMENT, "q, k, v and out must be 16-byte aligned");
+  if (workspace && (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return fail(MLA_ERR_INVALID_ARGUMENT, "workspace must be 256-byte aligned");
   if (batch > 65535 || n_heads > 65535 || (int64_t)n_q * n_heads * 128 > ((int64_t)1 << 40))
     return fail(MLA_ERR_UNSUPPORTED, "problem too large for one launch");
   int* status = nullptr;
   mla_status s = dense_status_word(&status);
   if (s != MLA_OK) return s;
   const float scale = softmax_scale > 0.f ? softmax_scale : (float)(1.0 / std::sqrt(128.0));
+  int dev = 0, sms = 0;
+  MLA_CUDA(cudaGetDevice(&dev));
+  MLA_CUDA(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
   return launch_dense(q, k, v, out, batch, n_q, n_kv, n_heads, scale, status,
+                      workspace_bytes ? workspace : nullptr, workspace_bytes, sms,
                       reinterpret_cast<cudaStream_t>(stream));
 }
 
