@@ -33,6 +33,37 @@ def test_library_exports_every_declared_symbol():
     assert set(B.EXPORTED) == declared
 
 
+def test_binding_signatures_match_header():
+    """Every declared function's parameter list (count and C type, pointers as one class) and
+    return type agree with the argtypes/restype the ctypes binding installs."""
+    lib = B.load_library()
+    header = open(os.path.join(ROOT, "include", "mla.h")).read()
+    header = re.sub(r"/\*.*?\*/", "", header, flags=re.S)
+    decls = re.findall(r"^\s*((?:const\s+)?\w+\s*\**)\s*(mla_\w+)\s*\(([^)]*)\)\s*;", header, re.M | re.S)
+    assert len(decls) == len(B.EXPORTED)
+    scalar = {"int32_t": ctypes.c_int32, "int64_t": ctypes.c_int64, "float": ctypes.c_float,
+              "double": ctypes.c_double, "size_t": ctypes.c_size_t, "mla_status": ctypes.c_int32,
+              "mla_buffer": ctypes.c_int32}   # enums are int-sized
+
+    def kind(ctype):
+        if ctype in (ctypes.c_void_p, ctypes.c_char_p) or (
+                isinstance(ctype, type) and issubclass(ctype, ctypes._Pointer)):
+            return "ptr"
+        return ctype
+
+    for ret, name, params in decls:
+        fn = getattr(lib, name)
+        params = " ".join(params.split())
+        plist = [] if params in ("", "void") else [q.strip() for q in params.split(",")]
+        assert len(plist) == len(fn.argtypes), f"{name}: {len(plist)} parameters, binding {len(fn.argtypes)}"
+        for q, at in zip(plist, fn.argtypes):
+            want = "ptr" if "*" in q else scalar[q.split()[0]]
+            assert kind(at) == want, f"{name}: parameter '{q}' bound as {at}"
+        ret = ret.replace(" ", "")
+        want_ret = None if ret == "void" else ("ptr" if "*" in ret else scalar[ret])
+        assert (fn.restype if want_ret is None else kind(fn.restype)) == want_ret, f"{name}: return {ret}"
+
+
 def test_config_check():
     assert B.mla_config_check(cfg()) == B.MLA_OK
     bad = [
