@@ -48,9 +48,11 @@ def parse_args(argv=None):
                    help="independent layer caches cycled so the step's inputs are not L2-resident")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-rows", type=int, default=1560, help="query tokens in the oracle's timed sample")
-    p.add_argument("--ncu-case", choices=("attention", "append", "steps"), default=None,
+    p.add_argument("--ncu-case", choices=("attention", "append", "steps", "dense"), default=None,
                    help="minimal launch sequence for an ncu capture (prints no benchmark line): "
-                        "'attention' = fill + 2 steps, 'append' = 2 x 21-frame fill, 'steps' = warmup + K steps")
+                        "'attention' = fill + 2 steps, 'append' = 2 x 21-frame fill, 'steps' = warmup + K steps, "
+                        "'dense' = the dense per-head baseline over the 21-frame window (2 split-key calls, "
+                        "then 1 one-pass call)")
     return p.parse_args(argv)
 
 
@@ -68,6 +70,19 @@ def run_ncu_case(args, local):
     dims = dict(w.dims)
     F, W, hidden = w.F, w.window_frames, dims["hidden"]
     nq = w.query_frames * F
+    if args.ncu_case == "dense":
+        H, n_kv = dims["n_heads"], W * F + nq
+        q = mla_synth.normal_bf16((1, nq, H, 128), 1.0, 1).to(dev)
+        k = mla_synth.normal_bf16((1, n_kv, H, 128), 1.0, 2).to(dev)
+        v = mla_synth.normal_bf16((1, n_kv, H, 128), 1.0, 3).to(dev)
+        o = torch.empty_like(q)
+        ws = torch.empty(B.mla_dense_workspace_bytes(1, nq, n_kv, H), dtype=torch.uint8, device=dev)
+        for _ in range(2):
+            B.mla_dense_attention(q, k, v, o, 0.0, None, workspace=ws)
+        B.mla_dense_attention(q, k, v, o, 0.0, None)
+        ok = B.mla_dense_sync() == 0
+        print(json.dumps({"ncu_case": args.ncu_case, "device_status_ok": ok}))
+        return 0 if ok else 1
     n_layers = 1 if args.ncu_case != "steps" else 2
     caches = []
     for layer in range(n_layers):
