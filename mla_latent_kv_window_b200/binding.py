@@ -219,6 +219,11 @@ def mla_dense_attention(q, k, v, out, softmax_scale: float = 0.0, stream=None, w
     workspace: None runs one pass per item; otherwise a uint8 device tensor (see
     mla_dense_workspace_bytes) that holds the split-key partials."""
     B, nq, H, D = q.shape
+    if k.dim() != 4 or k.shape[0] != B or k.shape[2:] != q.shape[2:] or v.shape != k.shape:
+        raise ValueError(f"k and v must be [{B}, n_kv, {H}, {D}] like each other; got {tuple(k.shape)}, "
+                         f"{tuple(v.shape)}")
+    if out.shape != q.shape:
+        raise ValueError(f"out must have the shape of q {tuple(q.shape)}; got {tuple(out.shape)}")
     ws, ws_bytes = None, 0
     if workspace is not None and workspace.numel() > 0:
         if not (workspace.is_cuda and workspace.is_contiguous()):
@@ -296,22 +301,37 @@ class LatentWindowCache:
         self.F = frame_h * frame_w
         self.handle = mla_cache_create(self.cfg, weights, stream)
 
-    def append(self, x, stream=None) -> None:
-        n = x.shape[-2] // self.F
-        mla_cache_append(self.handle, x, n, stream)
+    def _frames(self, x, name: str) -> int:
+        """Whole frames in x, which must be [batch, n * F, hidden] (the C calls take only a pointer
+        and a frame count, so the tensor's extent is checked here)."""
+        shape = tuple(x.shape)
+        if (len(shape) != 3 or shape[0] != self.cfg.batch or shape[2] != self.cfg.hidden or
+                shape[1] < self.F or shape[1] % self.F):
+            raise ValueError(f"{name} must be [{self.cfg.batch}, n * {self.F}, {self.cfg.hidden}] with "
+                             f"n >= 1; got {shape}")
+        return shape[1] // self.F
 
-    def attention(self, x_chunk, out=None, stream=None):
+    def _out_for(self, x_chunk, out):
         import torch
         if out is None:
-            out = torch.empty_like(x_chunk)
-        mla_window_attention(self.handle, x_chunk, x_chunk.shape[-2] // self.F, out, stream)
+            return torch.empty_like(x_chunk)
+        if out.shape != x_chunk.shape:
+            raise ValueError(f"out must have the shape of x_chunk {tuple(x_chunk.shape)}; got {tuple(out.shape)}")
+        return out
+
+    def append(self, x, stream=None) -> None:
+        mla_cache_append(self.handle, x, self._frames(x, "x"), stream)
+
+    def attention(self, x_chunk, out=None, stream=None):
+        n = self._frames(x_chunk, "x_chunk")
+        out = self._out_for(x_chunk, out)
+        mla_window_attention(self.handle, x_chunk, n, out, stream)
         return out
 
     def attention_reconstruct(self, x_chunk, out=None, stream=None):
-        import torch
-        if out is None:
-            out = torch.empty_like(x_chunk)
-        mla_window_attention_reconstruct(self.handle, x_chunk, x_chunk.shape[-2] // self.F, out, stream)
+        n = self._frames(x_chunk, "x_chunk")
+        out = self._out_for(x_chunk, out)
+        mla_window_attention_reconstruct(self.handle, x_chunk, n, out, stream)
         return out
 
     def state(self):

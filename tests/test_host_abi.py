@@ -160,3 +160,25 @@ def test_calls_validate_before_any_device_work():
     assert lib.mla_cache_sync(None, None) == B.MLA_ERR_INVALID_ARGUMENT
     lib.mla_cache_destroy(None)  # NULL-safe
     assert lib.mla_status_string(5) == b"MLA_ERR_DEVICE_TIMEOUT"
+
+
+def test_binding_checks_tensor_extents_before_calling():
+    """The C calls take a pointer and a frame count; the binding checks that the tensors really
+    are [batch, n * F, hidden] (and out the same) so that no call can read or write past them."""
+    import torch
+    c = B.LatentWindowCache.__new__(B.LatentWindowCache)   # no device: only the shape logic
+    c.cfg, c.F, c.handle = cfg(batch=2), 30 * 52, None
+    F, H = c.F, c.cfg.hidden
+    assert c._frames(torch.empty(2, 3 * F, H), "x") == 3
+    for bad in [(2, 3 * F + 1, H), (1, F, H), (2, F, H + 1), (2, 0, H), (3 * F, H)]:
+        with pytest.raises(ValueError):
+            c._frames(torch.empty(bad), "x")
+    x = torch.empty(2, F, H)
+    assert c._out_for(x, torch.empty(2, F, H)).shape == x.shape
+    with pytest.raises(ValueError):
+        c._out_for(x, torch.empty(2, F - 1, H))
+    q, kv = torch.empty(1, 5, 2, 128, dtype=torch.bfloat16), torch.empty(1, 7, 2, 128, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        B.mla_dense_attention(q, kv, torch.empty(1, 6, 2, 128, dtype=torch.bfloat16), q.clone())
+    with pytest.raises(ValueError):
+        B.mla_dense_attention(q, kv, kv, torch.empty(1, 4, 2, 128, dtype=torch.bfloat16))
