@@ -3,7 +3,8 @@
 Bar (bf16 inputs, fp32 accumulation): relative L2 error <= 1e-2 and max-abs error <= 3e-2 x RMS of
 the oracle output, for the layer output and the intermediates (ring contents, absorbed queries,
 latent-space attention output); ring slot placement exact.  Small cases compare every element;
-the full-size workloads compare seeded samples of query rows, which the oracle computes exactly.
+the full-size workloads compare seeded samples of query rows, which the oracle computes exactly
+(the benchmarked 21-frame, one-frame workload: every element).
 """
 import math
 
@@ -184,17 +185,22 @@ def sampled_check(pair: Pair, x_chunk, what: str, n_rows: int, seed: int):
 
 
 def test_wan_w21_q1_full_size():
+    # The benchmarked workload, every element: all 21 ring frames (32,760 rows of c_kv and
+    # k_rope), the absorbed queries and the layer output for all 1,560 query tokens.  (o_lat is
+    # compared element by element on the small workloads; here the oracle's per-head softmax
+    # matrices would take 5 GB.)
     w = mla_synth.WORKLOADS["wan_w21_q1"]
     p = Pair(w)
     p.append(p.hidden(w.fill_frames, mla_synth.fill_seed(w, 0)))
-    # ring parity on a few frames (all 21 would be 32760 rows; sample 3)
-    ckv, kr, n = p.gpu.read_ring(0)
-    contents = p.oracles[0].cache_contents()
-    for f, c, r in (contents[0], contents[10], contents[-1]):
-        s0 = ring_slot(f, 0, w.window_frames, w.F)
-        assert_close(ckv[s0:s0 + w.F], c, f"c_kv frame {f}")
-        assert_close(kr[s0:s0 + w.F], r, f"k_rope frame {f}")
-    sampled_check(p, p.hidden(1, mla_synth.chunk_seed(w, 0, 0)), "21-frame window", 96, 1)
+    check_ring(p, "21-frame fill")
+    x = p.hidden(1, mla_synth.chunk_seed(w, 0, 0))
+    out = p.attention(x)
+    nh = p.dims["n_heads"]
+    qp = p.gpu.copy_buffer(0, (1, w.F * nh, 224))
+    assert_close(qp[0], oracle_qp(p, x[0], 0), "21-frame window: Qp, every row")
+    assert_close(out[0], p.oracles[0].attention(x[0]), "21-frame window: out, every element")
+    assert torch.isfinite(out.float()).all()
+    p.check_status()
 
 
 def test_wan_b4_w21_q3_full_size():
