@@ -191,6 +191,15 @@ mla_status mla_window_attention_reconstruct(mla_cache* c, const void* x_chunk, i
  * best for this shape (enough items to fill the GPU evenly, or too few keys to split). */
 size_t mla_dense_workspace_bytes(int32_t batch, int32_t n_q, int32_t n_kv, int32_t n_heads);
 
+/* Host-only view of the key split mla_dense_attention launches on a GPU with num_sms SMs and a
+ * workspace of workspace_bytes bytes: *splits key ranges per (128-query tile, head, stream)
+ * item, each of *kv_per_split keys (a multiple of 128 when *splits > 1; the last range holds
+ * the rest and is never empty; *splits == 1 and *kv_per_split == n_kv without a workspace).
+ * No GPU needed.  MLA_ERR_INVALID_ARGUMENT for a NULL output or a size below 1. */
+mla_status mla_dense_split_plan(int32_t batch, int32_t n_q, int32_t n_kv, int32_t n_heads,
+                                int32_t num_sms, size_t workspace_bytes, int32_t* splits,
+                                int32_t* kv_per_split);
+
 /* Dense per-head attention, the layout VideoMLA replaces ([VideoMLA] §1: every cached token
  * keeps 12 x 128 keys and 12 x 128 values, 3,072 scalars): the measurement baseline of the
  * latent-window kernel.  Stateless; no device memory is allocated.

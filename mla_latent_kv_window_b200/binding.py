@@ -28,7 +28,8 @@ EXPORTED = (
     "mla_config_check", "mla_ring_slot", "mla_ring_bytes", "mla_cache_device_bytes",
     "mla_cache_create", "mla_cache_append", "mla_window_attention", "mla_window_attention_noalloc",
     "mla_window_attention_reconstruct", "mla_cache_selftest_timeout",
-    "mla_cache_destroy", "mla_dense_workspace_bytes", "mla_dense_attention", "mla_dense_sync",
+    "mla_cache_destroy", "mla_dense_split_plan", "mla_dense_workspace_bytes", "mla_dense_attention",
+    "mla_dense_sync",
     "mla_cache_state", "mla_cache_sync", "mla_cache_read", "mla_cache_debug_buffers", "mla_cache_copy_buffer",
     "mla_cache_profile_enable", "mla_cache_profile_read", "mla_status_string", "mla_last_error",
 )
@@ -89,6 +90,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "mla_window_attention_noalloc": (I32, [VP, VP, I32, VP, VP]),
         "mla_window_attention_reconstruct": (I32, [VP, VP, I32, VP, VP]),
         "mla_cache_selftest_timeout": (I32, [VP, VP, P(I32)]),
+        "mla_dense_split_plan": (I32, [I32, I32, I32, I32, I32, ctypes.c_size_t, P(I32), P(I32)]),
         "mla_dense_workspace_bytes": (ctypes.c_size_t, [I32, I32, I32, I32]),
         "mla_dense_attention": (I32, [VP, VP, VP, VP, I32, I32, I32, I32, I32, ctypes.c_float, VP,
                                       ctypes.c_size_t, VP]),
@@ -208,6 +210,15 @@ def mla_cache_selftest_timeout(cache: int, stream=None) -> bool:
     _check(load_library().mla_cache_selftest_timeout(cache, _stream_handle(stream), ctypes.byref(flag)),
            "mla_cache_selftest_timeout")
     return flag.value == 1
+
+
+def mla_dense_split_plan(batch: int, n_q: int, n_kv: int, n_heads: int, num_sms: int,
+                         workspace_bytes: int) -> tuple[int, int]:
+    """(key ranges per item, keys per range) that mla_dense_attention would launch (host only)."""
+    sp, kv = ctypes.c_int32(), ctypes.c_int32()
+    _check(load_library().mla_dense_split_plan(batch, n_q, n_kv, n_heads, num_sms, workspace_bytes,
+                                               ctypes.byref(sp), ctypes.byref(kv)), "mla_dense_split_plan")
+    return sp.value, kv.value
 
 
 def mla_dense_workspace_bytes(batch: int, n_q: int, n_kv: int, n_heads: int) -> int:

@@ -713,6 +713,21 @@ int dense_splits(int batch, int n_q, int n_kv, int n_heads, int num_sms) {
   return best;
 }
 
+// Key ranges actually launched: dense_splits, lowered until the workspace holds the partials,
+// the grid's z extent (batch x splits) fits and the last range is not empty.  Ranges are whole
+// 128-key tiles; one range (no workspace) covers all n_kv keys.
+void dense_plan(int batch, int n_q, int n_kv, int n_heads, int num_sms, size_t ws_bytes,
+                int* splits_out, int* kv_per_split_out) {
+  const int nt = (n_kv + 127) / 128;
+  int splits = ws_bytes ? dense_splits(batch, n_q, n_kv, n_heads, num_sms) : 1;
+  while (splits > 1 && (dense_ws_bytes(splits, batch, n_q, n_heads) > ws_bytes ||
+                        (int64_t)batch * splits > 65535 ||
+                        (splits - 1) * ((nt + splits - 1) / splits) >= nt))
+    --splits;
+  *splits_out = splits;
+  *kv_per_split_out = splits > 1 ? (nt + splits - 1) / splits * 128 : n_kv;
+}
+
 // Dense per-head attention over compact q [B][n_q][H][128], k, v [B][n_kv][H][128] (bf16).
 // With a workspace of dense_ws_bytes(s, ...) bytes the keys are split into s ranges (the count
 // dense_splits chooses, or fewer when the workspace holds fewer) and merged by a second kernel.
@@ -737,15 +752,10 @@ mla_status launch_dense(const void* q, const void* k, const void* v, void* out, 
   a.n_heads = n_heads;
   a.scale_log2 = scale * 1.4426950408889634f;
   a.out = static_cast<__nv_bfloat16*>(out);
-  const int nt = (n_kv + 127) / 128;
-  int splits = ws ? dense_splits(batch, n_q, n_kv, n_heads, num_sms) : 1;
-  while (splits > 1 && (dense_ws_bytes(splits, batch, n_q, n_heads) > ws_bytes ||
-                        (int64_t)batch * splits > 65535 ||
-                        (splits - 1) * ((nt + splits - 1) / splits) >= nt))
-    --splits;
-  const int per = (nt + splits - 1) / splits;
+  int splits = 1, kv_per_split = n_kv;
+  dense_plan(batch, n_q, n_kv, n_heads, num_sms, ws ? ws_bytes : 0, &splits, &kv_per_split);
   a.splits = splits;
-  a.kv_per_split = splits > 1 ? per * 128 : n_kv;
+  a.kv_per_split = kv_per_split;
   if (splits > 1) {
     const size_t rows = (size_t)batch * n_q * n_heads;
     a.o_part = static_cast<float*>(ws);
@@ -1366,6 +1376,19 @@ mla_status mla_cache_selftest_timeout(mla_cache* c, void* stream, int32_t* gave_
   int h = 0;
   MLA_CUDA(cudaMemcpy(&h, flag, sizeof(int), cudaMemcpyDeviceToHost));
   *gave_up = h;
+  return MLA_OK;
+}
+
+mla_status mla_dense_split_plan(int32_t batch, int32_t n_q, int32_t n_kv, int32_t n_heads,
+                                int32_t num_sms, size_t workspace_bytes, int32_t* splits,
+                                int32_t* kv_per_split) {
+  if (!splits || !kv_per_split) return fail(MLA_ERR_INVALID_ARGUMENT, "NULL argument");
+  if (batch < 1 || n_q < 1 || n_kv < 1 || n_heads < 1 || num_sms < 1)
+    return fail(MLA_ERR_INVALID_ARGUMENT, "batch, n_q, n_kv, n_heads and num_sms must be >= 1");
+  int s = 1, kvps = n_kv;
+  dense_plan(batch, n_q, n_kv, n_heads, num_sms, workspace_bytes, &s, &kvps);
+  *splits = s;
+  *kv_per_split = kvps;
   return MLA_OK;
 }
 

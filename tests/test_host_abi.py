@@ -182,3 +182,34 @@ def test_binding_checks_tensor_extents_before_calling():
         B.mla_dense_attention(q, kv, torch.empty(1, 6, 2, 128, dtype=torch.bfloat16), q.clone())
     with pytest.raises(ValueError):
         B.mla_dense_attention(q, kv, kv, torch.empty(1, 4, 2, 128, dtype=torch.bfloat16))
+
+
+def test_dense_split_plan_covers_every_key_once():
+    """The key ranges the dense kernel launches: whole 128-key tiles, the last range non-empty,
+    together exactly [0, n_kv); one range without a workspace; never more than 8, and the grid's
+    z extent (batch x ranges) within 65,535.  At the 21-frame, one-frame Wan shape (156 items on
+    148 SMs) the plan splits; with 444 items (three frames: three full waves) it does not."""
+    import random
+    big = 1 << 40
+    rng = random.Random(5)
+    shapes = [(1, 1560, 34320, 12), (1, 4680, 37440, 12), (2, 200, 1000, 3), (1, 5, 130, 2),
+              (1, 128, 128, 1), (3, 300, 77, 4), (1, 130, 1281, 2), (1, 40, 1, 2), (65535, 1, 5000, 1)]
+    shapes += [(rng.randint(1, 4), rng.randint(1, 5000), rng.randint(1, 120000), rng.randint(1, 16))
+               for _ in range(200)]
+    for batch, nq, nkv, nh in shapes:
+        for sms in (1, 7, 148):
+            assert B.mla_dense_split_plan(batch, nq, nkv, nh, sms, 0) == (1, nkv)
+            prev = 1
+            for ws in (1 << 20, 1 << 26, big):
+                s, per = B.mla_dense_split_plan(batch, nq, nkv, nh, sms, ws)
+                assert 1 <= s <= 8 and batch * s <= 65535
+                if s == 1:
+                    assert per == nkv
+                else:
+                    assert per % 128 == 0 and (s - 1) * per < nkv <= s * per
+                assert s >= prev or ws == (1 << 20)
+                prev = s
+    assert B.mla_dense_split_plan(1, 1560, 34320, 12, 148, big)[0] > 1
+    assert B.mla_dense_split_plan(1, 4680, 37440, 12, 148, big)[0] == 1
+    with pytest.raises(B.MLAError):
+        B.mla_dense_split_plan(0, 1, 1, 1, 148, big)
