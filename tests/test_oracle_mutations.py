@@ -7,8 +7,6 @@ import os
 import subprocess
 import sys
 
-import pytest
-
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 ORACLE = os.path.join(ROOT, "oracle", "mla_oracle.py")
 
@@ -48,6 +46,15 @@ MUTATIONS = [
      "            self.frames_appended += 1\n            entry = (self.frames_appended, c[sl], r[sl])"),
     ("sink frames never kept", "if len(self.sink) < self.n_sink:", "if len(self.sink) < self.n_sink and False:"),
     ("sink frames ordered after the window", "return self.sink + self.frames", "return self.frames + self.sink"),
+    ("token grid transposed (column-major h, w)", "return k // frame_w, k % frame_w", "return k % frame_w, k // frame_w"),
+    ("ring slot one frame ahead", "return (frame % window_frames) * tokens_per_frame + token",
+     "return ((frame + 1) % window_frames) * tokens_per_frame + token"),
+    ("RoPE axes in the order h, t, w", "for a, d_a in enumerate((rope_t, rope_h, rope_w)):",
+     "for a, d_a in enumerate((rope_h, rope_t, rope_w)):"),
+    ("dense baseline without the softmax scale", "S = (q[:, h, :] @ k[:, h, :].T) * scale",
+     "S = (q[:, h, :] @ k[:, h, :].T)"),
+    ("dense baseline normalising over queries", "out[:, h, :] = (E / E.sum(axis=1, keepdims=True)) @ v[:, h, :]",
+     "out[:, h, :] = (E / E.sum(axis=0, keepdims=True)) @ v[:, h, :]"),
 ]
 
 # Loads the given oracle source as the `oracle` package, then runs the pins in this process.
