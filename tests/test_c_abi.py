@@ -5,6 +5,7 @@ oracle's definition of the frame ring."""
 import os
 import shutil
 import subprocess
+import tempfile
 
 import pytest
 
@@ -70,3 +71,20 @@ def test_errors_from_c(c_output):
     assert int(status) == 1 and int(has_message) == 1
     assert c_output["status_name_0"] == ["MLA_OK"]
     assert c_output["status_name_5"] == ["MLA_ERR_DEVICE_TIMEOUT"]
+
+
+def test_full_path_client_compiles_and_links():
+    """tests/c_abi_rollout.c drives create / append / attention / sync / destroy from C with
+    device buffers of the CUDA runtime; here it must compile and link against libmla.so (it
+    needs a GPU to run)."""
+    gcc = shutil.which("gcc")
+    cuda = os.environ.get("CUDA_HOME", "/usr/local/cuda")
+    if gcc is None or not os.path.exists(os.path.join(cuda, "include", "cuda_runtime_api.h")):
+        pytest.skip("no C compiler or CUDA headers")
+    B.load_library()
+    exe = os.path.join(tempfile.mkdtemp(), "c_abi_rollout")
+    subprocess.run([gcc, "-std=c11", "-Wall", "-Wextra", "-Werror", "-I", os.path.join(ROOT, "include"),
+                    "-I", os.path.join(cuda, "include"), os.path.join(ROOT, "tests", "c_abi_rollout.c"),
+                    "-L", PKG, "-lmla", "-L", os.path.join(cuda, "lib64"), "-lcudart", "-lm",
+                    "-Wl,-rpath," + PKG, "-o", exe], check=True)
+    assert os.path.getsize(exe) > 0
