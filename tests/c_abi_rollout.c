@@ -1,7 +1,6 @@
 /* Plain C client (C11: the CUDA runtime headers use anonymous unions) of the whole path through
- * libmla.so: create a cache, fill the window, run the
- * attention call for a query chunk, append it, and read the status word, with device buffers
- * from the CUDA runtime.  tests/test_c_abi.py compiles and links it without a GPU; on a GPU it
+ * libmla.so: create a cache, fill the window, run the attention call for a query chunk, append
+ * it, and read the status word, with device buffers from the CUDA runtime.  tests/test_c_abi.py compiles and links it without a GPU; on a GPU it
  * runs as a rollout of a few frames of a small layer and exits 0 when every call succeeded and
  * the outputs are finite.  Inputs are seeded uniform values in [-1, 1) (weights scaled by
  * 1/sqrt(fan_in)), converted to bf16 on the host. */
