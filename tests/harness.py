@@ -1,8 +1,8 @@
 """Shared helpers of the GPU parity tests: run one seeded workload through the C ABI and the
 fp64 oracle on identical bf16 inputs, and compare with the stated tolerance.
 
-Tolerance (bf16 inputs, bf16 cache/queries/P/o_lat, fp32 accumulation) against the fp64 oracle:
-relative L2 error <= 1e-2 and max-abs error <= 3e-2 x RMS(oracle output).
+Tolerance (bf16 inputs and weights; fp16 cache, queries, P and o_lat; fp32 accumulation) against
+the fp64 oracle: relative L2 error <= 1e-2 and max-abs error <= 3e-2 x RMS(oracle output).
 """
 from __future__ import annotations
 

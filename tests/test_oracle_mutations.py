@@ -51,6 +51,15 @@ MUTATIONS = [
      "return ((frame + 1) % window_frames) * tokens_per_frame + token"),
     ("RoPE axes in the order h, t, w", "for a, d_a in enumerate((rope_t, rope_h, rope_w)):",
      "for a, d_a in enumerate((rope_h, rope_t, rope_w)):"),
+    ("ring contents rotated at the window-local index instead of the absolute one",
+     "for f, c, r in self.active_frames():\n            out.append((f, c.copy(), self._rope(r, f, hh, ww)))",
+     "for i, (f, c, r) in enumerate(self.active_frames()):\n            out.append((f, c.copy(), self._rope(r, i, hh, ww)))"),
+    ("ring contents with h and w swapped", "out.append((f, c.copy(), self._rope(r, f, hh, ww)))",
+     "out.append((f, c.copy(), self._rope(r, f, ww, hh)))"),
+    ("ring contents left unrotated", "out.append((f, c.copy(), self._rope(r, f, hh, ww)))",
+     "out.append((f, c.copy(), r.copy()))"),
+    ("ring contents one frame ahead in time", "out.append((f, c.copy(), self._rope(r, f, hh, ww)))",
+     "out.append((f, c.copy(), self._rope(r, f + 1, hh, ww)))"),
     ("dense baseline without the softmax scale", "S = (q[:, h, :] @ k[:, h, :].T) * scale",
      "S = (q[:, h, :] @ k[:, h, :].T)"),
     ("dense baseline normalising over queries", "out[:, h, :] = (E / E.sum(axis=1, keepdims=True)) @ v[:, h, :]",

@@ -395,3 +395,53 @@ def test_sink_segment_rotation_equals_local():
         k_loc = rope(loc["r"], loc["t_key"], loc["h_key"], loc["w_key"])
         np.testing.assert_allclose(s_gpu, q_loc @ k_loc.T, rtol=1e-10, atol=1e-12)
 
+
+
+# ---------------------------------------------------------------------------- ring contents (rotate at append)
+def _brute_ring_contents(dims, W, x_all, n_appended):
+    """What a ring rotating at append time holds, written out with the scalar loops of
+    tests/brute_mla.py: which frames survive is stated directly (the first sink_frames frames,
+    then the newest window_frames of the rest), and each token's positional key is turned at its
+    frame's ABSOLUTE index t = f and grid position (k // frame_w, k % frame_w)."""
+    S, Wn = dims.get("sink_frames", 0), dims["window_frames"]
+    F, fw = dims["frame_h"] * dims["frame_w"], dims["frame_w"]
+    split = (dims["rope_t"], dims["rope_h"], dims["rope_w"])
+    n_sink = min(n_appended, S)
+    kept = list(range(n_sink)) + list(range(max(n_sink, n_appended - Wn), n_appended))
+    out = []
+    for f in kept:
+        cs, rs = [], []
+        for k in range(F):
+            x = x_all[f * F + k]
+            cs.append(brute_mla.matvec(W["w_dkv"], x))
+            rs.append(brute_mla.rotate(brute_mla.matvec(W["w_kr"], x), f, k // fw, k % fw, split,
+                                       dims["rope_base"]))
+        out.append((f, cs, rs))
+    return out
+
+
+@pytest.mark.parametrize("sink", [0, 1, 2])
+def test_cache_contents_brute_force_absolute_index(sink):
+    # The GPU ring is checked against OracleLayer.cache_contents, so it is pinned here on its
+    # own: after appends that slide the window (and wrap a 3-frame ring twice), every kept frame's
+    # c_kv and k_rope (turned at the absolute frame index, App. D.5 read as "rotate at append")
+    # must equal the scalar-loop statement above.  A non-square frame grid (2 x 3) and
+    # unequal per-axis widths make an h/w swap or a wrong axis visible.
+    dims = _tiny_dims(window_frames=3, frame_h=2, frame_w=3, sink_frames=sink, d_rope=8,
+                      rope_t=2, rope_h=4, rope_w=2)
+    layer, w = _layer(dims, 31 + sink)
+    F = 6
+    x = mla_synth.make_hidden(1, 12 * F, dims["hidden"], 40 + sink)[0]
+    Wl = {k: v.double().tolist() for k, v in w.items()}
+    xl = x.double().tolist()
+    seen = 0
+    for n in (2, 1, 5, 1, 3):
+        layer.append(x[seen * F:(seen + n) * F])
+        seen += n
+        got = layer.cache_contents()
+        ref = _brute_ring_contents(dims, Wl, xl, seen)
+        assert [f for f, _, _ in got] == [f for f, _, _ in ref]
+        for (f, c, r), (_, c_ref, r_ref) in zip(got, ref):
+            np.testing.assert_allclose(c, np.array(c_ref), rtol=1e-13, atol=1e-13)
+            np.testing.assert_allclose(r, np.array(r_ref), rtol=1e-13, atol=1e-13)
+    assert seen == 12 and layer.frames_appended == 12
