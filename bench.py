@@ -36,6 +36,7 @@ FLOP_PER_QHK = 832          # 2*(192+32) for scores + 2*192 for P.c_kv, per (que
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 L2_BYTES = 126 * 1024 * 1024
+REF_HEADS = 4              # heads per reference-arm step (of 12)
 
 
 def parse_args(argv=None):
@@ -661,25 +662,28 @@ def cpu_baseline(w, rows: int) -> dict:
 
 
 def run_reference(args, rank, world):
-    """The oracle timed on the host cores as the reference arm (rank 0 only)."""
+    """The oracle timed on the host cores as the reference arm (rank 0 only).
+
+    One step is the benchmarked step's work in the oracle: append the previous query frame (the
+    window slides by one frame), then attend all 1,560 query tokens of the next frame over the
+    whole window and the frame itself, for REF_HEADS of the 12 heads (a different group each
+    step).  Heads are independent and cost the same (each materialises its own K and V over all
+    keys), so a step is a third of a full step's work in the same proportions, and the value, in
+    query-token equivalents (tokens x heads / 12) per second, measures the same rate as the
+    cpu_baseline leg's full step."""
     if rank != 0:
         return
-    import numpy as np
-
     import mla_synth
     w = mla_synth.WORKLOADS[WORKLOAD]
     orc = _oracle_layer(w)
     nq = w.query_frames * w.F
+    n_heads = w.dim("n_heads")
     chunks = [mla_synth.make_hidden(1, nq, w.dim("hidden"), mla_synth.chunk_seed(w, 0, s))[0] for s in range(4)]
-    rows_per_step = 8
-    heads = list(range(w.dim("n_heads")))
-    # One step: append the previous chunk (window slides by one frame) and attend a bounded sample of
-    # query rows of one head over the whole window + chunk.  Token-equivalents: rows * heads_used / 12.
+
     def step(s):
-        x = chunks[s % 4]
-        sel = np.arange(s * 37, s * 37 + rows_per_step * 97, 97) % nq
-        orc.attention(x, rows=sel, heads=[heads[s % len(heads)]])
-        orc.append(x)
+        heads = [(s * REF_HEADS + i) % n_heads for i in range(REF_HEADS)]
+        orc.attention(chunks[s % 4], heads=heads)
+        orc.append(chunks[s % 4])
 
     for s in range(args.warmup):
         step(s)
@@ -687,11 +691,12 @@ def run_reference(args, rank, world):
     for s in range(args.steps):
         step(args.warmup + s)
     dt = time.perf_counter() - t0
-    tok = args.steps * rows_per_step / len(heads)
+    tok = args.steps * nq * REF_HEADS / n_heads
     value = tok / dt
     cores = blas_threads()
-    sample = (f"per step: 1-frame append + {rows_per_step} query rows x 1 of 12 heads over all "
-              f"{w.window_frames * w.F + nq} keys (float64 NumPy oracle); value counts rows*heads/12 token-equivalents")
+    sample = (f"per step: 1-frame append + all {nq} query tokens x {REF_HEADS} of {n_heads} heads over all "
+              f"{w.window_frames * w.F + nq} keys (float64 NumPy oracle, per-head K/V materialised); "
+              f"value counts tokens*heads/{n_heads} token-equivalents")
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * dt / max(args.steps, 1), 3),
