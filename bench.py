@@ -193,6 +193,7 @@ class ClockSampler:
             self.t1 = time.time()
 
     def stop(self) -> dict:
+        """End sampling; the record of the timed region marked with mark()."""
         time.sleep(0.15)
         if self.proc:
             self.proc.terminate()
@@ -200,13 +201,17 @@ class ClockSampler:
                 self.proc.wait(timeout=5)
             except Exception:
                 self.proc.kill()
+        return self.window(self.t0, self.t1)
+
+    def window(self, t0, t1) -> dict:
+        """Median SM clock and the throttle reasons of the samples taken in [t0, t1] (host time)."""
         rows = []
-        for t, line in self.lines:
+        for t, line in list(self.lines):
             parts = [x.strip() for x in line.split(",")]
             if len(parts) < 9:
                 continue
             rows.append((t, parts))
-        inside = [r for t, r in rows if self.t0 is not None and self.t0 - 0.05 <= t <= (self.t1 or t) + 0.05]
+        inside = [r for t, r in rows if t0 is not None and t0 - 0.05 <= t <= (t1 or t) + 0.05]
         use = inside or [r for _, r in rows]
         sm = [float(r[1]) for r in use if r[1].replace(".", "").isdigit()]
         mx = [float(r[2]) for r in use if r[2].replace(".", "").isdigit()]
@@ -259,6 +264,15 @@ def run_ours(args, rank, local, world):
     stream = torch.cuda.current_stream()
 
     def step(s):
+        # One rollout step of one layer: the frame attends to the window plus itself, then its
+        # latents (computed by the query projection) become part of the window.
+        c = caches[s % L]
+        x = chunks[s % 4]
+        B.mla_window_attention(c.handle, x, w.query_frames, out, stream)
+        B.mla_cache_commit(c.handle, w.query_frames, stream)
+
+    def step_append(s):
+        # The same step with the frame's latents recomputed from x by mla_cache_append.
         c = caches[s % L]
         x = chunks[s % 4]
         B.mla_window_attention(c.handle, x, w.query_frames, out, stream)
@@ -304,7 +318,6 @@ def run_ours(args, rank, local, world):
     torch.cuda.synchronize()
     clocks.mark("stop")
     replicas.barrier()
-    clk = clocks.stop()
     ms_local = e0.elapsed_time(e1)
     ms = replicas.max_over_ranks(ms_local, dev)
 
@@ -323,10 +336,20 @@ def run_ours(args, rank, local, world):
             prof[k][0] += t
             prof[k][1] += n
         B.mla_cache_profile_enable(c.handle, False)
-    launches = 4 * args.steps   # each step launches Q-projection, attention, output projection, append
+    launches = 4 * args.steps   # each step launches Q-projection, attention, output projection, commit copy
     assert sum(n for _, n in prof.values()) == launches
     attn_ms = prof["attention"][0] / max(prof["attention"][1], 1)
     attn_ms = replicas.max_over_ranks(attn_ms, dev)
+
+    # ---- the same K steps with the frame appended by recomputing its latents from x
+    replicas.barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for s in range(args.steps):
+        step_append(args.warmup + 2 * args.steps + s)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms_append = replicas.max_over_ranks(e0.elapsed_time(e1), dev)
 
     tokens = world * nq * args.steps
     value = tokens / (ms / 1e3)
@@ -363,7 +386,7 @@ def run_ours(args, rank, local, world):
         if used[i]:
             compute.wait_event(drained[i])           # step s-2's output has left out_dev[i]
         B.mla_window_attention(c.handle, x_dev[i], w.query_frames, out_dev[i], compute)
-        B.mla_cache_append(c.handle, x_dev[i], w.query_frames, compute)
+        B.mla_cache_commit(c.handle, w.query_frames, compute)
         computed[i].record(compute)
         with torch.cuda.stream(d2h):
             d2h.wait_event(computed[i])
@@ -389,12 +412,37 @@ def run_ours(args, rank, local, world):
     e2e_value = world * nq * e2e_steps / (e2e_ms / 1e3)
 
     status_ok = all(B.mla_cache_sync(c.handle) == 0 for c in caches)
+    for c in caches:
+        c.close()
+    caches.clear()
+    torch.cuda.empty_cache()
+    # Every rank takes part in the batched leg (its streams are sharded over the ranks).
+    leg_t = {}
+    t_a = time.time()
+    batched = batched_leg(B, dev, stream, rank, world, tf_peak, hbm_peak)
+    leg_t["wan_b4_w21_q3"] = (t_a, time.time())
     layout = layout_baseline(B, w, dims, dev, stream, attn_ms, attn_flop) if rank == 0 else None
     nxt = next_rows(B, dev) if rank == 0 else None
+    t_a = time.time()
+    rollout = rollout_leg(B, dev, stream, tf_peak) if rank == 0 else None
+    leg_t["wan_30l_w21_q3_wrap"] = (t_a, time.time())
+    tiny = tiny_leg(B, dev, stream) if rank == 0 else None
+    clk = clocks.stop()
+    for name, leg in (("wan_b4_w21_q3", batched.get("attention") if batched else None),
+                      ("wan_30l_w21_q3_wrap", rollout)):
+        if leg is not None:
+            c = clocks.window(*leg_t[name])
+            leg["clocks"] = {"sm_mhz": c["sm_mhz"], "reasons": c["reasons"], "samples": c["samples_in_timed_region"]}
+            tf = leg.get("attention_tflops") or leg.get("attention_tflops_per_gpu")
+            if tf and c["sm_mhz"]:
+                # against what the tensor cores can do at the median sampled clock (8,192 flop/clk/SM)
+                leg["attention_frac_of_tensor_rate_at_clock"] = round(
+                    tf / (8192 * torch.cuda.get_device_properties(dev).multi_processor_count * c["sm_mhz"] * 1e-6), 4)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w, args.cpu_rows)
+        cpu["per_workload"] = cpu_workloads()
     replicas.barrier()
 
     if rank == 0:
@@ -402,13 +450,17 @@ def run_ours(args, rank, local, world):
             "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 5),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "precision": "bf16 hidden states, weights and output; fp16 cache planes, absorbed queries, P "
+                         "and o_lat (tcgen05 kind::f16 operands); fp32 accumulation and softmax",
+            "ms_per_step_append_recompute": round(ms_append / args.steps, 5),
             "data": "synthetic: seeded N(0,1) hidden states, N(0,1/fan_in) weights (no checkpoint)",
             "config": {
                 "workload": f"{WORKLOAD}: Wan-1.3B-shaped layer, 21-frame latent window (32,760 cached tokens) "
                             f"+ one 1,560-token query frame",
                 "hidden": hidden, "n_heads": dims["n_heads"], "d_latent": 192, "d_rope": 32, "d_nope": dims["d_nope"],
                 "tokens_per_frame": F, "window_frames": W, "query_tokens": nq, "keys": n_keys, "batch": 1,
-                "step": "mla_window_attention (Q-proj + latent-window attention + out-proj) then a 1-frame mla_cache_append",
+                "step": "mla_window_attention (Q-proj with the frame's latents + latent-window attention + "
+                        "out-proj) then mla_cache_commit (the frame's latents moved into the ring slot)",
                 "l2": f"inputs larger than L2: {L} independent layer caches cycled "
                       f"({L * per_cache_bytes / 2**20:.0f} MB > 126 MB)",
                 "parallelism": f"replicas x{world} (no data-path collective)",
@@ -443,6 +495,11 @@ def run_ours(args, rank, local, world):
             "device_status_ok": status_ok,
             "clocks": clk,
         }
+        line["workloads"] = {k: v for k, v in (("tiny", tiny), ("wan_30l_w21_q3_wrap", rollout),
+                                               ("wan_b4_w21_q3", batched.get("attention") if batched else None))
+                             if v is not None}
+        if batched:
+            line["append_roofline_b4"] = batched["fill"]
         if layout is not None:
             line["layout_baseline"] = layout
         if nxt is not None:
@@ -450,9 +507,171 @@ def run_ours(args, rank, local, world):
         if cpu is not None:
             line["cpu_baseline"] = cpu
         print(json.dumps(line), flush=True)
+    replicas.shutdown()
+
+
+def _profiled_attention_ms(B, caches, fn, warm=1, reps=3):
+    """Run fn (warm + reps times) with per-launch events on every cache; returns the per-launch
+    device ms of each kernel kind over the timed reps, and the launch counts."""
+    import torch
+    for c in caches:
+        B.mla_cache_profile_enable(c.handle, True)
+    for _ in range(warm):
+        fn()
+    torch.cuda.synchronize()
+    for c in caches:
+        B.mla_cache_profile_read(c.handle)
+    for _ in range(reps):
+        fn()
+    torch.cuda.synchronize()
+    tot = {k: [0.0, 0] for k in B.KERNEL_NAMES}
+    for c in caches:
+        for k, (t, n) in B.mla_cache_profile_read(c.handle).items():
+            tot[k][0] += t
+            tot[k][1] += n
+        B.mla_cache_profile_enable(c.handle, False)
+    return {k: (t / n if n else 0.0, n) for k, (t, n) in tot.items()}
+
+
+def rollout_leg(B, dev, stream, tf_peak, reps=2):
+    """The 30-layer rollout of the Wan-1.3B geometry: 30 layers with independent weights, each
+    with a 21-frame ring that has wrapped (24 frames appended, the oldest 3 evicted); one 3-frame
+    chunk (4,680 query tokens) is denoised in 4 steps (every step runs all 30 layers against
+    the same caches), then its latents are committed to every layer's window.  Reported per
+    layer-step: query tokens/s over the whole chunk (120 layer-steps + 30 commits), and the
+    attention kernel's TFLOP/s over 37,440 keys."""
+    import torch
+
+    import mla_synth
+    w = mla_synth.WORKLOADS["wan_30l_w21_q3_wrap"]
+    dims = dict(w.dims)
+    F, hidden, Q = w.F, dims["hidden"], w.query_frames
+    caches = []
+    for layer in range(w.layers):
+        wts = {k: v.to(dev) for k, v in mla_synth.make_weights(dims, mla_synth.weight_seed(w, layer)).items()}
+        c = B.LatentWindowCache(dims, wts, w.frame_h, w.frame_w, w.window_frames, Q)
+        c.append(mla_synth.make_hidden(1, w.fill_frames * F, hidden, mla_synth.fill_seed(w, layer)).to(dev))
+        caches.append(c)
+    xs = [mla_synth.make_hidden(1, Q * F, hidden, mla_synth.chunk_seed(w, 0, st)).to(dev) for st in range(w.steps)]
+    out = torch.empty_like(xs[0])
+
+    def chunk():
+        for st in range(w.steps):
+            for c in caches:
+                B.mla_window_attention(c.handle, xs[st], Q, out, stream)
+        for c in caches:
+            B.mla_cache_commit(c.handle, Q, stream)
+
+    chunk()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        chunk()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / reps
+    prof = _profiled_attention_ms(B, caches, chunk, warm=0, reps=1)
+    ok = all(B.mla_cache_sync(c.handle) == 0 for c in caches)
+    _, valid = caches[0].state()
     for c in caches:
         c.close()
-    replicas.shutdown()
+    nq = Q * F
+    keys = valid * F + nq
+    layer_steps = w.layers * w.steps
+    a_ms = prof["attention"][0]
+    flop = FLOP_PER_QHK * nq * dims["n_heads"] * keys
+    return {"workload": "30 Wan-1.3B-shaped layers, 21-frame wrapped ring, 3-frame chunk (4,680 query tokens) "
+                        "x 4 denoising steps, then the chunk committed to every layer",
+            "keys": keys, "query_tokens_per_layer_step": nq, "layer_steps_per_chunk": layer_steps,
+            "ms_per_chunk": round(ms, 3),
+            "query_tokens_per_s_per_layer_step": round(nq * layer_steps / (ms / 1e3), 1),
+            "attention_ms": round(a_ms, 4), "attention_tflops": round(flop / (a_ms / 1e3) / 1e12, 1),
+            "attention_frac_of_peak": round(flop / (a_ms / 1e3) / 1e12 / tf_peak, 4),
+            "kernel_ms_per_launch": {k: round(t, 5) for k, (t, n) in prof.items() if n},
+            "status_ok": ok}
+
+
+def batched_leg(B, dev, stream, rank, world, tf_peak, hbm_peak, reps=5):
+    """B = 4 independent streams (per-stream hidden-state scale in [0.5, 2]), each a 21-frame
+    window and a 3-frame chunk, sharded over the ranks (replicas.shard): each rank holds a cache
+    of its own streams, no collective on the data path.  Also the fill of those windows
+    (mla_cache_append of 21 frames per stream), the append's HBM roofline point at B = 4."""
+    import torch
+
+    import mla_synth
+    from mla_latent_kv_window_b200 import replicas
+    w = mla_synth.WORKLOADS["wan_b4_w21_q3"]
+    dims = dict(w.dims)
+    F, hidden, Q, W = w.F, dims["hidden"], w.query_frames, w.window_frames
+    mine = list(replicas.shard(w.batch, rank, world))
+    nb = len(mine)
+    fill_ms = attn_call_ms = a_ms = 0.0
+    ok = True
+    if nb:
+        scales = mla_synth.stream_scales(w.batch, w.seed)
+        wts = {k: v.to(dev) for k, v in mla_synth.make_weights(dims, mla_synth.weight_seed(w, 0)).items()}
+        c = B.LatentWindowCache(dims, wts, w.frame_h, w.frame_w, W, Q, batch=nb)
+        x_fill = mla_synth.make_hidden(w.batch, W * F, hidden, mla_synth.fill_seed(w, 0), scales)[mine].to(dev)
+        c.append(x_fill)
+        torch.cuda.synchronize()
+        # Fill roofline: x is 4 x 32,760 x 1536 bf16 = 403 MB, larger than L2, so every fill
+        # reads it from HBM.
+        fill_ms = _event_ms(lambda: B.mla_cache_append(c.handle, x_fill, W, stream), stream, reps=reps, warm=2)
+        del x_fill
+        x = mla_synth.make_hidden(w.batch, Q * F, hidden, mla_synth.chunk_seed(w, 0, 0), scales)[mine].to(dev)
+        out = torch.empty_like(x)
+        attn_call_ms = _event_ms(lambda: B.mla_window_attention(c.handle, x, Q, out, stream), stream, reps=reps, warm=2)
+        prof = _profiled_attention_ms(B, [c], lambda: B.mla_window_attention(c.handle, x, Q, out, stream))
+        a_ms = prof["attention"][0]
+        ok = B.mla_cache_sync(c.handle) == 0
+        c.close()
+    fill_ms = replicas.max_over_ranks(fill_ms, dev)
+    attn_call_ms = replicas.max_over_ranks(attn_call_ms, dev)
+    a_ms = replicas.max_over_ranks(a_ms, dev)
+    nq, keys = Q * F, W * F + Q * F
+    per_rank_streams = max(len(replicas.shard(w.batch, r, world)) for r in range(world))
+    flop = FLOP_PER_QHK * per_rank_streams * nq * dims["n_heads"] * keys
+    fill_bytes = per_rank_streams * W * F * (hidden * 2 + 224 * 2) + 224 * hidden * 2
+    return {
+        "attention": {
+            "workload": f"B = 4 streams sharded over {world} GPU(s) ({per_rank_streams} per GPU at most), "
+                        f"21-frame window, 3-frame chunk, per-stream scale in [0.5, 2]",
+            "keys": keys, "query_tokens": w.batch * nq, "call_ms": round(attn_call_ms, 4),
+            "query_tokens_per_s": round(w.batch * nq / (attn_call_ms / 1e3), 1),
+            "attention_ms": round(a_ms, 4),
+            "attention_tflops_per_gpu": round(flop / (a_ms / 1e3) / 1e12, 1) if a_ms else None,
+            "attention_frac_of_peak": round(flop / (a_ms / 1e3) / 1e12 / tf_peak, 4) if a_ms else None,
+            "status_ok": ok},
+        "fill": {
+            "kernel": "tc_gemm_kernel<224,latent> (21-frame fill of the B = 4 streams, x from HBM)",
+            "bound": "hbm", "ms_per_launch": round(fill_ms, 5),
+            "achieved": round(fill_bytes / (fill_ms / 1e3) / 1e9, 1), "peak": hbm_peak, "unit": "GB/s",
+            "frac": round(fill_bytes / (fill_ms / 1e3) / 1e9 / hbm_peak, 4),
+            "algorithmic": f"{per_rank_streams} x 32,760 tokens x (3072 B in + 448 B out) + 688,128 B weights "
+                           f"= {fill_bytes / 1e6:.1f} MB per GPU",
+            "status_ok": ok},
+    }
+
+
+def tiny_leg(B, dev, stream):
+    """The small workload (4 x 6 frames, 2-frame window, one query frame): launch-bound."""
+    import torch
+
+    import mla_synth
+    w = mla_synth.WORKLOADS["tiny"]
+    dims = dict(w.dims)
+    wts = {k: v.to(dev) for k, v in mla_synth.make_weights(dims, mla_synth.weight_seed(w, 0)).items()}
+    c = B.LatentWindowCache(dims, wts, w.frame_h, w.frame_w, w.window_frames, w.query_frames)
+    c.append(mla_synth.make_hidden(1, w.fill_frames * w.F, dims["hidden"], mla_synth.fill_seed(w, 0)).to(dev))
+    x = mla_synth.make_hidden(1, w.F, dims["hidden"], mla_synth.chunk_seed(w, 0, 0)).to(dev)
+    out = torch.empty_like(x)
+    ms = _event_ms(lambda: B.mla_window_attention(c.handle, x, 1, out, stream), stream, reps=20)
+    ok = B.mla_cache_sync(c.handle) == 0
+    c.close()
+    return {"workload": "4 x 6-token frames, 2-frame window, one query frame (72 keys)", "call_ms": round(ms, 4),
+            "query_tokens_per_s": round(w.F / (ms / 1e3), 1), "status_ok": ok,
+            "note": "launch-bound: three kernels for 24 query tokens"}
 
 
 def _event_ms(fn, stream, reps=10, warm=3):
@@ -659,6 +878,35 @@ def cpu_baseline(w, rows: int) -> dict:
             "seconds": round(dt, 2),
             "sample": f"{rows} of {x.shape[0]} query tokens of one step (12 heads, {w.window_frames * w.F + x.shape[0]} keys, "
                       f"float64 NumPy, per-head K/V materialised)"}
+
+
+def cpu_workloads(rows: int = 96) -> dict:
+    """The oracle on a bounded sample of each other workload: `rows` query tokens (all heads,
+    all keys) of one attention call, window filled beforehand (not timed)."""
+    import numpy as np
+
+    import mla_synth
+    from oracle import OracleLayer
+    res = {}
+    for name in ("tiny", "wan_30l_w21_q3_wrap", "wan_b4_w21_q3", "wan_w63_q1"):
+        w = mla_synth.WORKLOADS[name]
+        dims = dict(w.dims)
+        dims.update(frame_h=w.frame_h, frame_w=w.frame_w, window_frames=w.window_frames)
+        orc = OracleLayer(dims, mla_synth.make_weights(dict(w.dims), mla_synth.weight_seed(w, 0)))
+        scales = mla_synth.stream_scales(w.batch, w.seed) if w.stream_scale else None
+        orc.append(mla_synth.make_hidden(w.batch, w.fill_frames * w.F, dims["hidden"],
+                                         mla_synth.fill_seed(w, 0), scales)[0])
+        x = mla_synth.make_hidden(w.batch, w.query_frames * w.F, dims["hidden"],
+                                  mla_synth.chunk_seed(w, 0, 0), scales)[0]
+        n = min(rows, x.shape[0])
+        sel = np.linspace(0, x.shape[0] - 1, n).astype(np.int64)
+        t0 = time.perf_counter()
+        orc.attention(x, rows=sel)
+        dt = time.perf_counter() - t0
+        keys = len(orc.active_frames()) * w.F + x.shape[0]
+        res[name] = {"value": round(n / dt, 3), "unit": UNIT, "seconds": round(dt, 2),
+                     "sample": f"{n} of {x.shape[0]} query tokens of one call (stream 0, all heads, {keys} keys)"}
+    return res
 
 
 def run_reference(args, rank, world):

@@ -26,13 +26,22 @@
  *    frame, tokens of a frame in row-major (h, w) order ([VideoMLA] App. C.1, S = F H W).
  *  - Positions are implicit: the i-th frame ever appended has temporal index t = i; a query
  *    chunk gets the indices the next append will use.  Token k of a frame sits at
- *    (h, w) = (k / frame_w, k % frame_w).
+ *    (h, w) = (k / frame_w, k % frame_w).  Angles are formed in fp32 from t, exact for
+ *    t < 2^24: an append or attention call that would reach frame index 2^24 returns
+ *    MLA_ERR_UNSUPPORTED (2^24 latent frames are days of video).
  *  - Calls are stream-ordered and asynchronous: append and attention make no host sync.
  *    `stream` is a cudaStream_t (NULL = legacy default stream).
  *  - Errors: arguments are validated on the host before anything is launched; a failed check
  *    returns MLA_ERR_INVALID_ARGUMENT / MLA_ERR_UNSUPPORTED / MLA_ERR_STATE and changes no
  *    state.  Kernels never trap: a device-side wait that runs out of time sets the cache's
  *    status word, which mla_cache_sync() returns as MLA_ERR_DEVICE_TIMEOUT.
+ *  - Range: the cache planes (c_kv, k_rope), the absorbed queries, P and o_lat are fp16
+ *    internally (16-bit like the paper's bf16/fp16 cache, [VideoMLA] §1; fp16 keeps three more
+ *    mantissa bits, bf16 more exponent range).  A projected value whose magnitude exceeds
+ *    65504 (the fp16 maximum) is clamped to +-65504; the kernel records it and computes on,
+ *    and the next mla_cache_sync() returns MLA_ERR_RANGE once.  P is bounded by 256 and o_lat
+ *    by the largest cached |c_kv|, so only the projections can clamp.  Hidden states and
+ *    weights stay bf16, out is bf16.
  *  - Threading: a cache may be used by one host thread and one stream at a time.
  */
 #ifndef MLA_LATENT_WINDOW_H
@@ -54,7 +63,8 @@ typedef enum {
   MLA_ERR_OUT_OF_MEMORY = 3,    /* cudaMalloc failed                                 */
   MLA_ERR_CUDA = 4,             /* a CUDA runtime call failed                        */
   MLA_ERR_DEVICE_TIMEOUT = 5,   /* a kernel's bounded wait ran out (status word)    */
-  MLA_ERR_STATE = 6             /* call not valid in the cache's current state      */
+  MLA_ERR_STATE = 6,            /* call not valid in the cache's current state      */
+  MLA_ERR_RANGE = 7             /* a value exceeded the fp16 range and was clamped   */
 } mla_status;
 
 /* The problem statement of one attention layer ([VideoMLA] §3, §4.1, App. D.1).
@@ -123,7 +133,8 @@ size_t mla_cache_device_bytes(const mla_config* cfg);
  * ([VideoMLA] §3.3 reconstructs per-head K/V from the latent through W_UK/W_UV; folding them
  * into the query and output projections is the standard MLA absorption), the RoPE tables and
  * a zeroed ring.  Synchronises `stream` once before returning, so the caller may free the
- * weights afterwards.  *out receives the handle (NULL on failure). */
+ * weights afterwards.  *out receives the handle (NULL on failure).  MLA_ERR_RANGE (and no
+ * cache) when an fp16 weight - W_OV, or the dense form's W_UK / W_UV - exceeds +-65504. */
 mla_status mla_cache_create(const mla_config* cfg, const mla_weights* w, void* stream,
                             mla_cache** out);
 
@@ -142,10 +153,25 @@ mla_status mla_cache_append(mla_cache* c, const void* x, int32_t n_frames, void*
  * frame index, which differs from the local one by a single offset for window and chunk
  * frames; for the sink keys the query's temporal RoPE bands are turned back by that offset.
  * The chunk's latents go to a scratch tail, not into the ring: call mla_cache_append with the
- * final hidden states to make them part of the window.  With an empty window (nothing
- * appended yet) the chunk attends to itself alone. */
+ * final hidden states, or mla_cache_commit when those are this call's x_chunk, to make them
+ * part of the window.  With an empty window (nothing appended yet) the chunk attends to itself
+ * alone. */
 mla_status mla_window_attention(mla_cache* c, const void* x_chunk, int32_t n_frames, void* out,
                                 void* stream);
+
+/* Append the chunk of the last attention call on this cache to the window, using the latents
+ * that call already computed: the same result as mla_cache_append(c, x_chunk, n_frames) with
+ * that call's x_chunk, without reading x_chunk again or recomputing c_kv and k_rope.  This is
+ * the rollout's last step of a chunk ([VideoMLA] App. D.4: denoise the chunk against the
+ * window, then append its latents) when the hidden states appended are the ones the last
+ * denoising step attended with.  The latents move from the chunk tail to the rows
+ * mla_ring_slot names (frames already in place are not copied; one small copy kernel per frame
+ * that moves).
+ *  - n_frames must equal the last attention call's n_frames (mla_window_attention, _noalloc or
+ *    _reconstruct), and no append or commit may have happened since; otherwise MLA_ERR_STATE
+ *    and nothing changes.
+ *  - Stream-ordered like mla_cache_append. */
+mla_status mla_cache_commit(mla_cache* c, int32_t n_frames, void* stream);
 
 /* Same computation and result as mla_window_attention, for callers that must not allocate
  * device memory while they run: code whose device memory belongs to a pooled or budgeted
@@ -161,7 +187,11 @@ mla_status mla_window_attention(mla_cache* c, const void* x_chunk, int32_t n_fra
  *  - Limit: batch * n_frames * F * n_heads * 832 bytes (plus 256 for alignment) must fit in
  *    32 MiB, else MLA_ERR_INVALID_ARGUMENT with the required size in mla_last_error().
  *  - The first call on a device looks up the array's device address (once per device, with
- *    the cache's device current); make that first call before any stream capture.
+ *    the cache's device current) and keeps it for the life of the process; make that first
+ *    call before any stream capture.  A device reset (cudaDeviceReset, or anything else that
+ *    destroys the device's primary context) invalidates that address together with every
+ *    cache on the device: do not call this entry point again in a process that has reset the
+ *    device while the library was loaded.
  *  - Every call on a device shares the one array and leaves the last call's contents in it.
  *    Nothing in it has to start at zero (each call writes every row it reads back), but calls
  *    whose kernels overlap on the GPU (other streams, other caches) race on it: serialise them.
@@ -212,7 +242,8 @@ mla_status mla_dense_split_plan(int32_t batch, int32_t n_q, int32_t n_kv, int32_
  * `stream` completes; with mla_dense_workspace_bytes(...) bytes or more the keys are split
  * into ranges whose fp32 partials a second kernel merges (fewer ranges if it is smaller).
  * Device waits are bounded; a timeout is reported by mla_dense_sync (one status word per
- * device, shared by all dense calls). */
+ * device, shared by all dense calls, whose address the first call on a device looks up and
+ * keeps: a device reset invalidates it, as it invalidates every cache). */
 mla_status mla_dense_attention(const void* q, const void* k, const void* v, void* out,
                                int32_t batch, int32_t n_q, int32_t n_kv, int32_t n_heads,
                                int32_t d_head, float softmax_scale, void* workspace,
@@ -239,8 +270,9 @@ void mla_cache_destroy(mla_cache* c);
  * valid window frames (min(appended, sink_frames) + min(max(appended - sink_frames, 0), W)). */
 mla_status mla_cache_state(const mla_cache* c, int64_t* frames_appended, int32_t* valid_frames);
 
-/* Synchronise `stream` and return the device status word: MLA_OK, or the error a kernel
- * recorded (MLA_ERR_DEVICE_TIMEOUT).  Reading clears nothing. */
+/* Synchronise `stream` and return the device status: MLA_OK, or the fatal error a kernel
+ * recorded (MLA_ERR_DEVICE_TIMEOUT; it stays set), else MLA_ERR_RANGE when a projected value
+ * was clamped to the fp16 range since the previous sync (reported once, then cleared). */
 mla_status mla_cache_sync(mla_cache* c, void* stream);
 
 /* Copy stream b's cached planes to host memory, in physical row order (the rows mla_ring_slot
@@ -270,7 +302,7 @@ mla_status mla_cache_debug_buffers(const mla_cache* c, mla_debug_buffers* out);
 typedef enum {
   MLA_BUFFER_QP = 0,     /* Qp of the last attention call (fp16)   */
   MLA_BUFFER_O_LAT = 1,  /* o_lat of the last attention call (fp16) */
-  MLA_BUFFER_W_QCAT = 2, /* absorbed query + latent weights (bf16)  */
+  MLA_BUFFER_W_QCAT = 2, /* absorbed query + latent weights, rows [hi | lo] of 2 x hidden bf16 */
   MLA_BUFFER_W_OV = 3    /* absorbed output weights (fp16)          */
 } mla_buffer;
 mla_status mla_cache_copy_buffer(const mla_cache* c, mla_buffer which, void* host_dst, size_t bytes,

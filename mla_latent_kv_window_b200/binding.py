@@ -10,7 +10,8 @@ import ctypes
 import os
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(HERE, "libmla.so")
+# MLA_LIBRARY selects another build of the same library (the MLA_DEBUG build, libmla_debug.so).
+LIB_PATH = os.environ.get("MLA_LIBRARY") or os.path.join(HERE, "libmla.so")
 
 # mla_status values
 MLA_OK = 0
@@ -20,13 +21,15 @@ MLA_ERR_OUT_OF_MEMORY = 3
 MLA_ERR_CUDA = 4
 MLA_ERR_DEVICE_TIMEOUT = 5
 MLA_ERR_STATE = 6
+MLA_ERR_RANGE = 7
 
 MLA_KERNEL_APPEND, MLA_KERNEL_QPROJ, MLA_KERNEL_ATTENTION, MLA_KERNEL_OPROJ = range(4)
 KERNEL_NAMES = ("append", "qproj", "attention", "oproj")
 
 EXPORTED = (
     "mla_config_check", "mla_ring_slot", "mla_ring_bytes", "mla_cache_device_bytes",
-    "mla_cache_create", "mla_cache_append", "mla_window_attention", "mla_window_attention_noalloc",
+    "mla_cache_create", "mla_cache_append", "mla_cache_commit", "mla_window_attention",
+    "mla_window_attention_noalloc",
     "mla_window_attention_reconstruct", "mla_cache_selftest_timeout",
     "mla_cache_destroy", "mla_dense_split_plan", "mla_dense_workspace_bytes", "mla_dense_attention",
     "mla_dense_sync",
@@ -86,6 +89,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "mla_cache_device_bytes": (ctypes.c_size_t, [P(mla_config)]),
         "mla_cache_create": (I32, [P(mla_config), P(mla_weights), VP, P(VP)]),
         "mla_cache_append": (I32, [VP, VP, I32, VP]),
+        "mla_cache_commit": (I32, [VP, I32, VP]),
         "mla_window_attention": (I32, [VP, VP, I32, VP, VP]),
         "mla_window_attention_noalloc": (I32, [VP, VP, I32, VP, VP]),
         "mla_window_attention_reconstruct": (I32, [VP, VP, I32, VP, VP]),
@@ -181,6 +185,10 @@ def mla_cache_create(cfg: mla_config, weights: dict, stream=None) -> int:
 def mla_cache_append(cache: int, x, n_frames: int, stream=None) -> None:
     _check(load_library().mla_cache_append(cache, _dev_ptr(x, "x"), n_frames, _stream_handle(stream)),
            "mla_cache_append")
+
+
+def mla_cache_commit(cache: int, n_frames: int, stream=None) -> None:
+    _check(load_library().mla_cache_commit(cache, n_frames, _stream_handle(stream)), "mla_cache_commit")
 
 
 def mla_window_attention(cache: int, x_chunk, n_frames: int, out, stream=None) -> None:
@@ -332,6 +340,9 @@ class LatentWindowCache:
 
     def append(self, x, stream=None) -> None:
         mla_cache_append(self.handle, x, self._frames(x, "x"), stream)
+
+    def commit(self, n_frames: int, stream=None) -> None:
+        mla_cache_commit(self.handle, n_frames, stream)
 
     def attention(self, x_chunk, out=None, stream=None):
         n = self._frames(x_chunk, "x_chunk")

@@ -2,6 +2,9 @@
 //
 //   D[m, n] = sum_k A[z][m, k] * B[n, k]    (A: [batch][M][K], B: [N][K], K-major, both bf16 or
 //                                            both fp16, fp32 accumulation)
+// With a_kwrap > 0, A has only a_kwrap columns and column k of the product reads A's column
+// k mod a_kwrap: D = A B_0^T + A B_1^T for B = [B_0 | B_1], the form of a weight carried as a
+// bf16 pair hi + lo (two bf16 products per element, one fp32 accumulator).
 //
 // Persistent: one CTA per SM walks the tiles t = blockIdx.x, blockIdx.x + gridDim.x, ... of a
 // (row tile, column block, batch) grid.  Each 128 x BN tile accumulates in fp32 tensor memory:
@@ -40,7 +43,9 @@
 //               map_o2 = k_rope (fp16), at rows dst_row0 + m of the cache planes (the host
 //               encodes the maps at the destination rows, so each launch writes one
 //               contiguous row range per stream).  The latent path is 16-bit like the paper's
-//               cache; fp16 keeps three more mantissa bits than bf16 for the same bytes.
+//               cache; fp16 keeps three more mantissa bits than bf16 for the same bytes.  A
+//               value beyond the fp16 range is clamped to +-65504 and sets the status block's
+//               range word (not fatal; mla_cache_sync reports it).
 //   RoPE applies to the chunks with col mod 224 == 192 (every 224-column block is 192 + 32).
 //   kEpiDense   bf16 to map_o0 at column (col / head_in) * head_out + col % head_in (identity
 //               when head_in == 0), with RoPE on the chunks where col mod rope_period ==
@@ -161,7 +166,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                    const __grid_constant__ CUtensorMap map_o0,
                    const __grid_constant__ CUtensorMap map_o1,
                    const __grid_constant__ CUtensorMap map_o2, int32_t M, int32_t K,
-                   int32_t b_row0, GemmTiles tiles, EpiArgs ep, int* status) {
+                   int32_t a_kwrap, int32_t b_row0, GemmTiles tiles, EpiArgs ep, int* status) {
   using L = GemmSmem<BN, A_STAGES, B_STAGES, M_SUB>;
   // B_STAGES == 0: one ring for A and B (one producer, one full/empty barrier pair per stage,
   // one wait and one commit per k-block); otherwise separate rings with their own producers.
@@ -247,8 +252,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           const int s = g % A_STAGES;
           if (!mbar_wait(&a_empty[s], ((uint32_t)(g / A_STAGES) & 1u) ^ 1u, status)) { ok = false; break; }
           const int kx = ((kb + rot) % num_kb) * 64;
+          const int kxa = a_kwrap > 0 && kx >= a_kwrap ? kx - a_kwrap : kx;
           mbar_arrive_expect_tx(&a_full[s], L::kABytes + L::kBBytes);
-          tma_load_3d_hint(smem + s * L::kABytes, &map_a, &a_full[s], kx, m0, z, pa);
+          tma_load_3d_hint(smem + s * L::kABytes, &map_a, &a_full[s], kxa, m0, z, pa);
           tma_load_3d_hint(smem + L::kBOffset + s * L::kBBytes, &map_b, &a_full[s], kx,
                            b_row0 + y * BN, 0, pb);
         }
@@ -281,7 +287,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           const int kx = ((kb + rot) % num_kb) * 64;
           mbar_arrive_expect_tx(&full[s], bytes);
           if (is_a)
-            tma_load_3d_hint(smem + s * L::kABytes, &map_a, &full[s], kx, m0, z, policy);
+            tma_load_3d_hint(smem + s * L::kABytes, &map_a, &full[s],
+                             a_kwrap > 0 && kx >= a_kwrap ? kx - a_kwrap : kx, m0, z, policy);
           else
             tma_load_3d_hint(smem + L::kBOffset + s * L::kBBytes, &map_b, &full[s], kx,
                              b_row0 + y * BN, 0, policy);
@@ -352,6 +359,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const uint32_t swz = (lane >> 1) & 3u;
     int issued = 0;                            // tensor stores issued by this warp (lane 0)
     float2 rf[16];                             // RoPE factors of this thread's row
+    float amax = 0.f;                          // largest |value| this thread packed to fp16
     for (int i = 0; i < my_tiles; ++i) {
       const int buf = i % kAccBufs;
       int m0t, y, z;
@@ -409,6 +417,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
             for (int q = 0; q < 32; ++q) v[q] *= ep.q_scale;
           }
+#pragma unroll
+          for (int q = 0; q < 32; ++q) amax = fmaxf(amax, fabsf(v[q]));
         }
         // Box issued % 2 is free once at most one later store is still reading.
         if (lane == 0) bulk_wait_read_1();
@@ -452,6 +462,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       // This thread has read all its accumulator columns of the tile.
       tc_fence_before();
       mbar_arrive(&acc_empty[buf]);
+    }
+    // fp16 packing saturates at +-65504 (cvt.satfinite): record that it happened.  Rows and
+    // columns past the launch's extent hold zeros (the loads zero-fill), so every value counts.
+    if constexpr (kEpi == kEpiLatent) {
+      if (__any_sync(0xffffffffu, !(amax <= kF16Max)) && lane == 0)
+        atomicOr(status + kStatusRangeWord, 1);
     }
     if (lane == 0) bulk_wait_all();
   }

@@ -66,6 +66,8 @@ struct TileShape {
 };
 constexpr TileShape kShapeQ224{224, 1, 0.333}, kShapeQ160W{160, 2, 0.468},
     kShapeQ224W{224, 2, 0.597}, kShapeL32{32, 1, 0.318};
+// Temporal positions are formed in fp32 from the integer frame index (exact below 2^24).
+constexpr int64_t kMaxFrames = int64_t(1) << 24;
 constexpr int kAttnStages = 4;      // 4 key tiles in flight (Q and P live in tensor memory)
 
 thread_local std::string g_last_error;
@@ -166,9 +168,12 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 }
 
 // ------------------------------------------------------------------------------ kernels
-// Create-time derivation of the absorbed weights (fp32 accumulation, one bf16 rounding).
-// Wqcat rows, per head h: [h*224, h*224+192) = W_UK[h]^T W_Q[h], [h*224+192, h*224+224) = W_QR[h];
-// then [n_h*224, n_h*224+192) = W_DKV and [n_h*224+192, (n_h+1)*224) = W_KR.
+// Create-time derivation of the absorbed weights (fp32 accumulation), stored as bf16 pairs:
+// row r of Wqcat is [hi | lo] (2 * hidden columns), hi = bf16(w), lo = bf16(w - hi).  Rows,
+// per head h: [h*224, h*224+192) = W_UK[h]^T W_Q[h], [h*224+192, h*224+224) = W_QR[h];
+// then [n_h*224, n_h*224+192) = W_DKV and [n_h*224+192, (n_h+1)*224) = W_KR.  The absorbed
+// product carried in one bf16 (8 significant bits) would perturb every score by about 2^-10
+// relative, which sharp softmaxes (large hidden states) turn into visible output errors.
 // With a low-rank query the head rows come precomposed in fp32: qabs_f32 [n_heads*192][hidden]
 // (W_UK[h]^T W_Q[h] W_DQ) and qr_f32 [n_heads*32][hidden] (W_QR W_DQ); w_q, w_qr, w_uk unused.
 __global__ void build_wqcat_kernel(const __nv_bfloat16* __restrict__ w_q,
@@ -203,7 +208,11 @@ __global__ void build_wqcat_kernel(const __nv_bfloat16* __restrict__ w_q,
     acc = c < kLatent ? __bfloat162float(w_dkv[(size_t)c * hidden + k])
                       : __bfloat162float(w_kr[(size_t)(c - kLatent) * hidden + k]);
   }
-  wqcat[(size_t)rowq * hidden + k] = __float2bfloat16_rn(acc);
+  // hi + lo: the weight to about 16 significant bits in two bf16 halves of the row (the lo half
+  // is zero where the weight is the caller's own bf16 value).
+  const __nv_bfloat16 hi = __float2bfloat16_rn(acc);
+  wqcat[(size_t)rowq * 2 * hidden + k] = hi;
+  wqcat[(size_t)rowq * 2 * hidden + hidden + k] = __float2bfloat16_rn(acc - __bfloat162float(hi));
 }
 
 // W_OV[o][h*192 + c] = sum_j W_O[o][h*d_head + j] * W_UV[h*d_head + j][c], stored fp16 (it
@@ -225,10 +234,18 @@ __global__ void compose_kernel(const TA* __restrict__ A, int64_t a_sz, int64_t a
   for (int k = 0; k < K; ++k) acc += (float)a[(int64_t)k * a_sk] * (float)b[(int64_t)k * b_sk];
   C[z * c_sz + (int64_t)m * N + n] = acc;
 }
+// fp32 -> fp16, clamped to +-65504; a clamp sets *range (the status block's range word).
+__device__ __forceinline__ __half to_f16_checked(float v, int* range) {
+  if (!(fabsf(v) <= mla::kF16Max)) {
+    atomicOr(range, 1);
+    v = fminf(fmaxf(v, -mla::kF16Max), mla::kF16Max);
+  }
+  return __float2half_rn(v);
+}
 __global__ void build_wov_kernel(const __nv_bfloat16* __restrict__ w_o,
                                  const __nv_bfloat16* __restrict__ w_uv,
                                  __half* __restrict__ wov, int hidden, int n_heads,
-                                 int d_head) {
+                                 int d_head, int* range) {
   const int col = blockIdx.x * blockDim.x + threadIdx.x;  // h*192 + c
   const int o = blockIdx.y;
   if (col >= n_heads * kLatent) return;
@@ -241,7 +258,7 @@ __global__ void build_wov_kernel(const __nv_bfloat16* __restrict__ w_o,
     acc += __bfloat162float(w_o[(size_t)o * in_o + r]) *
            __bfloat162float(w_uv[(size_t)r * kLatent + c]);
   }
-  wov[(size_t)o * (n_heads * kLatent) + col] = __float2half_rn(acc);
+  wov[(size_t)o * (n_heads * kLatent) + col] = to_f16_checked(acc, range);
 }
 
 template <typename K>
@@ -271,9 +288,9 @@ __global__ void build_wqd_kernel(const __nv_bfloat16* __restrict__ w_q,
   wqd[(size_t)row * hidden + k] = __float2bfloat16_rn(v);
 }
 __global__ void bf16_to_f16_kernel(const __nv_bfloat16* __restrict__ in, __half* __restrict__ out,
-                                   int64_t n) {
+                                   int64_t n, int* range) {
   const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (i < n) out[i] = __float2half_rn(__bfloat162float(in[i]));
+  if (i < n) out[i] = to_f16_checked(__bfloat162float(in[i]), range);
 }
 // k_rope of every key into the RoPE channels [d_nope, 128) of every head of the dense K:
 // kd[z][n][h][d_nope + r] = krope[z][n][r].
@@ -287,6 +304,32 @@ __global__ void krope_broadcast_kernel(const __half* __restrict__ krope, int64_t
   for (int i = threadIdx.x; i < n_heads * kRope; i += blockDim.x) {
     const int h = i / kRope, r = i % kRope;
     dst[h * 128 + r] = __float2bfloat16_rn(__half2float(src[r]));
+  }
+}
+
+// Move `rows` rows of both latent planes of every stream from src_row to dst_row (16-byte
+// pieces: 24 per c_kv row, 4 per k_rope row).  The two ranges never overlap (mla_cache_commit).
+__global__ void move_rows_kernel(__half* __restrict__ ckv, __half* __restrict__ krope,
+                                 int64_t rows_per_stream, int64_t src_row, int64_t dst_row,
+                                 int64_t rows, int* status) {
+  constexpr int kPieces = kLatent / 8 + kRope / 8;   // 16-byte pieces per row of both planes
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int z = blockIdx.y;
+  mla::grid_dependency_wait();
+  if (i >= rows * kPieces) return;
+  const int64_t r = i / kPieces;
+  const int u = (int)(i - r * kPieces);
+  if (!mla::in_bounds(src_row + r < rows_per_stream && dst_row + r < rows_per_stream && src_row >= 0 &&
+                      dst_row >= 0, status))
+    return;
+  if (u < kLatent / 8) {
+    const uint4* s = reinterpret_cast<const uint4*>(ckv + (z * rows_per_stream + src_row + r) * kLatent);
+    uint4* d = reinterpret_cast<uint4*>(ckv + (z * rows_per_stream + dst_row + r) * kLatent);
+    d[u] = s[u];
+  } else {
+    const uint4* s = reinterpret_cast<const uint4*>(krope + (z * rows_per_stream + src_row + r) * kRope);
+    uint4* d = reinterpret_cast<uint4*>(krope + (z * rows_per_stream + dst_row + r) * kRope);
+    d[u - kLatent / 8] = s[u - kLatent / 8];
   }
 }
 
@@ -313,14 +356,14 @@ template <int BN, int SA, int SB, int EPI, bool F16, int M_SUB = 1>
 mla_status launch_gemm(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& mo0,
                        const CUtensorMap& mo1, const CUtensorMap& mo2, int M, int K, int b_row0,
                        mla::GemmTiles tiles, const EpiArgs& ep, int* status, int num_sms,
-                       cudaStream_t st, const char* what) {
+                       cudaStream_t st, const char* what, int a_kwrap = 0) {
   const int n = tiles.count();
   if (n <= 0) return MLA_OK;
   const int grid = n < num_sms ? n : num_sms;
   const cudaError_t e = launch_pdl(mla::tc_gemm_kernel<BN, SA, SB, EPI, F16, M_SUB>, dim3(grid),
                                    dim3(mla::kGemmThreads),
                                    mla::GemmSmem<BN, SA, SB, M_SUB>::kBytes, st, ma, mb, mo0, mo1,
-                                   mo2, M, K, b_row0, tiles, ep, status);
+                                   mo2, M, K, a_kwrap, b_row0, tiles, ep, status);
   if (e != cudaSuccess) return fail(MLA_ERR_CUDA, "%s launch failed: %s", what, cudaGetErrorString(e));
   return check_launch(what);
 }
@@ -335,6 +378,10 @@ struct mla_cache {
   int64_t sink_rows = 0;           // sink region: sink_frames * F rounded up to 128 rows
   int64_t max_q_tokens = 0;        // max_chunk * F
   int64_t frames_appended = 0;
+  // Chunk of the last attention call whose latents sit in the chunk tail (mla_cache_commit):
+  // its frame count (0: none) and the frames_appended it was computed at.
+  int32_t pending_frames = 0;
+  int64_t pending_at = -1;
   float softmax_scale = 0.f;
   RopeBands rope{};
   int device = 0;
@@ -382,6 +429,12 @@ struct mla_cache {
 };
 
 namespace {
+
+// The last attention call's chunk latents are in the chunk tail (see mla_cache_commit).
+void set_pending(mla_cache* c, int32_t n_frames) {
+  c->pending_frames = n_frames;
+  c->pending_at = c->frames_appended;
+}
 
 // Valid sink frames (vs) and valid window frames (vw) of a cache: the first sink_frames frames
 // ever appended are the sink, the newest W of the others the window.
@@ -469,7 +522,11 @@ mla_status launch_latent_gemm(mla_cache* c, const void* x, int64_t rows, int64_t
                               __half* qp = nullptr, int64_t qp_tokens = 0) {
   const mla_config& cfg = c->cfg;
   const int n_cols = with_queries ? (cfg.n_heads + 1) * kQK : kQK;   // columns of this launch
-  const int num_kb = cfg.hidden / 64;
+  // With queries the absorbed weights' lo halves are multiplied too (K = 2 x hidden, A wraps);
+  // the latent-only launch reads the hi halves, which hold W_DKV and W_KR exactly.
+  const int K = with_queries ? 2 * cfg.hidden : cfg.hidden;
+  const int a_kwrap = with_queries ? cfg.hidden : 0;
+  const int num_kb = K / 64;
   // Pick the tile shape with the least estimated time (waves x k-blocks x k-block time).
   auto tiles_of = [&](const TileShape& t) {
     return mla::GemmTiles{(int32_t)((rows + 128 * t.m_sub - 1) / (128 * t.m_sub)),
@@ -525,19 +582,19 @@ mla_status launch_latent_gemm(mla_cache* c, const void* x, int64_t rows, int64_t
   const char* what = "latent projection";
   if (shape.bn == 32)
     return launch_gemm<32, kProjNarrowAStages, kProjNarrowBStages, mla::kEpiLatent, false, 1>(
-        map_x, c->map_wqcat32, map_qp, map_ckv, map_krope, (int)rows, cfg.hidden, b_row0, tiles,
-        ep, c->status, c->num_sms, st, what);
+        map_x, c->map_wqcat32, map_qp, map_ckv, map_krope, (int)rows, K, b_row0, tiles,
+        ep, c->status, c->num_sms, st, what, a_kwrap);
   if (shape.bn == 160)
     return launch_gemm<160, kProjMidAStages, kProjMidBStages, mla::kEpiLatent, false, 2>(
-        map_x, c->map_wqcat160, map_qp, map_ckv, map_krope, (int)rows, cfg.hidden, b_row0, tiles,
-        ep, c->status, c->num_sms, st, what);
+        map_x, c->map_wqcat160, map_qp, map_ckv, map_krope, (int)rows, K, b_row0, tiles,
+        ep, c->status, c->num_sms, st, what, a_kwrap);
   if (shape.m_sub == 2)
     return launch_gemm<kQK, kProjWideAStages, kProjWideBStages, mla::kEpiLatent, false, 2>(
-        map_x, c->map_wqcat, map_qp, map_ckv, map_krope, (int)rows, cfg.hidden, b_row0, tiles,
-        ep, c->status, c->num_sms, st, what);
+        map_x, c->map_wqcat, map_qp, map_ckv, map_krope, (int)rows, K, b_row0, tiles,
+        ep, c->status, c->num_sms, st, what, a_kwrap);
   return launch_gemm<kQK, kProjAStages, kProjBStages, mla::kEpiLatent, false, 1>(
-      map_x, c->map_wqcat, map_qp, map_ckv, map_krope, (int)rows, cfg.hidden, b_row0, tiles, ep,
-      c->status, c->num_sms, st, what);
+      map_x, c->map_wqcat, map_qp, map_ckv, map_krope, (int)rows, K, b_row0, tiles, ep,
+      c->status, c->num_sms, st, what, a_kwrap);
 }
 
 // Output projection out[z][m][:] = o_lat[z][m][:] W_OV^T over nq tokens per stream.
@@ -584,6 +641,10 @@ mla_status launch_attention(mla_cache* c, const __half* qp, int64_t qp_batch_str
   a.n_keys = (int32_t)n_keys;
   a.o_lat = o_lat;
   a.o_lat_batch_stride = o_lat_batch_stride;
+  // Capacity of the row buffers (debug bounds checks): both hold the same rows per stream.
+  a.qp_rows_cap = qp_batch_stride / kQK < o_lat_batch_stride / kLatent ? qp_batch_stride / kQK
+                                                                         : o_lat_batch_stride / kLatent;
+  a.batch = cfg.batch;
   // Sink keys (rows [0, sink_rows), valid below vs * F) are stored rotated at their absolute
   // frame index, which is also their window-local one; the queries (rotated at absolute t) must
   // meet them at their local t = absolute t + delta, delta = (vs + vw) - frames_appended: turn
@@ -617,11 +678,12 @@ mla_status launch_attention(mla_cache* c, const __half* qp, int64_t qp_batch_str
 // attention output (o_lat) of one call, in a fixed per-device array instead of cache-owned
 // buffers.  Every GPU that loads this library holds these 32 MiB until the process exits.
 constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;
+// Per-device tables of looked-up device addresses (the no-alloc scratch, the dense status word).
+constexpr int kMaxDevices = 64;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
 namespace {
 
-constexpr int kMaxDevices = 64;
 std::mutex g_noalloc_mu;
 void* g_noalloc_ptr[kMaxDevices] = {};
 
@@ -657,12 +719,12 @@ namespace {
 
 constexpr int kDenseStages = 3;
 std::mutex g_dense_mu;
-int* g_dense_status_ptr[64] = {};
+int* g_dense_status_ptr[kMaxDevices] = {};
 
 mla_status dense_status_word(int** out) {
   int dev = 0;
   MLA_CUDA(cudaGetDevice(&dev));
-  if (dev < 0 || dev >= 64) return fail(MLA_ERR_UNSUPPORTED, "device index %d too large", dev);
+  if (dev < 0 || dev >= kMaxDevices) return fail(MLA_ERR_UNSUPPORTED, "device index %d too large", dev);
   std::lock_guard<std::mutex> lock(g_dense_mu);
   if (!g_dense_status_ptr[dev]) {
     void* p = nullptr;
@@ -786,6 +848,7 @@ const char* mla_status_string(mla_status s) {
     case MLA_ERR_CUDA: return "MLA_ERR_CUDA";
     case MLA_ERR_DEVICE_TIMEOUT: return "MLA_ERR_DEVICE_TIMEOUT";
     case MLA_ERR_STATE: return "MLA_ERR_STATE";
+    case MLA_ERR_RANGE: return "MLA_ERR_RANGE";
   }
   return "MLA_ERR_UNKNOWN";
 }
@@ -861,7 +924,7 @@ size_t mla_cache_device_bytes(const mla_config* cfg) {
   b += (size_t)c.batch * rows * kQK * 2;                   // ckv + krope (ring + chunk tail)
   b += (size_t)c.batch * q * c.n_heads * kQK * 2;          // Qp
   b += (size_t)c.batch * q * c.n_heads * kLatent * 2;      // o_lat
-  b += (size_t)(c.n_heads + 1) * kQK * c.hidden * 2;       // Wqcat
+  b += (size_t)(c.n_heads + 1) * kQK * c.hidden * 4;       // Wqcat (bf16 hi + lo)
   b += (size_t)c.hidden * c.n_heads * kLatent * 2;         // W_OV
   b += 256;                                                // status word
   b += (size_t)(c.frame_h + c.frame_w) * 16 * 8;           // RoPE h / w tables
@@ -945,7 +1008,7 @@ mla_status mla_cache_create(const mla_config* cfg, const mla_weights* w, void* s
   MLA_TRY(cudaMalloc(&c->krope, ring_rows * kRope * 2));
   MLA_TRY(cudaMalloc(&c->qp, q_rows * k.n_heads * kQK * 2));
   MLA_TRY(cudaMalloc(&c->o_lat, q_rows * k.n_heads * kLatent * 2));
-  MLA_TRY(cudaMalloc(&c->wqcat, (size_t)(k.n_heads + 1) * kQK * k.hidden * 2));
+  MLA_TRY(cudaMalloc(&c->wqcat, (size_t)(k.n_heads + 1) * kQK * 2 * k.hidden * 2));
   MLA_TRY(cudaMalloc(&c->wov, (size_t)k.hidden * k.n_heads * kLatent * 2));
   MLA_TRY(cudaMalloc(&c->status, 256));
   const std::vector<float2> rope_hw = make_rope_hw(k);
@@ -1000,7 +1063,7 @@ mla_status mla_cache_create(const mla_config* cfg, const mla_weights* w, void* s
     dim3 g2((k.n_heads * kLatent + 255) / 256, k.hidden);
     build_wov_kernel<<<g2, 256, 0, st>>>((const __nv_bfloat16*)w->w_o,
                                          (const __nv_bfloat16*)w->w_uv, c->wov, k.hidden,
-                                         k.n_heads, k.d_head);
+                                         k.n_heads, k.d_head, c->status + mla::kStatusRangeWord);
     MLA_TRY(cudaGetLastError());
   }
   // Weights of the reconstruct-then-dense form (training-time layout, [VideoMLA] §3.3).
@@ -1027,9 +1090,9 @@ mla_status mla_cache_create(const mla_config* cfg, const mla_weights* w, void* s
     MLA_TRY(cudaGetLastError());
     const int64_t n_uk = (int64_t)nh * dn * kLatent, n_uv = (int64_t)nh * 128 * kLatent;
     bf16_to_f16_kernel<<<(unsigned)((n_uk + 255) / 256), 256, 0, st>>>(
-        (const __nv_bfloat16*)w->w_uk, c->wukh, n_uk);
+        (const __nv_bfloat16*)w->w_uk, c->wukh, n_uk, c->status + mla::kStatusRangeWord);
     bf16_to_f16_kernel<<<(unsigned)((n_uv + 255) / 256), 256, 0, st>>>(
-        (const __nv_bfloat16*)w->w_uv, c->wuvh, n_uv);
+        (const __nv_bfloat16*)w->w_uv, c->wuvh, n_uv, c->status + mla::kStatusRangeWord);
     MLA_TRY(cudaGetLastError());
     MLA_TRY(cudaMemcpyAsync(c->wo, w->w_o, (size_t)k.hidden * nh * 128 * 2,
                             cudaMemcpyDeviceToDevice, st));
@@ -1045,16 +1108,16 @@ mla_status mla_cache_create(const mla_config* cfg, const mla_weights* w, void* s
                       qd_cols * k.hidden * 2, 64, kOutBN, CU_TENSOR_MAP_SWIZZLE_128B)) != MLA_OK)
       return cleanup(s);
   }
-  s = make_map(&c->map_wqcat, c->wqcat, k.hidden, (uint64_t)(k.n_heads + 1) * kQK, 1,
-               (uint64_t)k.hidden * 2, (uint64_t)(k.n_heads + 1) * kQK * k.hidden * 2, 64, kQK,
+  s = make_map(&c->map_wqcat, c->wqcat, 2 * (uint64_t)k.hidden, (uint64_t)(k.n_heads + 1) * kQK, 1,
+               (uint64_t)k.hidden * 4, (uint64_t)(k.n_heads + 1) * kQK * k.hidden * 4, 64, kQK,
                CU_TENSOR_MAP_SWIZZLE_128B);
   if (s != MLA_OK) return cleanup(s);
-  s = make_map(&c->map_wqcat160, c->wqcat, k.hidden, (uint64_t)(k.n_heads + 1) * kQK, 1,
-               (uint64_t)k.hidden * 2, (uint64_t)(k.n_heads + 1) * kQK * k.hidden * 2, 64, 160,
+  s = make_map(&c->map_wqcat160, c->wqcat, 2 * (uint64_t)k.hidden, (uint64_t)(k.n_heads + 1) * kQK, 1,
+               (uint64_t)k.hidden * 4, (uint64_t)(k.n_heads + 1) * kQK * k.hidden * 4, 64, 160,
                CU_TENSOR_MAP_SWIZZLE_128B);
   if (s != MLA_OK) return cleanup(s);
-  s = make_map(&c->map_wqcat32, c->wqcat, k.hidden, (uint64_t)(k.n_heads + 1) * kQK, 1,
-               (uint64_t)k.hidden * 2, (uint64_t)(k.n_heads + 1) * kQK * k.hidden * 2, 64, 32,
+  s = make_map(&c->map_wqcat32, c->wqcat, 2 * (uint64_t)k.hidden, (uint64_t)(k.n_heads + 1) * kQK, 1,
+               (uint64_t)k.hidden * 4, (uint64_t)(k.n_heads + 1) * kQK * k.hidden * 4, 64, 32,
                CU_TENSOR_MAP_SWIZZLE_128B);
   if (s != MLA_OK) return cleanup(s);
   s = make_map(&c->map_wov, c->wov, (uint64_t)k.n_heads * kLatent, k.hidden, 1,
@@ -1098,6 +1161,14 @@ mla_status mla_cache_create(const mla_config* cfg, const mla_weights* w, void* s
   if (attr_status != MLA_OK) return cleanup(attr_status);
 
   MLA_TRY(cudaStreamSynchronize(st));
+  {
+    // The fp16 weights (W_OV, and the dense form's W_UK, W_UV) must fit the fp16 range.
+    int range = 0;
+    MLA_TRY(cudaMemcpy(&range, c->status + mla::kStatusRangeWord, sizeof(int), cudaMemcpyDeviceToHost));
+    if (range != 0)
+      return cleanup(fail(MLA_ERR_RANGE, "an fp16 weight (W_OV = W_O W_UV per head, or W_UK / W_UV) "
+                                         "exceeds the fp16 range +-65504"));
+  }
 #undef MLA_TRY
   *out = c;
   return MLA_OK;
@@ -1109,6 +1180,9 @@ mla_status mla_cache_append(mla_cache* c, const void* x, int32_t n_frames, void*
   if (!aligned16(x)) return fail(MLA_ERR_INVALID_ARGUMENT, "x must be 16-byte aligned");
   if ((int64_t)n_frames * c->F > ((int64_t)1 << 30))
     return fail(MLA_ERR_INVALID_ARGUMENT, "too many frames in one append");
+  if (c->frames_appended + n_frames > kMaxFrames)
+    return fail(MLA_ERR_UNSUPPORTED, "temporal index would pass 2^24 frames (RoPE angles are formed "
+                                     "in fp32 from the frame index, exact below 2^24)");
   const mla_config& cfg = c->cfg;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const int64_t S = cfg.sink_frames, W = cfg.window_frames;
@@ -1147,6 +1221,52 @@ mla_status mla_cache_append(mla_cache* c, const void* x, int32_t n_frames, void*
   }
   if (s != MLA_OK) return s;
   c->frames_appended += n_frames;
+  c->pending_frames = 0;
+  return MLA_OK;
+}
+
+mla_status mla_cache_commit(mla_cache* c, int32_t n_frames, void* stream) {
+  if (!c) return fail(MLA_ERR_INVALID_ARGUMENT, "NULL cache");
+  if (c->pending_frames == 0 || c->pending_at != c->frames_appended)
+    return fail(MLA_ERR_STATE, "no attention chunk to commit (no attention call since the last "
+                               "append or commit)");
+  if (n_frames != c->pending_frames)
+    return fail(MLA_ERR_STATE, "n_frames %d differs from the last attention call's %d", n_frames,
+                c->pending_frames);
+  const mla_config& cfg = c->cfg;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t S = cfg.sink_frames, W = cfg.window_frames, F = c->F;
+  int64_t vs, vw;
+  valid_counts(c, vs, vw);
+  const int64_t base_row = c->sink_rows + vw * F;   // where the attention call put the chunk
+  const int64_t A = c->frames_appended;
+  // Non-sink frames of the chunk that survive: the last W of them.
+  const int64_t first_sink_free = A < S ? (S - A < n_frames ? S - A : n_frames) : 0;
+  const int64_t n_window = n_frames - first_sink_free;
+  const int64_t skip = n_window > W ? n_window - W : 0;
+  {
+    ProfScope p(c, MLA_KERNEL_APPEND, st);
+    // In chunk order: a frame's destination can be the source of an earlier frame of the same
+    // chunk (sink frames fill up first), never of a later one, so frame-by-frame launches in
+    // this order read every source before it is overwritten.
+    for (int64_t i = 0; i < n_frames; ++i) {
+      if (i >= first_sink_free && i - first_sink_free < skip) continue;   // evicted in the chunk
+      const int64_t t = A + i;
+      const int64_t dst = t < S ? t * F : c->sink_rows + ((t - S) % W) * F;
+      const int64_t src = base_row + i * F;
+      if (dst == src) continue;
+      const int64_t work = F * (kLatent / 8 + kRope / 8);
+      dim3 grid((unsigned)((work + 255) / 256), (unsigned)cfg.batch);
+      const cudaError_t e = launch_pdl(move_rows_kernel, grid, dim3(256), 0, st, c->ckv, c->krope,
+                                       (int64_t)c->rows_per_stream, src, dst, F, c->status);
+      if (e != cudaSuccess)
+        return fail(MLA_ERR_CUDA, "commit copy launch failed: %s", cudaGetErrorString(e));
+      const mla_status s = check_launch("commit copy");
+      if (s != MLA_OK) return s;
+    }
+  }
+  c->frames_appended += n_frames;
+  c->pending_frames = 0;
   return MLA_OK;
 }
 
@@ -1159,6 +1279,8 @@ mla_status mla_window_attention(mla_cache* c, const void* x_chunk, int32_t n_fra
                 cfg.max_chunk_frames);
   if (!aligned16(x_chunk) || !aligned16(out))
     return fail(MLA_ERR_INVALID_ARGUMENT, "x_chunk and out must be 16-byte aligned");
+  if (c->frames_appended + n_frames > kMaxFrames)
+    return fail(MLA_ERR_UNSUPPORTED, "temporal index of the chunk would pass 2^24 frames");
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const int64_t nq = (int64_t)n_frames * c->F;
   int64_t vs, vw;
@@ -1188,6 +1310,7 @@ mla_status mla_window_attention(mla_cache* c, const void* x_chunk, int32_t n_fra
     ProfScope p(c, MLA_KERNEL_OPROJ, st);
     s = launch_out_proj(c, c->o_lat, c->max_q_tokens, nq, out, st, "output projection");
   }
+  if (s == MLA_OK) set_pending(c, n_frames);
   return s;
 }
 
@@ -1200,6 +1323,8 @@ mla_status mla_window_attention_noalloc(mla_cache* c, const void* x_chunk, int32
                 cfg.max_chunk_frames);
   if (!aligned16(x_chunk) || !aligned16(out))
     return fail(MLA_ERR_INVALID_ARGUMENT, "x_chunk and out must be 16-byte aligned");
+  if (c->frames_appended + n_frames > kMaxFrames)
+    return fail(MLA_ERR_UNSUPPORTED, "temporal index of the chunk would pass 2^24 frames");
   const int64_t nq = (int64_t)n_frames * c->F;
   const int64_t R = nq * cfg.n_heads;                    // Qp / o_lat rows per stream
   const size_t qp_bytes = align256((size_t)cfg.batch * R * kQK * 2);
@@ -1234,7 +1359,9 @@ mla_status mla_window_attention_noalloc(mla_cache* c, const void* x_chunk, int32
   if ((s = launch_attention(c, qp, R * kQK, R, n_keys, o_lat, R * kLatent, st, false)) != MLA_OK)
     return s;
   // 3. output projection from the scratch o_lat
-  return launch_out_proj(c, o_lat, nq, nq, out, st, "no-alloc output projection");
+  s = launch_out_proj(c, o_lat, nq, nq, out, st, "no-alloc output projection");
+  if (s == MLA_OK) set_pending(c, n_frames);
+  return s;
 }
 
 mla_status mla_window_attention_reconstruct(mla_cache* c, const void* x_chunk, int32_t n_frames,
@@ -1250,6 +1377,8 @@ mla_status mla_window_attention_reconstruct(mla_cache* c, const void* x_chunk, i
                 cfg.max_chunk_frames);
   if (!aligned16(x_chunk) || !aligned16(out))
     return fail(MLA_ERR_INVALID_ARGUMENT, "x_chunk and out must be 16-byte aligned");
+  if (c->frames_appended + n_frames > kMaxFrames)
+    return fail(MLA_ERR_UNSUPPORTED, "temporal index of the chunk would pass 2^24 frames");
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const int nh = cfg.n_heads, dn = cfg.d_nope;
   const uint64_t hd = (uint64_t)nh * 128;                 // dense row: n_h heads x 128
@@ -1358,9 +1487,11 @@ mla_status mla_window_attention_reconstruct(mla_cache* c, const void* x_chunk, i
     EpiArgs ep{};
     ep.n_cols = cfg.hidden;
     const mla::GemmTiles tiles{(int32_t)((nq + 127) / 128), (cfg.hidden + kOutBN - 1) / kOutBN, cfg.batch};
-    return launch_gemm<kOutBN, kOutAStages, kOutBStages, mla::kEpiStore, false>(
+    s = launch_gemm<kOutBN, kOutAStages, kOutBStages, mla::kEpiStore, false>(
         ma, c->map_wo, mo, mo, mo, (int)nq, (int)hd, 0, tiles, ep, c->status, c->num_sms, st,
         "dense output projection");
+    if (s == MLA_OK) set_pending(c, n_frames);
+    return s;
   }
 }
 
@@ -1453,10 +1584,18 @@ mla_status mla_cache_state(const mla_cache* c, int64_t* frames_appended, int32_t
 
 mla_status mla_cache_sync(mla_cache* c, void* stream) {
   if (!c) return fail(MLA_ERR_INVALID_ARGUMENT, "NULL cache");
-  MLA_CUDA(cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)));
-  int word = 0;
-  MLA_CUDA(cudaMemcpy(&word, c->status, sizeof(int), cudaMemcpyDeviceToHost));
-  if (word != 0) return fail((mla_status)word, "a kernel recorded device status %d", word);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  MLA_CUDA(cudaStreamSynchronize(st));
+  int words[mla::kStatusRangeWord + 1] = {0};
+  MLA_CUDA(cudaMemcpy(words, c->status, sizeof(words), cudaMemcpyDeviceToHost));
+  if (words[0] != 0) return fail((mla_status)words[0], "a kernel recorded device status %d", words[0]);
+  if (words[mla::kStatusRangeWord] != 0) {
+    // Reported once: clear the word so that the next sync covers the calls made after this one.
+    MLA_CUDA(cudaMemsetAsync(c->status + mla::kStatusRangeWord, 0, sizeof(int), st));
+    MLA_CUDA(cudaStreamSynchronize(st));
+    return fail(MLA_ERR_RANGE, "a projected value exceeded the fp16 range and was clamped to "
+                               "+-65504 (cache planes or absorbed queries) since the last sync");
+  }
   return MLA_OK;
 }
 
@@ -1501,7 +1640,7 @@ mla_status mla_cache_copy_buffer(const mla_cache* c, mla_buffer which, void* hos
   switch (which) {
     case MLA_BUFFER_QP: src = c->qp; total = q_rows * kQK * 2; break;
     case MLA_BUFFER_O_LAT: src = c->o_lat; total = q_rows * kLatent * 2; break;
-    case MLA_BUFFER_W_QCAT: src = c->wqcat; total = (size_t)(k.n_heads + 1) * kQK * k.hidden * 2; break;
+    case MLA_BUFFER_W_QCAT: src = c->wqcat; total = (size_t)(k.n_heads + 1) * kQK * k.hidden * 4; break;
     case MLA_BUFFER_W_OV: src = c->wov; total = (size_t)k.hidden * k.n_heads * kLatent * 2; break;
     default: return fail(MLA_ERR_INVALID_ARGUMENT, "unknown buffer %d", (int)which);
   }

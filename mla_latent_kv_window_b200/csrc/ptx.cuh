@@ -15,6 +15,26 @@ namespace mla {
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s per wait
 constexpr int kStatusTimeout = 5;                  // == MLA_ERR_DEVICE_TIMEOUT
+// Words of a cache's 256-byte status block: [0] the first fatal error (a wait that ran out;
+// every bounded wait gives up once it is set), [1] the timeout self-test's flag, [2] set when
+// a value converted to 16-bit float exceeded the fp16 range (+-65504) and was clamped - not
+// fatal: the kernels run on and mla_cache_sync reports it.
+constexpr int kStatusRangeWord = 2;
+constexpr float kF16Max = 65504.f;
+constexpr int kStatusBounds = 8;                   // == MLA_ERR_BOUNDS
+
+// Bounds checks of the MLA_DEBUG build: in_bounds(cond, status) is cond, and a false cond
+// records MLA_ERR_BOUNDS in the status word (first error wins) so that the caller skips the
+// access; in the normal build it is `true` and costs nothing.  Every plain (non-TMA) global
+// access whose index is computed in a kernel goes through it.
+#ifdef MLA_DEBUG
+__device__ __forceinline__ bool in_bounds(bool cond, int* status) {
+  if (!cond) atomicCAS(status, 0, kStatusBounds);
+  return cond;
+}
+#else
+__device__ __forceinline__ bool in_bounds(bool, int*) { return true; }
+#endif
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

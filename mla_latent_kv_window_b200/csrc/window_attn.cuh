@@ -79,6 +79,8 @@ struct AttnArgs {
   int32_t sink_tiles;          // leading key tiles that hold sink frames (0: no sink)
   int32_t sink_keys;           // valid sink keys; keys [sink_keys, 128 * sink_tiles) are padding
   float2 sink_rot[16];         // (cos, sin) turning each RoPE pair of Q for the sink keys
+  int64_t qp_rows_cap;         // rows each stream's Qp and o_lat buffers hold (bounds checks)
+  int32_t batch;               // streams the buffers hold (bounds checks)
 };
 
 template <int KV_STAGES>
@@ -231,7 +233,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const int gr = m0 + row;
       const uint4* src = reinterpret_cast<const uint4*>(args.qp + z * args.qp_batch_stride +
                                                         (int64_t)gr * 224);
-      const bool in = gr < args.rows;
+      const bool in = gr < args.rows && in_bounds(gr < args.qp_rows_cap && z < args.batch, status);
 #pragma unroll 1
       for (int c = 0; c < 4; ++c) {                // columns [32c, 32c + 32) of 112
         uint32_t q[32];
@@ -363,7 +365,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
       }
       const int gr = m0 + row;
-      if (gr < args.rows) {
+      if (gr < args.rows && in_bounds(gr < args.qp_rows_cap && z < args.batch, status)) {
         fence_proxy_async_smem();
         bulk_store(args.o_lat + z * args.o_lat_batch_stride + (int64_t)gr * 192, st_row, 384);
         bulk_commit();

@@ -227,10 +227,12 @@ def test_wan_w63_q1_full_size():
 def test_wan_30_layers_4_steps_wrapped():
     # 30 independent layers; each: append 24 frames (the ring wraps once, frames 3..23 stay), four
     # denoising steps with a fresh 3-frame chunk over the same window, then the step-4 chunk is
-    # appended.  The oracle checks sampled rows of layers 0 and 29 (steps 0 and 3); every layer's
-    # output must be finite and its status word clean.
+    # appended (even layers: mla_cache_append of its hidden states; odd layers: mla_cache_commit
+    # of the latents the last step computed).  The oracle checks 256 sampled rows at 8
+    # layer-steps spread over layers and steps; every layer's output must be finite and its
+    # status word clean.
     w = mla_synth.WORKLOADS["wan_30l_w21_q3_wrap"]
-    checked = {0: (0, 3), 29: (0, 3)}
+    checked = {0: (0, 3), 7: (1,), 13: (2,), 19: (1, 2), 29: (0, 3)}
     for layer in range(w.layers):
         p = Pair(w, layer=layer)
         oracle_on = layer in checked
@@ -240,11 +242,16 @@ def test_wan_30_layers_4_steps_wrapped():
         for step in range(w.steps):
             x = p.hidden(w.query_frames, mla_synth.chunk_seed(w, layer, step))
             if oracle_on and step in checked[layer]:
-                sampled_check(p, x, f"layer {layer} step {step}", 32, 100 * layer + step)
+                sampled_check(p, x, f"layer {layer} step {step}", 256, 100 * layer + step)
             else:
                 out = p.attention(x)
                 assert torch.isfinite(out.float()).all()
-        p.append(x, oracle=oracle_on)
+        if layer % 2:
+            p.gpu.commit(w.query_frames)
+            if oracle_on:
+                p.oracles[0].append(x[0])
+        else:
+            p.append(x, oracle=oracle_on)
         assert p.gpu.state() == (27, 21)
         if oracle_on:
             ckv, kr, _ = p.gpu.read_ring(0)
@@ -317,6 +324,31 @@ def test_sink_w6_q3_full_size():
         assert_close(kr[s0:s0 + w.F], r, f"k_rope frame {f}")
     sampled_check(p, p.hidden(3, mla_synth.chunk_seed(w, 0, 0)), "sink + 6-frame window", 64, 6)
 
+
+def test_sink_batched_scaled_streams():
+    # Two streams, each with its own sink frame, window and hidden-state scale in [0.5, 2]
+    # (sharper softmax for the larger one): every element after the window has slid.
+    w = mla_synth.Workload("sink_b2", frame_h=4, frame_w=6, window_frames=2, fill_frames=5,
+                           query_frames=2, batch=2, seed=21, sink_frames=1, stream_scale=True)
+    p = Pair(w, max_chunk_frames=2)
+    p.append(p.hidden(2, 730))
+    full_check(p, p.hidden(2, 731), "sink, 2 scaled streams, window filling")
+    p.append(p.hidden(3, 732))
+    check_ring(p, "sink, 2 scaled streams")
+    full_check(p, p.hidden(2, 733), "sink, 2 scaled streams, slid window")
+
+
+def test_sink_w6_q3_two_streams_sampled():
+    # The long-rollout configuration with B = 2 scaled streams: sampled rows of each stream.
+    base = mla_synth.WORKLOADS["sink_w6_q3"]
+    w = mla_synth.Workload("sink_w6_q3_b2", frame_h=base.frame_h, frame_w=base.frame_w,
+                           window_frames=base.window_frames, fill_frames=base.fill_frames,
+                           query_frames=base.query_frames, batch=2, seed=6100, sink_frames=1,
+                           stream_scale=True)
+    p = Pair(w)
+    p.append(p.hidden(w.fill_frames, mla_synth.fill_seed(w, 0)))
+    assert p.gpu.state() == (10, 7)
+    sampled_check(p, p.hidden(3, mla_synth.chunk_seed(w, 0, 0)), "sink + 6-frame window, B = 2", 64, 7)
 
 
 # ---------------------------------------------------------------------------- reconstruct-then-dense

@@ -158,8 +158,10 @@ def test_calls_validate_before_any_device_work():
     assert lib.mla_cache_append(None, None, 1, None) == B.MLA_ERR_INVALID_ARGUMENT
     assert lib.mla_window_attention(None, None, 1, None, None) == B.MLA_ERR_INVALID_ARGUMENT
     assert lib.mla_cache_sync(None, None) == B.MLA_ERR_INVALID_ARGUMENT
+    assert lib.mla_cache_commit(None, 1, None) == B.MLA_ERR_INVALID_ARGUMENT
     lib.mla_cache_destroy(None)  # NULL-safe
     assert lib.mla_status_string(5) == b"MLA_ERR_DEVICE_TIMEOUT"
+    assert lib.mla_status_string(B.MLA_ERR_RANGE) == b"MLA_ERR_RANGE"
 
 
 def test_binding_checks_tensor_extents_before_calling():
