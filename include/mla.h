@@ -42,6 +42,12 @@
  *    and the next mla_cache_sync() returns MLA_ERR_RANGE once.  P is bounded by 256 and o_lat
  *    by the largest cached |c_kv|, so only the projections can clamp.  Hidden states and
  *    weights stay bf16, out is bf16.
+ *  - Debug build (libmla_debug.so, the same sources compiled with MLA_DEBUG): every plain
+ *    global access whose index a kernel computes is bounds-checked first (a violation skips the
+ *    access and records MLA_ERR_BOUNDS in the status word), the tensor maps over the library's
+ *    own buffers are checked against the buffers' extents on the host, and every device buffer
+ *    of a cache carries a 4 KiB guard band that mla_cache_sync checks (MLA_ERR_BOUNDS when a
+ *    kernel wrote into one).  A stand-in for a memory checker; same results, slower.
  *  - Threading: a cache may be used by one host thread and one stream at a time.
  */
 #ifndef MLA_LATENT_WINDOW_H
@@ -64,7 +70,8 @@ typedef enum {
   MLA_ERR_CUDA = 4,             /* a CUDA runtime call failed                        */
   MLA_ERR_DEVICE_TIMEOUT = 5,   /* a kernel's bounded wait ran out (status word)    */
   MLA_ERR_STATE = 6,            /* call not valid in the cache's current state      */
-  MLA_ERR_RANGE = 7             /* a value exceeded the fp16 range and was clamped   */
+  MLA_ERR_RANGE = 7,            /* a value exceeded the fp16 range and was clamped   */
+  MLA_ERR_BOUNDS = 8            /* debug build: an index or a guard band out of range */
 } mla_status;
 
 /* The problem statement of one attention layer ([VideoMLA] §3, §4.1, App. D.1).
@@ -263,6 +270,15 @@ mla_status mla_dense_sync(void* stream);
  * reporting without faulting a GPU. */
 mla_status mla_cache_selftest_timeout(mla_cache* c, void* stream, int32_t* gave_up);
 
+/* Diagnostic self-test of the debug build's bounds checks: launches the chunk-commit copy kernel
+ * with a row range that runs one row past the end of the cache's planes; the kernel's bounds
+ * check catches the out-of-range row before any access to it (the in-range row is copied onto
+ * itself), records MLA_ERR_BOUNDS and the kernel returns.  Synchronises `stream`; *caught
+ * receives 1 when the status word then holds MLA_ERR_BOUNDS.  The status word stays set: use a
+ * fresh cache afterwards.  MLA_ERR_UNSUPPORTED (and nothing launched) in the normal build,
+ * which has no bounds checks.  Not part of the method. */
+mla_status mla_cache_selftest_bounds(mla_cache* c, void* stream, int32_t* caught);
+
 /* Free everything the cache owns (synchronises the device first).  NULL-safe. */
 void mla_cache_destroy(mla_cache* c);
 
@@ -271,8 +287,10 @@ void mla_cache_destroy(mla_cache* c);
 mla_status mla_cache_state(const mla_cache* c, int64_t* frames_appended, int32_t* valid_frames);
 
 /* Synchronise `stream` and return the device status: MLA_OK, or the fatal error a kernel
- * recorded (MLA_ERR_DEVICE_TIMEOUT; it stays set), else MLA_ERR_RANGE when a projected value
- * was clamped to the fp16 range since the previous sync (reported once, then cleared). */
+ * recorded (MLA_ERR_DEVICE_TIMEOUT, or MLA_ERR_BOUNDS in the debug build; it stays set), else
+ * MLA_ERR_BOUNDS when (debug build) a guard band after one of the cache's buffers or after the
+ * allocation-free scratch was overwritten, else MLA_ERR_RANGE when a projected value was clamped
+ * to the fp16 range since the previous sync (reported once, then cleared). */
 mla_status mla_cache_sync(mla_cache* c, void* stream);
 
 /* Copy stream b's cached planes to host memory, in physical row order (the rows mla_ring_slot

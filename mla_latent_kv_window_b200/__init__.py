@@ -9,6 +9,7 @@ from .binding import (  # noqa: F401
     mla_cache_device_bytes, mla_cache_profile_enable, mla_cache_profile_read, mla_cache_read,
     mla_cache_state, mla_cache_sync, mla_config, mla_config_check, mla_ring_bytes, mla_ring_slot,
     mla_window_attention, mla_window_attention_noalloc, mla_dense_attention, mla_dense_sync,
+    mla_cache_selftest_timeout, mla_cache_selftest_bounds,
     mla_dense_workspace_bytes, MLA_OK, MLA_ERR_INVALID_ARGUMENT, MLA_ERR_UNSUPPORTED,
-    MLA_ERR_OUT_OF_MEMORY, MLA_ERR_CUDA, MLA_ERR_DEVICE_TIMEOUT, MLA_ERR_STATE, MLA_ERR_RANGE,
+    MLA_ERR_OUT_OF_MEMORY, MLA_ERR_CUDA, MLA_ERR_DEVICE_TIMEOUT, MLA_ERR_STATE, MLA_ERR_RANGE, MLA_ERR_BOUNDS,
 )

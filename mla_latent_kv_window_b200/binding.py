@@ -22,6 +22,7 @@ MLA_ERR_CUDA = 4
 MLA_ERR_DEVICE_TIMEOUT = 5
 MLA_ERR_STATE = 6
 MLA_ERR_RANGE = 7
+MLA_ERR_BOUNDS = 8
 
 MLA_KERNEL_APPEND, MLA_KERNEL_QPROJ, MLA_KERNEL_ATTENTION, MLA_KERNEL_OPROJ = range(4)
 KERNEL_NAMES = ("append", "qproj", "attention", "oproj")
@@ -30,7 +31,7 @@ EXPORTED = (
     "mla_config_check", "mla_ring_slot", "mla_ring_bytes", "mla_cache_device_bytes",
     "mla_cache_create", "mla_cache_append", "mla_cache_commit", "mla_window_attention",
     "mla_window_attention_noalloc",
-    "mla_window_attention_reconstruct", "mla_cache_selftest_timeout",
+    "mla_window_attention_reconstruct", "mla_cache_selftest_timeout", "mla_cache_selftest_bounds",
     "mla_cache_destroy", "mla_dense_split_plan", "mla_dense_workspace_bytes", "mla_dense_attention",
     "mla_dense_sync",
     "mla_cache_state", "mla_cache_sync", "mla_cache_read", "mla_cache_debug_buffers", "mla_cache_copy_buffer",
@@ -94,6 +95,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "mla_window_attention_noalloc": (I32, [VP, VP, I32, VP, VP]),
         "mla_window_attention_reconstruct": (I32, [VP, VP, I32, VP, VP]),
         "mla_cache_selftest_timeout": (I32, [VP, VP, P(I32)]),
+        "mla_cache_selftest_bounds": (I32, [VP, VP, P(I32)]),
         "mla_dense_split_plan": (I32, [I32, I32, I32, I32, I32, ctypes.c_size_t, P(I32), P(I32)]),
         "mla_dense_workspace_bytes": (ctypes.c_size_t, [I32, I32, I32, I32]),
         "mla_dense_attention": (I32, [VP, VP, VP, VP, I32, I32, I32, I32, I32, ctypes.c_float, VP,
@@ -217,6 +219,15 @@ def mla_cache_selftest_timeout(cache: int, stream=None) -> bool:
     flag = ctypes.c_int32()
     _check(load_library().mla_cache_selftest_timeout(cache, _stream_handle(stream), ctypes.byref(flag)),
            "mla_cache_selftest_timeout")
+    return flag.value == 1
+
+
+def mla_cache_selftest_bounds(cache: int, stream=None) -> bool:
+    """Run the debug build's bounds-check self-test; True when the kernel's check caught the
+    out-of-range row (raises MLAError with MLA_ERR_UNSUPPORTED on the normal build)."""
+    flag = ctypes.c_int32()
+    _check(load_library().mla_cache_selftest_bounds(cache, _stream_handle(stream), ctypes.byref(flag)),
+           "mla_cache_selftest_bounds")
     return flag.value == 1
 
 

@@ -48,6 +48,8 @@ struct DenseArgs {
   int32_t kv_per_split;  // keys per range (a multiple of 128)
   float* o_part;       // splits > 1: [splits][B][n_q][n_heads][128] unnormalised O
   float2* ml_part;     // splits > 1: [splits][B][n_q][n_heads] (max in log2 units, sum)
+  int64_t part_rows;   // rows the partials hold (splits x B x n_q x n_heads; bounds checks)
+  int32_t batch;       // streams (bounds checks)
 };
 
 template <int KV_STAGES>
@@ -266,7 +268,7 @@ __global__ void __launch_bounds__(kDenseThreads, 1)
         tmem_ld32(tmem_o + lane_off + cq * 32, o);
         tmem_ld_wait();
         tmem_regs_ready(o);
-        if (q < args.n_q) {
+        if (q < args.n_q && in_bounds(prow < args.part_rows, status)) {
           float4* dst = reinterpret_cast<float4*>(args.o_part + prow * 128 + cq * 32);
 #pragma unroll
           for (int v4 = 0; v4 < 8; ++v4)
@@ -274,7 +276,8 @@ __global__ void __launch_bounds__(kDenseThreads, 1)
                                   __uint_as_float(o[4 * v4 + 2]), __uint_as_float(o[4 * v4 + 3]));
         }
       }
-      if (q < args.n_q) args.ml_part[prow] = make_float2(m_used * c, l_sum);
+      if (q < args.n_q && in_bounds(prow < args.part_rows, status))
+        args.ml_part[prow] = make_float2(m_used * c, l_sum);
     } else if (ok && mbar_wait(pv_done, (uint32_t)(nt - 1) & 1u, status)) {
       tc_fence_after();
       const float inv_l = 1.f / l_sum;
@@ -299,7 +302,7 @@ __global__ void __launch_bounds__(kDenseThreads, 1)
       for (int rr = 0; rr < 32; rr += 2) {   // two rows per pass, 16 lanes x 16 bytes each
         const int trow = sub * 32 + rr + (lane >> 4);
         const int q = m0 + trow;
-        if (q < args.n_q) {
+        if (q < args.n_q && in_bounds(z < args.batch && h < args.n_heads, status)) {
           __nv_bfloat16* o = args.out + (((int64_t)z * args.n_q + q) * args.n_heads + h) * 128;
           reinterpret_cast<uint4*>(o)[lane & 15] =
               reinterpret_cast<const uint4*>(smem + L::kKV + trow * kStride)[lane & 15];
@@ -321,11 +324,13 @@ __global__ void __launch_bounds__(kDenseThreads, 1)
 // four of the 128 channels per lane.
 __global__ void dense_combine_kernel(const float* __restrict__ o_part,
                                      const float2* __restrict__ ml_part, int splits, int batch,
-                                     int n_q, int n_heads, __nv_bfloat16* __restrict__ out) {
+                                     int n_q, int n_heads, __nv_bfloat16* __restrict__ out,
+                                     int64_t part_rows, int* status) {
   const int64_t rows = (int64_t)batch * n_q * n_heads;
   const int64_t r = (int64_t)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (r >= rows) return;
+  if (!in_bounds((int64_t)(splits - 1) * rows + r < part_rows, status)) return;
   float mmax = -INFINITY;
   for (int s = 0; s < splits; ++s) mmax = fmaxf(mmax, ml_part[(int64_t)s * rows + r].x);
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);

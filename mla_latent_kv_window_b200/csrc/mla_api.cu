@@ -21,6 +21,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <algorithm>
 #include <mutex>
 #include <string>
 #include <utility>
@@ -68,6 +69,16 @@ constexpr TileShape kShapeQ224{224, 1, 0.333}, kShapeQ160W{160, 2, 0.468},
     kShapeQ224W{224, 2, 0.597}, kShapeL32{32, 1, 0.318};
 // Temporal positions are formed in fp32 from the integer frame index (exact below 2^24).
 constexpr int64_t kMaxFrames = int64_t(1) << 24;
+
+// Guard bands of the MLA_DEBUG build: every device buffer of a cache is allocated kGuardBytes
+// longer and the tail is filled with kGuardByte; mla_cache_sync checks that no kernel wrote
+// into it.  Zero in the normal build.
+#ifdef MLA_DEBUG
+constexpr size_t kGuardBytes = 4096;
+#else
+constexpr size_t kGuardBytes = 0;
+#endif
+constexpr unsigned char kGuardByte = 0xA5;
 constexpr int kAttnStages = 4;      // 4 key tiles in flight (Q and P live in tensor memory)
 
 thread_local std::string g_last_error;
@@ -296,9 +307,11 @@ __global__ void bf16_to_f16_kernel(const __nv_bfloat16* __restrict__ in, __half*
 // kd[z][n][h][d_nope + r] = krope[z][n][r].
 __global__ void krope_broadcast_kernel(const __half* __restrict__ krope, int64_t krope_stream_rows,
                                        __nv_bfloat16* __restrict__ kd, int n_keys, int n_heads,
-                                       int d_nope) {
+                                       int d_nope, int64_t kd_rows_cap, int* status) {
   const int n = blockIdx.x;
   const int z = blockIdx.y;
+  // kd rows are compact per call ([z][n]); the buffer holds kd_rows_cap of them.
+  if (!mla::in_bounds(n < krope_stream_rows && ((int64_t)z * n_keys + n) < kd_rows_cap, status)) return;
   const __half* src = krope + ((int64_t)z * krope_stream_rows + n) * kRope;
   __nv_bfloat16* dst = kd + ((int64_t)z * n_keys + n) * n_heads * 128 + d_nope;
   for (int i = threadIdx.x; i < n_heads * kRope; i += blockDim.x) {
@@ -417,6 +430,12 @@ struct mla_cache {
   CUtensorMap map_wqcat32{};       // ... and in 32-row boxes (32-column latent blocks)
   CUtensorMap map_wov{};           // B operand of the output projection: box 64 x 192
 
+  struct Guard {
+    const unsigned char* p;   // first guard byte (the buffer's end)
+    const char* name;
+  };
+  std::vector<Guard> guards;   // MLA_DEBUG build only
+
   bool profiling = false;
   struct Rec {
     int kind;
@@ -442,6 +461,41 @@ void valid_counts(const mla_cache* c, int64_t& vs, int64_t& vw) {
   const int64_t A = c->frames_appended, S = c->cfg.sink_frames, W = c->cfg.window_frames;
   vs = A < S ? A : S;
   vw = A - vs < W ? A - vs : W;
+}
+
+// cudaMalloc of a cache buffer; the MLA_DEBUG build adds a guard band after it (filled on
+// `st`) and records it for mla_cache_sync.
+template <typename T>
+cudaError_t alloc_buffer(mla_cache* c, T** p, size_t bytes, const char* name, cudaStream_t st) {
+  void* v = nullptr;
+  cudaError_t e = cudaMalloc(&v, bytes + kGuardBytes);
+  if (e != cudaSuccess) return e;
+  *p = static_cast<T*>(v);
+  if (kGuardBytes) {
+    unsigned char* g = static_cast<unsigned char*>(v) + bytes;
+    c->guards.push_back({g, name});
+    e = cudaMemsetAsync(g, kGuardByte, kGuardBytes, st);
+  }
+  return e;
+}
+
+// Host-side extent check of a tensor map over a buffer the library owns (MLA_DEBUG build):
+// the last byte the map can reach must lie inside [buf, buf + buf_bytes).
+mla_status check_extent(const void* base, uint64_t inner_bytes, uint64_t rows, uint64_t row_stride,
+                        uint64_t batch, uint64_t batch_stride, const void* buf, size_t buf_bytes,
+                        const char* what) {
+#ifdef MLA_DEBUG
+  const uintptr_t b0 = reinterpret_cast<uintptr_t>(buf), a = reinterpret_cast<uintptr_t>(base);
+  if (rows == 0 || batch == 0) return MLA_OK;
+  const uintptr_t last = a + (batch - 1) * batch_stride + (rows - 1) * row_stride + inner_bytes;
+  if (a < b0 || last > b0 + buf_bytes)
+    return fail(MLA_ERR_BOUNDS, "%s: tensor map reaches %zu bytes past its buffer", what,
+                (size_t)(last > b0 + buf_bytes ? last - (b0 + buf_bytes) : 0));
+#else
+  (void)base; (void)inner_bytes; (void)rows; (void)row_stride; (void)batch; (void)batch_stride;
+  (void)buf; (void)buf_bytes; (void)what;
+#endif
+  return MLA_OK;
 }
 
 cudaEvent_t take_event(mla_cache* c) {
@@ -568,6 +622,23 @@ mla_status launch_latent_gemm(mla_cache* c, const void* x, int64_t rows, int64_t
   } else {
     map_qp = map_ckv;   // no query columns in this launch
   }
+  {
+    // MLA_DEBUG build: the output maps stay inside the cache planes and the Qp buffer.
+    const size_t plane_bytes = (size_t)cfg.batch * c->rows_per_stream * kLatent * 2;
+    if ((s = check_extent(c->ckv + dst_row0 * kLatent, kLatent * 2, rows, kLatent * 2, cfg.batch,
+                          plane_rows * kLatent * 2, c->ckv, plane_bytes, "c_kv output")) != MLA_OK ||
+        (s = check_extent(c->krope + dst_row0 * kRope, kRope * 2, rows, kRope * 2, cfg.batch,
+                          plane_rows * kRope * 2, c->krope, plane_bytes / kLatent * kRope,
+                          "k_rope output")) != MLA_OK)
+      return s;
+    if (with_queries) {
+      const uint64_t qcols = (uint64_t)cfg.n_heads * kQK;
+      const size_t qp_bytes = (size_t)cfg.batch * (qp == c->qp ? c->max_q_tokens : qp_tokens) * qcols * 2;
+      if ((s = check_extent(qp, qcols * 2, rows, qcols * 2, cfg.batch, (uint64_t)qp_tokens * qcols * 2,
+                            qp, qp_bytes, "Qp output")) != MLA_OK)
+        return s;
+    }
+  }
   EpiArgs ep{};
   ep.latent_col0 = cfg.n_heads * kQK;
   ep.n_cols = (cfg.n_heads + 1) * kQK;
@@ -607,6 +678,9 @@ mla_status launch_out_proj(mla_cache* c, const __half* o_lat, int64_t o_lat_toke
   if ((s = make_map(&ma, o_lat, kin, nq, cfg.batch, kin * 2, (uint64_t)o_lat_tokens * kin * 2,
                     64, 128, CU_TENSOR_MAP_SWIZZLE_128B, true)) != MLA_OK)
     return s;
+  if ((s = check_extent(o_lat, kin * 2, nq, kin * 2, cfg.batch, (uint64_t)o_lat_tokens * kin * 2, o_lat,
+                        (size_t)cfg.batch * o_lat_tokens * kin * 2, "o_lat input")) != MLA_OK)
+    return s;
   if ((s = make_out_map(&mo, out, cfg.hidden, nq, cfg.batch, (uint64_t)cfg.hidden * 2,
                         (uint64_t)nq * cfg.hidden * 2, false)) != MLA_OK)
     return s;
@@ -634,6 +708,17 @@ mla_status launch_attention(mla_cache* c, const __half* qp, int64_t qp_batch_str
                     (uint64_t)c->rows_per_stream * kRope * 2, 32, 128,
                     CU_TENSOR_MAP_SWIZZLE_64B, true)) != MLA_OK)
     return s;
+  {
+    // MLA_DEBUG build: the key maps stay inside the cache planes.
+    const size_t rows_all = (size_t)cfg.batch * c->rows_per_stream;
+    if ((s = check_extent(c->ckv, kLatent * 2, n_keys, kLatent * 2, cfg.batch,
+                          (uint64_t)c->rows_per_stream * kLatent * 2, c->ckv, rows_all * kLatent * 2,
+                          "c_kv keys")) != MLA_OK ||
+        (s = check_extent(c->krope, kRope * 2, n_keys, kRope * 2, cfg.batch,
+                          (uint64_t)c->rows_per_stream * kRope * 2, c->krope, rows_all * kRope * 2,
+                          "k_rope keys")) != MLA_OK)
+      return s;
+  }
   mla::AttnArgs a{};
   a.qp = qp;
   a.qp_batch_stride = qp_batch_stride;
@@ -680,7 +765,7 @@ mla_status launch_attention(mla_cache* c, const __half* qp, int64_t qp_batch_str
 constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;
 // Per-device tables of looked-up device addresses (the no-alloc scratch, the dense status word).
 constexpr int kMaxDevices = 64;
-static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes + kGuardBytes];
 
 namespace {
 
@@ -701,10 +786,26 @@ mla_status noalloc_scratch(void** out) {
     if (e != cudaSuccess || p == nullptr)
       return fail(MLA_ERR_CUDA, "cudaGetSymbolAddress of the no-alloc scratch failed: %s",
                   cudaGetErrorString(e));
+    if (kGuardBytes) {
+      // MLA_DEBUG build: the guard band after the scratch (no allocation: the array holds it).
+      const cudaError_t e2 =
+          cudaMemset(static_cast<unsigned char*>(p) + kNoAllocScratchBytes, kGuardByte, kGuardBytes);
+      if (e2 != cudaSuccess)
+        return fail(MLA_ERR_CUDA, "guard band of the no-alloc scratch: %s", cudaGetErrorString(e2));
+    }
     g_noalloc_ptr[dev] = p;
   }
   *out = g_noalloc_ptr[dev];
   return MLA_OK;
+}
+
+// Guard band of the current device's no-alloc scratch, if that scratch has been set up.
+const unsigned char* noalloc_guard() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  return g_noalloc_ptr[dev] ? static_cast<const unsigned char*>(g_noalloc_ptr[dev]) + kNoAllocScratchBytes
+                            : nullptr;
 }
 
 size_t align256(size_t n) { return (n + 255) & ~size_t(255); }
@@ -818,6 +919,12 @@ mla_status launch_dense(const void* q, const void* k, const void* v, void* out, 
   dense_plan(batch, n_q, n_kv, n_heads, num_sms, ws ? ws_bytes : 0, &splits, &kv_per_split);
   a.splits = splits;
   a.kv_per_split = kv_per_split;
+  a.batch = batch;
+  a.part_rows = (int64_t)splits * batch * n_q * n_heads;
+#ifdef MLA_DEBUG
+  if (splits > 1 && dense_ws_bytes(splits, batch, n_q, n_heads) > ws_bytes)
+    return fail(MLA_ERR_BOUNDS, "dense split partials need more than the %zu-byte workspace", ws_bytes);
+#endif
   if (splits > 1) {
     const size_t rows = (size_t)batch * n_q * n_heads;
     a.o_part = static_cast<float*>(ws);
@@ -831,7 +938,7 @@ mla_status launch_dense(const void* q, const void* k, const void* v, void* out, 
   if (s2 != MLA_OK || splits == 1) return s2;
   const int64_t rows = (int64_t)batch * n_q * n_heads;
   mla::dense_combine_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(
-      a.o_part, a.ml_part, splits, batch, n_q, n_heads, static_cast<__nv_bfloat16*>(out));
+      a.o_part, a.ml_part, splits, batch, n_q, n_heads, static_cast<__nv_bfloat16*>(out), a.part_rows, status);
   return check_launch("dense split combine");
 }
 
@@ -849,6 +956,7 @@ const char* mla_status_string(mla_status s) {
     case MLA_ERR_DEVICE_TIMEOUT: return "MLA_ERR_DEVICE_TIMEOUT";
     case MLA_ERR_STATE: return "MLA_ERR_STATE";
     case MLA_ERR_RANGE: return "MLA_ERR_RANGE";
+    case MLA_ERR_BOUNDS: return "MLA_ERR_BOUNDS";
   }
   return "MLA_ERR_UNKNOWN";
 }
@@ -1004,15 +1112,15 @@ mla_status mla_cache_create(const mla_config* cfg, const mla_weights* w, void* s
   const mla_config& k = *cfg;
   const size_t ring_rows = (size_t)k.batch * c->rows_per_stream;
   const size_t q_rows = (size_t)k.batch * c->max_q_tokens;
-  MLA_TRY(cudaMalloc(&c->ckv, ring_rows * kLatent * 2));
-  MLA_TRY(cudaMalloc(&c->krope, ring_rows * kRope * 2));
-  MLA_TRY(cudaMalloc(&c->qp, q_rows * k.n_heads * kQK * 2));
-  MLA_TRY(cudaMalloc(&c->o_lat, q_rows * k.n_heads * kLatent * 2));
-  MLA_TRY(cudaMalloc(&c->wqcat, (size_t)(k.n_heads + 1) * kQK * 2 * k.hidden * 2));
-  MLA_TRY(cudaMalloc(&c->wov, (size_t)k.hidden * k.n_heads * kLatent * 2));
-  MLA_TRY(cudaMalloc(&c->status, 256));
+  MLA_TRY(alloc_buffer(c, &c->ckv, ring_rows * kLatent * 2, "c_kv plane", st));
+  MLA_TRY(alloc_buffer(c, &c->krope, ring_rows * kRope * 2, "k_rope plane", st));
+  MLA_TRY(alloc_buffer(c, &c->qp, q_rows * k.n_heads * kQK * 2, "Qp", st));
+  MLA_TRY(alloc_buffer(c, &c->o_lat, q_rows * k.n_heads * kLatent * 2, "o_lat", st));
+  MLA_TRY(alloc_buffer(c, &c->wqcat, (size_t)(k.n_heads + 1) * kQK * 2 * k.hidden * 2, "W_qcat", st));
+  MLA_TRY(alloc_buffer(c, &c->wov, (size_t)k.hidden * k.n_heads * kLatent * 2, "W_OV", st));
+  MLA_TRY(alloc_buffer(c, &c->status, 256, "status block", st));
   const std::vector<float2> rope_hw = make_rope_hw(k);
-  MLA_TRY(cudaMalloc(&c->rope_hw, rope_hw.size() * sizeof(float2)));
+  MLA_TRY(alloc_buffer(c, &c->rope_hw, rope_hw.size() * sizeof(float2), "RoPE table", st));
   MLA_TRY(cudaMemcpyAsync(c->rope_hw, rope_hw.data(), rope_hw.size() * sizeof(float2),
                           cudaMemcpyHostToDevice, st));
   MLA_TRY(cudaMemsetAsync(c->ckv, 0, ring_rows * kLatent * 2, st));
@@ -1072,10 +1180,10 @@ mla_status mla_cache_create(const mla_config* cfg, const mla_weights* w, void* s
   DevTmp qeff_f32;
   if (c->dense_ok) {
     const int nh = k.n_heads, dn = k.d_nope;
-    MLA_TRY(cudaMalloc(&c->wqd, (size_t)nh * 128 * k.hidden * 2));
-    MLA_TRY(cudaMalloc(&c->wukh, (size_t)nh * dn * kLatent * 2));
-    MLA_TRY(cudaMalloc(&c->wuvh, (size_t)nh * 128 * kLatent * 2));
-    MLA_TRY(cudaMalloc(&c->wo, (size_t)k.hidden * nh * 128 * 2));
+    MLA_TRY(alloc_buffer(c, &c->wqd, (size_t)nh * 128 * k.hidden * 2, "dense W_Q", st));
+    MLA_TRY(alloc_buffer(c, &c->wukh, (size_t)nh * dn * kLatent * 2, "dense W_UK", st));
+    MLA_TRY(alloc_buffer(c, &c->wuvh, (size_t)nh * 128 * kLatent * 2, "dense W_UV", st));
+    MLA_TRY(alloc_buffer(c, &c->wo, (size_t)k.hidden * nh * 128 * 2, "dense W_O", st));
     if (k.d_q > 0) {
       // W_Q W_DQ in fp32 (W_QR W_DQ is qr_f32 above).
       MLA_TRY(cudaMalloc(&qeff_f32.p, (size_t)nh * dn * k.hidden * 4));
@@ -1387,6 +1495,8 @@ mla_status mla_window_attention_reconstruct(mla_cache* c, const void* x_chunk, i
     // dense cache the latent layout avoids (B x rows x n_h x 128 x 2 bytes each).  All four or
     // none: a failed allocation leaves the cache as it was.
     void* p[5] = {nullptr, nullptr, nullptr, nullptr, nullptr};
+    const char* names[5] = {"dense Q", "dense O", "dense K", "dense V", "dense split partials"};
+    const size_t n_guards = c->guards.size();
     const size_t bytes[5] = {(size_t)cfg.batch * c->max_q_tokens * hd * 2,
                              (size_t)cfg.batch * c->max_q_tokens * hd * 2,
                              (size_t)cfg.batch * c->rows_per_stream * hd * 2,
@@ -1394,9 +1504,10 @@ mla_status mla_window_attention_reconstruct(mla_cache* c, const void* x_chunk, i
                              dense_ws_bytes(kDenseMaxSplits, cfg.batch, (int)c->max_q_tokens, nh)};
     for (int i = 0; i < 5; ++i) {
       if (bytes[i] == 0) continue;
-      const cudaError_t e = cudaMalloc(&p[i], bytes[i]);
+      const cudaError_t e = alloc_buffer(c, &p[i], bytes[i], names[i], st);
       if (e != cudaSuccess) {
-        for (int k = 0; k < i; ++k) cudaFree(p[k]);
+        for (int k = 0; k <= i; ++k) cudaFree(p[k]);
+        c->guards.resize(n_guards);
         return fail(e == cudaErrorMemoryAllocation ? MLA_ERR_OUT_OF_MEMORY : MLA_ERR_CUDA,
                     "dense-form buffers: cudaMalloc of %zu bytes failed: %s", bytes[i],
                     cudaGetErrorString(e));
@@ -1462,7 +1573,8 @@ mla_status mla_window_attention_reconstruct(mla_cache* c, const void* x_chunk, i
              c->num_sms, st, "key reconstruction")) != MLA_OK)
       return s;
     krope_broadcast_kernel<<<dim3((unsigned)n_keys, (unsigned)cfg.batch), 128, 0, st>>>(
-        c->krope, c->rows_per_stream, c->kd, (int)n_keys, nh, dn);
+        c->krope, c->rows_per_stream, c->kd, (int)n_keys, nh, dn,
+        (int64_t)cfg.batch * c->rows_per_stream, c->status);
     if ((s = check_launch("k_rope broadcast")) != MLA_OK) return s;
     EpiArgs ev{};
     ev.n_cols = (int)hd;
@@ -1508,6 +1620,28 @@ mla_status mla_cache_selftest_timeout(mla_cache* c, void* stream, int32_t* gave_
   MLA_CUDA(cudaMemcpy(&h, flag, sizeof(int), cudaMemcpyDeviceToHost));
   *gave_up = h;
   return MLA_OK;
+}
+
+mla_status mla_cache_selftest_bounds(mla_cache* c, void* stream, int32_t* caught) {
+  if (!c || !caught) return fail(MLA_ERR_INVALID_ARGUMENT, "NULL argument");
+#ifndef MLA_DEBUG
+  return fail(MLA_ERR_UNSUPPORTED, "bounds checks exist only in the MLA_DEBUG build (libmla_debug.so)");
+#else
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  // Rows [last, last + 2) of every stream onto themselves: row `last` is the last row of the
+  // planes (copied onto itself, a no-op), row last + 1 is past them and must be caught.
+  const int64_t last = c->rows_per_stream - 1;
+  const int64_t work = 2 * (kLatent / 8 + kRope / 8);
+  move_rows_kernel<<<dim3((unsigned)((work + 255) / 256), (unsigned)c->cfg.batch), 256, 0, st>>>(
+      c->ckv, c->krope, (int64_t)c->rows_per_stream, last, last, 2, c->status);
+  mla_status s = check_launch("bounds self-test");
+  if (s != MLA_OK) return s;
+  MLA_CUDA(cudaStreamSynchronize(st));
+  int word = 0;
+  MLA_CUDA(cudaMemcpy(&word, c->status, sizeof(int), cudaMemcpyDeviceToHost));
+  *caught = word == MLA_ERR_BOUNDS ? 1 : 0;
+  return MLA_OK;
+#endif
 }
 
 mla_status mla_dense_split_plan(int32_t batch, int32_t n_q, int32_t n_kv, int32_t n_heads,
@@ -1589,6 +1723,18 @@ mla_status mla_cache_sync(mla_cache* c, void* stream) {
   int words[mla::kStatusRangeWord + 1] = {0};
   MLA_CUDA(cudaMemcpy(words, c->status, sizeof(words), cudaMemcpyDeviceToHost));
   if (words[0] != 0) return fail((mla_status)words[0], "a kernel recorded device status %d", words[0]);
+  if (kGuardBytes) {
+    // MLA_DEBUG build: no kernel may have written past the end of a buffer.
+    std::vector<unsigned char> h(kGuardBytes);
+    auto intact = [&](const unsigned char* g) {
+      return cudaMemcpy(h.data(), g, kGuardBytes, cudaMemcpyDeviceToHost) == cudaSuccess &&
+             std::all_of(h.begin(), h.end(), [](unsigned char b) { return b == kGuardByte; });
+    };
+    for (const auto& g : c->guards)
+      if (!intact(g.p)) return fail(MLA_ERR_BOUNDS, "guard band after the %s was overwritten", g.name);
+    if (const unsigned char* g = noalloc_guard())
+      if (!intact(g)) return fail(MLA_ERR_BOUNDS, "guard band after the no-alloc scratch was overwritten");
+  }
   if (words[mla::kStatusRangeWord] != 0) {
     // Reported once: clear the word so that the next sync covers the calls made after this one.
     MLA_CUDA(cudaMemsetAsync(c->status + mla::kStatusRangeWord, 0, sizeof(int), st));

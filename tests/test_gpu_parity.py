@@ -78,12 +78,11 @@ def full_check(pair: Pair, x_chunk, what: str, intermediates: bool = True):
             qp = pair.gpu.copy_buffer(0, (pair.w.batch, pair.gpu.cfg.max_chunk_frames * pair.F * nh, 224))
             assert_close(qp[b, :nq * nh], oracle_qp(pair, x_chunk[b], b), f"{what}: Qp (stream {b})")
             ol = pair.gpu.copy_buffer(1, (pair.w.batch, pair.gpu.cfg.max_chunk_frames * pair.F * nh, 192))
-            # o_lat is an internal fp16 intermediate, not an output: its RMS is well below its
-            # peaks (rows that attend sharply copy one latent), so the rounding of the bf16
-            # weights and fp16 queries shows up as a larger max-abs/RMS than in the projected
-            # output.  Same L2 bar; the observed max-abs/RMS is printed (pytest -s).
+            # o_lat, the fp16 latent-space attention output, meets the same bar as the layer
+            # output (worst observed max-abs/RMS 6.5e-3); the observed errors are printed
+            # (pytest -s).
             rel_o, mx_o = assert_close(ol[b, :nq * nh], parts["Pc"].reshape(-1, 192),
-                                       f"{what}: o_lat (stream {b})", max_tol=1e-1)
+                                       f"{what}: o_lat (stream {b})")
             print(f"o_lat parity [{what}, stream {b}]: rel L2 {rel_o:.3e}, max-abs/RMS {mx_o:.3e}")
     pair.check_status()
     return out
