@@ -51,7 +51,8 @@ def parse_args(argv=None):
     p.add_argument("--cpu-rows", type=int, default=1560, help="query tokens in the oracle's timed sample")
     p.add_argument("--ncu-case", choices=("attention", "append", "steps", "dense"), default=None,
                    help="minimal launch sequence for an ncu capture (prints no benchmark line): "
-                        "'attention' = fill + 2 steps, 'append' = 2 x 21-frame fill, 'steps' = warmup + K steps, "
+                        "'attention' = fill + 2 steps, 'append' = 2 x 21-frame fill, 'steps' = warmup + K steps "
+                        "(attention + commit), "
                         "'dense' = the dense per-head baseline over the 21-frame window (2 split-key calls, "
                         "then 1 one-pass call)")
     return p.parse_args(argv)
@@ -101,7 +102,7 @@ def run_ncu_case(args, local):
         for s in range(n):
             c = caches[s % n_layers]
             c.attention(x, out)
-            c.append(x)
+            c.commit(w.query_frames)
     torch.cuda.synchronize()
     ok = all(B.mla_cache_sync(c.handle) == 0 for c in caches)
     print(json.dumps({"ncu_case": args.ncu_case, "device_status_ok": ok}))
