@@ -180,6 +180,24 @@ mla_status mla_window_attention(mla_cache* c, const void* x_chunk, int32_t n_fra
  *  - Stream-ordered like mla_cache_append. */
 mla_status mla_cache_commit(mla_cache* c, int32_t n_frames, void* stream);
 
+/* One frame's move inside a stream's latent planes: rows [src_row, src_row + rows) go to
+ * [dst_row, dst_row + rows) (both plane rows, per stream). */
+typedef struct {
+  int64_t src_row, dst_row, rows;
+} mla_row_move;
+
+/* Host-only view of the moves mla_cache_commit launches for a chunk of n_frames frames attended
+ * when frames_appended frames had been appended: the chunk's latents sit at the chunk tail (the
+ * rows right after the valid sink region and window) and each surviving frame goes to the rows
+ * mla_ring_slot names for its frame index; frames already in place are not listed, and frames
+ * the chunk itself evicts (more than W new window frames) are skipped.  The moves must be applied
+ * in the listed order: a destination may be the source of an earlier move, never of a later one.
+ * *n_moves receives the count; at most max_moves are written (MLA_ERR_INVALID_ARGUMENT if more
+ * are needed, or for an invalid config, n_frames outside [1, max_chunk_frames], or
+ * frames_appended < 0).  No GPU needed. */
+mla_status mla_commit_plan(const mla_config* cfg, int64_t frames_appended, int32_t n_frames,
+                           mla_row_move* moves, int32_t max_moves, int32_t* n_moves);
+
 /* Same computation and result as mla_window_attention, for callers that must not allocate
  * device memory while they run: code whose device memory belongs to a pooled or budgeted
  * allocator it may not bypass, and latency-critical loops that cannot afford the implicit

@@ -4,7 +4,7 @@ The compute path lives in csrc/ (CUDA kernels behind the C ABI of include/mla.h)
 marshals torch tensors and streams into those calls.  Build with build.py.
 """
 from .binding import (  # noqa: F401
-    EXPORTED, LatentWindowCache, MLAError, load_library, make_config, mla_cache_append, mla_cache_commit,
+    EXPORTED, LatentWindowCache, MLAError, load_library, make_config, mla_cache_append, mla_cache_commit, mla_commit_plan,
     mla_cache_copy_buffer, mla_cache_create, mla_cache_debug_buffers, mla_cache_destroy,
     mla_cache_device_bytes, mla_cache_profile_enable, mla_cache_profile_read, mla_cache_read,
     mla_cache_state, mla_cache_sync, mla_config, mla_config_check, mla_ring_bytes, mla_ring_slot,

@@ -29,7 +29,7 @@ KERNEL_NAMES = ("append", "qproj", "attention", "oproj")
 
 EXPORTED = (
     "mla_config_check", "mla_ring_slot", "mla_ring_bytes", "mla_cache_device_bytes",
-    "mla_cache_create", "mla_cache_append", "mla_cache_commit", "mla_window_attention",
+    "mla_cache_create", "mla_cache_append", "mla_cache_commit", "mla_commit_plan", "mla_window_attention",
     "mla_window_attention_noalloc",
     "mla_window_attention_reconstruct", "mla_cache_selftest_timeout", "mla_cache_selftest_bounds",
     "mla_cache_destroy", "mla_dense_split_plan", "mla_dense_workspace_bytes", "mla_dense_attention",
@@ -67,6 +67,10 @@ class mla_debug_buffers(ctypes.Structure):
         [("rows_per_stream", ctypes.c_int64)]
 
 
+class mla_row_move(ctypes.Structure):
+    _fields_ = [("src_row", ctypes.c_int64), ("dst_row", ctypes.c_int64), ("rows", ctypes.c_int64)]
+
+
 class mla_profile(ctypes.Structure):
     _fields_ = [("ms", ctypes.c_double * 4), ("launches", ctypes.c_int64 * 4)]
 
@@ -91,6 +95,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "mla_cache_create": (I32, [P(mla_config), P(mla_weights), VP, P(VP)]),
         "mla_cache_append": (I32, [VP, VP, I32, VP]),
         "mla_cache_commit": (I32, [VP, I32, VP]),
+        "mla_commit_plan": (I32, [P(mla_config), I64, I32, P(mla_row_move), I32, P(I32)]),
         "mla_window_attention": (I32, [VP, VP, I32, VP, VP]),
         "mla_window_attention_noalloc": (I32, [VP, VP, I32, VP, VP]),
         "mla_window_attention_reconstruct": (I32, [VP, VP, I32, VP, VP]),
@@ -191,6 +196,15 @@ def mla_cache_append(cache: int, x, n_frames: int, stream=None) -> None:
 
 def mla_cache_commit(cache: int, n_frames: int, stream=None) -> None:
     _check(load_library().mla_cache_commit(cache, n_frames, _stream_handle(stream)), "mla_cache_commit")
+
+
+def mla_commit_plan(cfg: mla_config, frames_appended: int, n_frames: int) -> list:
+    """Host-only: the (src_row, dst_row, rows) moves mla_cache_commit makes, in order."""
+    buf = (mla_row_move * max(n_frames, 1))()
+    n = ctypes.c_int32()
+    _check(load_library().mla_commit_plan(ctypes.byref(cfg), frames_appended, n_frames, buf,
+                                          max(n_frames, 1), ctypes.byref(n)), "mla_commit_plan")
+    return [(buf[i].src_row, buf[i].dst_row, buf[i].rows) for i in range(n.value)]
 
 
 def mla_window_attention(cache: int, x_chunk, n_frames: int, out, stream=None) -> None:

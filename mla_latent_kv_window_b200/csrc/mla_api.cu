@@ -457,10 +457,13 @@ void set_pending(mla_cache* c, int32_t n_frames) {
 
 // Valid sink frames (vs) and valid window frames (vw) of a cache: the first sink_frames frames
 // ever appended are the sink, the newest W of the others the window.
-void valid_counts(const mla_cache* c, int64_t& vs, int64_t& vw) {
-  const int64_t A = c->frames_appended, S = c->cfg.sink_frames, W = c->cfg.window_frames;
+void valid_counts_of(const mla_config& cfg, int64_t A, int64_t& vs, int64_t& vw) {
+  const int64_t S = cfg.sink_frames, W = cfg.window_frames;
   vs = A < S ? A : S;
   vw = A - vs < W ? A - vs : W;
+}
+void valid_counts(const mla_cache* c, int64_t& vs, int64_t& vw) {
+  valid_counts_of(c->cfg, c->frames_appended, vs, vw);
 }
 
 // cudaMalloc of a cache buffer; the MLA_DEBUG build adds a guard band after it (filled on
@@ -1014,6 +1017,38 @@ mla_status mla_ring_slot(const mla_config* cfg, int64_t frame, int32_t token, in
   return MLA_OK;
 }
 
+mla_status mla_commit_plan(const mla_config* cfg, int64_t frames_appended, int32_t n_frames,
+                           mla_row_move* moves, int32_t max_moves, int32_t* n_moves) {
+  if (!cfg || !n_moves || (max_moves > 0 && !moves))
+    return fail(MLA_ERR_INVALID_ARGUMENT, "NULL argument");
+  mla_status s = mla_config_check(cfg);
+  if (s != MLA_OK) return s;
+  const mla_config& k = *cfg;
+  if (n_frames < 1 || n_frames > k.max_chunk_frames || frames_appended < 0)
+    return fail(MLA_ERR_INVALID_ARGUMENT, "n_frames must be in [1, max_chunk_frames] and frames_appended >= 0");
+  const int64_t S = k.sink_frames, W = k.window_frames, F = (int64_t)k.frame_h * k.frame_w;
+  const int64_t A = frames_appended, sink_rows = sink_rows_of(k);
+  int64_t vs, vw;
+  valid_counts_of(k, A, vs, vw);
+  const int64_t base_row = sink_rows + vw * F;      // where the attention call put the chunk
+  // Chunk frames that become sink frames, then the others, of which only the last W survive.
+  const int64_t to_sink = A < S ? (S - A < n_frames ? S - A : n_frames) : 0;
+  const int64_t n_window = n_frames - to_sink;
+  const int64_t skip = n_window > W ? n_window - W : 0;
+  int32_t n = 0;
+  for (int64_t i = 0; i < n_frames; ++i) {
+    if (i >= to_sink && i - to_sink < skip) continue;            // evicted within the chunk
+    const int64_t t = A + i;
+    const int64_t dst = t < S ? t * F : sink_rows + ((t - S) % W) * F;
+    const int64_t src = base_row + i * F;
+    if (dst == src) continue;                                    // already in place
+    if (n >= max_moves) return fail(MLA_ERR_INVALID_ARGUMENT, "more than max_moves moves");
+    moves[n++] = mla_row_move{src, dst, F};
+  }
+  *n_moves = n;
+  return MLA_OK;
+}
+
 size_t mla_ring_bytes(const mla_config* cfg) {
   if (!cfg || cfg->batch <= 0 || cfg->window_frames <= 0 || cfg->frame_h <= 0 ||
       cfg->frame_w <= 0 || cfg->d_latent <= 0 || cfg->d_rope < 0 || cfg->sink_frames < 0)
@@ -1343,34 +1378,23 @@ mla_status mla_cache_commit(mla_cache* c, int32_t n_frames, void* stream) {
                 c->pending_frames);
   const mla_config& cfg = c->cfg;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const int64_t S = cfg.sink_frames, W = cfg.window_frames, F = c->F;
-  int64_t vs, vw;
-  valid_counts(c, vs, vw);
-  const int64_t base_row = c->sink_rows + vw * F;   // where the attention call put the chunk
-  const int64_t A = c->frames_appended;
-  // Non-sink frames of the chunk that survive: the last W of them.
-  const int64_t first_sink_free = A < S ? (S - A < n_frames ? S - A : n_frames) : 0;
-  const int64_t n_window = n_frames - first_sink_free;
-  const int64_t skip = n_window > W ? n_window - W : 0;
+  std::vector<mla_row_move> moves((size_t)n_frames);
+  int32_t n_moves = 0;
+  mla_status s = mla_commit_plan(&cfg, c->frames_appended, n_frames, moves.data(), n_frames, &n_moves);
+  if (s != MLA_OK) return s;
   {
     ProfScope p(c, MLA_KERNEL_APPEND, st);
-    // In chunk order: a frame's destination can be the source of an earlier frame of the same
-    // chunk (sink frames fill up first), never of a later one, so frame-by-frame launches in
-    // this order read every source before it is overwritten.
-    for (int64_t i = 0; i < n_frames; ++i) {
-      if (i >= first_sink_free && i - first_sink_free < skip) continue;   // evicted in the chunk
-      const int64_t t = A + i;
-      const int64_t dst = t < S ? t * F : c->sink_rows + ((t - S) % W) * F;
-      const int64_t src = base_row + i * F;
-      if (dst == src) continue;
-      const int64_t work = F * (kLatent / 8 + kRope / 8);
+    // In the plan's order (a destination can be the source of an earlier move only), one launch
+    // per frame, stream-ordered.
+    for (int32_t i = 0; i < n_moves; ++i) {
+      const int64_t work = moves[i].rows * (kLatent / 8 + kRope / 8);
       dim3 grid((unsigned)((work + 255) / 256), (unsigned)cfg.batch);
       const cudaError_t e = launch_pdl(move_rows_kernel, grid, dim3(256), 0, st, c->ckv, c->krope,
-                                       (int64_t)c->rows_per_stream, src, dst, F, c->status);
+                                       (int64_t)c->rows_per_stream, moves[i].src_row,
+                                       moves[i].dst_row, moves[i].rows, c->status);
       if (e != cudaSuccess)
         return fail(MLA_ERR_CUDA, "commit copy launch failed: %s", cudaGetErrorString(e));
-      const mla_status s = check_launch("commit copy");
-      if (s != MLA_OK) return s;
+      if ((s = check_launch("commit copy")) != MLA_OK) return s;
     }
   }
   c->frames_appended += n_frames;
