@@ -1,0 +1,49 @@
+"""GPU: seeded random shapes and call sequences against the fp64 oracle (every element).
+
+Each case draws a small model (4 or 12 heads of 128, hidden 512 or 1536), a frame grid (1 to 40
+tokens, ragged against the 128-key tiles), a window of 1 to 4 frames, 0 to 2 sink frames, 1 to 3
+streams with their own scales, chunks of 1 to 3 frames, and a sequence of appends, attention calls
+and commits; after every attention call every output element is compared with the oracle, and
+after every append or commit every cached frame's rows.
+"""
+import random
+
+import pytest
+import torch
+
+import mla_synth
+from tests.harness import Pair
+from tests.test_gpu_parity import check_ring, full_check
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("case", range(12))
+def test_random_shapes_and_sequences(case):
+    rng = random.Random(1000 + case)
+    heads = rng.choice([4, 12])
+    dims = dict(mla_synth.DIMS_WAN13B, hidden=128 * heads, n_heads=heads)
+    fh, fw = rng.randint(1, 5), rng.randint(1, 8)
+    max_chunk = rng.randint(1, 3)
+    w = mla_synth.Workload(f"fuzz{case}", frame_h=fh, frame_w=fw, window_frames=rng.randint(1, 4),
+                           fill_frames=0, query_frames=max_chunk, batch=rng.randint(1, 3),
+                           seed=7000 + case, stream_scale=True, sink_frames=rng.choice([0, 0, 1, 2]),
+                           dims=tuple(sorted(dims.items())))
+    p = Pair(w, max_chunk_frames=max_chunk)
+    seed = 90000 + 100 * case
+    for _ in range(8):
+        op = rng.random()
+        n = rng.randint(1, max_chunk)
+        x = p.hidden(n, seed)
+        seed += 1
+        if op < 0.35:
+            p.append(x)
+            check_ring(p, f"fuzz {case}: after append of {n}")
+        else:
+            full_check(p, x, f"fuzz {case}: {n}-frame chunk", intermediates=op < 0.5)
+            if op > 0.7:
+                p.gpu.commit(n)
+                for b, o in enumerate(p.oracles):
+                    o.append(x[b])
+                check_ring(p, f"fuzz {case}: after commit of {n}")
+    p.gpu.close()

@@ -60,6 +60,8 @@ MUTATIONS = [
      "out.append((f, c.copy(), r.copy()))"),
     ("ring contents one frame ahead in time", "out.append((f, c.copy(), self._rope(r, f, hh, ww)))",
      "out.append((f, c.copy(), self._rope(r, f + 1, hh, ww)))"),
+    ("a head subset drops all but its first head", "for h in (range(nh) if heads is None else heads):",
+     "for h in (range(nh) if heads is None else heads[:1]):"),
     ("dense baseline without the softmax scale", "S = (q[:, h, :] @ k[:, h, :].T) * scale",
      "S = (q[:, h, :] @ k[:, h, :].T)"),
     ("dense baseline normalising over queries", "out[:, h, :] = (E / E.sum(axis=1, keepdims=True)) @ v[:, h, :]",

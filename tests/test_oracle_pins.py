@@ -445,3 +445,14 @@ def test_cache_contents_brute_force_absolute_index(sink):
             np.testing.assert_allclose(c, np.array(c_ref), rtol=1e-13, atol=1e-13)
             np.testing.assert_allclose(r, np.array(r_ref), rtol=1e-13, atol=1e-13)
     assert seen == 12 and layer.frames_appended == 12
+
+
+def test_head_subsets_add_up_to_the_full_output():
+    # The output projection is linear in the per-head outputs, so attention restricted to a
+    # subset of heads (used to time bounded samples) must give that subset's share of the output:
+    # disjoint subsets covering every head add up to the full output.
+    layer, _, _, x_q = _tiny_run(_dims(frame_h=2, frame_w=3, window_frames=2, hidden=256, n_heads=4,
+                                       d_head=64, d_nope=64), fill=3)
+    full = layer.attention(x_q)
+    parts = layer.attention(x_q, heads=[0, 2]) + layer.attention(x_q, heads=[1]) + layer.attention(x_q, heads=[3])
+    np.testing.assert_allclose(parts, full, rtol=1e-12, atol=1e-12)
