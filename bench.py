@@ -655,6 +655,27 @@ def batched_leg(B, dev, stream, rank, world, tf_peak, hbm_peak, reps=5):
     }
 
 
+def graph_replay_ms(B, c, x, out, reps=20):
+    """Per-call ms of one attention call on cache c, launched directly and as a CUDA-graph replay
+    (the call captured once with static x and out buffers; valid while the cache state it saw at
+    capture is unchanged, i.e. for the denoising steps of one chunk)."""
+    import torch
+    st = torch.cuda.current_stream()
+    direct = _event_ms(lambda: c.attention(x, out, st), st, reps=reps)
+    side = torch.cuda.Stream()
+    side.wait_stream(st)
+    with torch.cuda.stream(side):
+        c.attention(x, out)
+    st.wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        c.attention(x, out)
+    replay = _event_ms(g.replay, st, reps=reps)
+    del g
+    return direct, replay
+
+
 def tiny_leg(B, dev, stream):
     """The small workload (4 x 6 frames, 2-frame window, one query frame): launch-bound."""
     import torch
@@ -668,10 +689,12 @@ def tiny_leg(B, dev, stream):
     x = mla_synth.make_hidden(1, w.F, dims["hidden"], mla_synth.chunk_seed(w, 0, 0)).to(dev)
     out = torch.empty_like(x)
     ms = _event_ms(lambda: B.mla_window_attention(c.handle, x, 1, out, stream), stream, reps=20)
+    direct, replay = graph_replay_ms(B, c, x, out)
     ok = B.mla_cache_sync(c.handle) == 0
     c.close()
     return {"workload": "4 x 6-token frames, 2-frame window, one query frame (72 keys)", "call_ms": round(ms, 4),
             "query_tokens_per_s": round(w.F / (ms / 1e3), 1), "status_ok": ok,
+            "cuda_graph": {"direct_call_ms": round(direct, 4), "graph_replay_ms": round(replay, 4)},
             "note": "launch-bound: three kernels for 24 query tokens"}
 
 
