@@ -29,6 +29,7 @@
 
 #include "../../include/mla.h"
 #include "gemm_tc.cuh"
+#include "query_proj.cuh"
 #include "window_attn.cuh"
 #include "dense_attn.cuh"
 
@@ -298,6 +299,32 @@ __global__ void build_wqd_kernel(const __nv_bfloat16* __restrict__ w_q,
   }
   wqd[(size_t)row * hidden + k] = __float2bfloat16_rn(v);
 }
+// Two-step query weights, wq2 [latent_row0 + 224][hidden], a copy of the caller's bf16 values:
+// per head h, rows h*160 + j hold W_Q[h*128 + j] (j < 128) and W_QR[h*32 + j - 128] (the next 32
+// rows); rows [n_h*160, latent_row0) are zero; then W_DKV (192 rows) and W_KR (32 rows).
+// latent_row0 is n_h*160 rounded up to a multiple of 224, the period by which the latent-only
+// projection (tc_gemm_kernel) tells the c_kv and k_rope columns of its block apart.
+__global__ void build_wq2_kernel(const __nv_bfloat16* __restrict__ w_q,
+                                 const __nv_bfloat16* __restrict__ w_qr,
+                                 const __nv_bfloat16* __restrict__ w_dkv,
+                                 const __nv_bfloat16* __restrict__ w_kr,
+                                 __nv_bfloat16* __restrict__ wq2, int hidden, int n_heads,
+                                 int latent_row0) {
+  const int k = blockIdx.x * blockDim.x + threadIdx.x;
+  const int row = blockIdx.y;
+  if (k >= hidden) return;
+  const int per = mla::kQpBN;
+  const __nv_bfloat16* src = nullptr;
+  if (row < n_heads * per) {
+    const int h = row / per, j = row % per;
+    src = j < mla::kQpNope ? w_q + (size_t)(h * mla::kQpNope + j) * hidden
+                           : w_qr + (size_t)(h * kRope + j - mla::kQpNope) * hidden;
+  } else if (row >= latent_row0) {
+    const int j = row - latent_row0;
+    src = j < kLatent ? w_dkv + (size_t)j * hidden : w_kr + (size_t)(j - kLatent) * hidden;
+  }
+  wq2[(size_t)row * hidden + k] = src ? src[k] : __float2bfloat16_rn(0.f);
+}
 __global__ void bf16_to_f16_kernel(const __nv_bfloat16* __restrict__ in, __half* __restrict__ out,
                                    int64_t n, int* range) {
   const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
@@ -404,7 +431,17 @@ struct mla_cache {
   __half* krope = nullptr;
   __half* qp = nullptr;            // fp16 absorbed queries
   __half* o_lat = nullptr;         // fp16 P . c_kv
-  __nv_bfloat16* wqcat = nullptr;  // bf16: multiplies the caller's bf16 hidden states
+  // Query and latent projection weights (bf16: they multiply the caller's bf16 hidden states).
+  // Full-rank query with d_nope = 128 (two_step): the caller's rows [W_Q[h]; W_QR[h]] per head,
+  // then W_DKV and W_KR, hidden columns each; query_proj_kernel multiplies them and then
+  // W_UK[h] (wuk16).  Otherwise the absorbed bf16 pairs [hi | lo] of 2 * hidden columns.
+  __nv_bfloat16* wqcat = nullptr;
+  bool two_step = false;
+  int64_t wq_rows = 0;             // rows of wqcat
+  int64_t wq_cols = 0;             // columns of a wqcat row (hidden or 2 * hidden)
+  int32_t latent_row0 = 0;         // first W_DKV row of wqcat (a multiple of 224)
+  __half* wuk16 = nullptr;         // two_step: W_UK [n_h*128][192] fp16 (multiplies the fp16 q pair)
+  CUtensorMap map_wuk16{};
   __half* wov = nullptr;           // fp16: multiplies o_lat
   float2* rope_hw = nullptr;       // RoPE (cos, sin) of the h and w bands, [16][frame_h + frame_w]
 
@@ -578,11 +615,14 @@ mla_status launch_latent_gemm(mla_cache* c, const void* x, int64_t rows, int64_t
                               bool with_queries, int64_t t0, int64_t dst_row0, cudaStream_t st,
                               __half* qp = nullptr, int64_t qp_tokens = 0) {
   const mla_config& cfg = c->cfg;
+  // Full-rank query with d_nope = 128: query_proj_kernel (256-row tiles, the caller's weights
+  // and W_UK in two chained products).
+  const bool two_step = with_queries && c->two_step;
   const int n_cols = with_queries ? (cfg.n_heads + 1) * kQK : kQK;   // columns of this launch
-  // With queries the absorbed weights' lo halves are multiplied too (K = 2 x hidden, A wraps);
-  // the latent-only launch reads the hi halves, which hold W_DKV and W_KR exactly.
-  const int K = with_queries ? 2 * cfg.hidden : cfg.hidden;
-  const int a_kwrap = with_queries ? cfg.hidden : 0;
+  // With absorbed queries the weights' lo halves are multiplied too (K = 2 x hidden, A wraps);
+  // the latent-only launch reads the first hidden columns, which hold W_DKV and W_KR exactly.
+  const int K = with_queries && !two_step ? 2 * cfg.hidden : cfg.hidden;
+  const int a_kwrap = with_queries && !two_step ? cfg.hidden : 0;
   const int num_kb = K / 64;
   // Pick the tile shape with the least estimated time (waves x k-blocks x k-block time).
   auto tiles_of = [&](const TileShape& t) {
@@ -603,8 +643,8 @@ mla_status launch_latent_gemm(mla_cache* c, const void* x, int64_t rows, int64_t
 
   CUtensorMap map_x, map_ckv, map_krope, map_qp;
   mla_status s = make_map(&map_x, x, cfg.hidden, rows, cfg.batch, (uint64_t)cfg.hidden * 2,
-                          (uint64_t)x_batch_rows * cfg.hidden * 2, 64, 128 * shape.m_sub,
-                          CU_TENSOR_MAP_SWIZZLE_128B);
+                          (uint64_t)x_batch_rows * cfg.hidden * 2, 64,
+                          two_step ? 256 : 128 * shape.m_sub, CU_TENSOR_MAP_SWIZZLE_128B);
   if (s != MLA_OK) return s;
   const uint64_t plane_rows = (uint64_t)c->rows_per_stream;
   if ((s = make_out_map(&map_ckv, c->ckv + dst_row0 * kLatent, kLatent, rows, cfg.batch,
@@ -643,8 +683,10 @@ mla_status launch_latent_gemm(mla_cache* c, const void* x, int64_t rows, int64_t
     }
   }
   EpiArgs ep{};
-  ep.latent_col0 = cfg.n_heads * kQK;
-  ep.n_cols = (cfg.n_heads + 1) * kQK;
+  // Output columns are B rows: the latent block starts at the absorbed heads' end (queries) or
+  // at the weights' latent rows (latent only).
+  ep.latent_col0 = with_queries ? cfg.n_heads * kQK : c->latent_row0;
+  ep.n_cols = ep.latent_col0 + kQK;
   ep.t0 = t0;
   ep.tokens_per_frame = c->F;
   ep.frame_w = cfg.frame_w;
@@ -652,8 +694,20 @@ mla_status launch_latent_gemm(mla_cache* c, const void* x, int64_t rows, int64_t
   ep.rope = c->rope;
   ep.rope_hw = c->rope_hw;
   ep.frame_h = cfg.frame_h;
-  const int b_row0 = with_queries ? 0 : cfg.n_heads * kQK;
   const char* what = "latent projection";
+  if (two_step) {
+    const mla::GemmTiles qt{(int32_t)((rows + 255) / 256), cfg.n_heads + 2, cfg.batch};
+    const int n = qt.count();
+    if (n <= 0) return MLA_OK;
+    const cudaError_t e = launch_pdl(mla::query_proj_kernel, dim3(n < c->num_sms ? n : c->num_sms),
+                                     dim3(mla::kQpThreads), mla::QpSmem::kBytes, st, map_x,
+                                     c->map_wqcat160, c->map_wuk16, map_qp, map_ckv, map_krope,
+                                     (int)rows, cfg.hidden, cfg.n_heads, c->latent_row0, qt, ep,
+                                     c->status);
+    if (e != cudaSuccess) return fail(MLA_ERR_CUDA, "query projection launch failed: %s", cudaGetErrorString(e));
+    return check_launch("query projection");
+  }
+  const int b_row0 = with_queries ? 0 : c->latent_row0;
   if (shape.bn == 32)
     return launch_gemm<32, kProjNarrowAStages, kProjNarrowBStages, mla::kEpiLatent, false, 1>(
         map_x, c->map_wqcat32, map_qp, map_ckv, map_krope, (int)rows, K, b_row0, tiles,
@@ -1067,7 +1121,11 @@ size_t mla_cache_device_bytes(const mla_config* cfg) {
   b += (size_t)c.batch * rows * kQK * 2;                   // ckv + krope (ring + chunk tail)
   b += (size_t)c.batch * q * c.n_heads * kQK * 2;          // Qp
   b += (size_t)c.batch * q * c.n_heads * kLatent * 2;      // o_lat
-  b += (size_t)(c.n_heads + 1) * kQK * c.hidden * 4;       // Wqcat (bf16 hi + lo)
+  if (c.d_q == 0 && c.d_nope == mla::kQpNope)              // the caller's query and latent
+    b += ((size_t)(c.n_heads * mla::kQpBN + kQK - 1) / kQK * kQK + kQK) * c.hidden * 2 +
+         (size_t)c.n_heads * mla::kQpNope * kLatent * 2;      // weights (bf16), W_UK (fp16)
+  else
+    b += (size_t)(c.n_heads + 1) * kQK * c.hidden * 4;     // Wqcat (bf16 hi + lo)
   b += (size_t)c.hidden * c.n_heads * kLatent * 2;         // W_OV
   b += 256;                                                // status word
   b += (size_t)(c.frame_h + c.frame_w) * 16 * 8;           // RoPE h / w tables
@@ -1090,6 +1148,7 @@ void mla_cache_destroy(mla_cache* c) {
   cudaFree(c->qp);
   cudaFree(c->o_lat);
   cudaFree(c->wqcat);
+  cudaFree(c->wuk16);
   cudaFree(c->wov);
   cudaFree(c->rope_hw);
   cudaFree(c->wqd);
@@ -1151,7 +1210,13 @@ mla_status mla_cache_create(const mla_config* cfg, const mla_weights* w, void* s
   MLA_TRY(alloc_buffer(c, &c->krope, ring_rows * kRope * 2, "k_rope plane", st));
   MLA_TRY(alloc_buffer(c, &c->qp, q_rows * k.n_heads * kQK * 2, "Qp", st));
   MLA_TRY(alloc_buffer(c, &c->o_lat, q_rows * k.n_heads * kLatent * 2, "o_lat", st));
-  MLA_TRY(alloc_buffer(c, &c->wqcat, (size_t)(k.n_heads + 1) * kQK * 2 * k.hidden * 2, "W_qcat", st));
+  c->two_step = k.d_q == 0 && k.d_nope == mla::kQpNope;
+  c->latent_row0 = c->two_step ? (k.n_heads * mla::kQpBN + kQK - 1) / kQK * kQK : k.n_heads * kQK;
+  c->wq_rows = (int64_t)c->latent_row0 + kQK;
+  c->wq_cols = c->two_step ? k.hidden : 2 * (int64_t)k.hidden;
+  MLA_TRY(alloc_buffer(c, &c->wqcat, (size_t)c->wq_rows * c->wq_cols * 2, "W_qcat", st));
+  if (c->two_step)
+    MLA_TRY(alloc_buffer(c, &c->wuk16, (size_t)k.n_heads * mla::kQpNope * kLatent * 2, "W_UK fp16", st));
   MLA_TRY(alloc_buffer(c, &c->wov, (size_t)k.hidden * k.n_heads * kLatent * 2, "W_OV", st));
   MLA_TRY(alloc_buffer(c, &c->status, 256, "status block", st));
   const std::vector<float2> rope_hw = make_rope_hw(k);
@@ -1198,10 +1263,19 @@ mla_status mla_cache_create(const mla_config* cfg, const mla_weights* w, void* s
           w_qr, 0, dq, 1, w_dq, 0, k.hidden, qr_f32.p, 0, nh * kRope, k.hidden, dq);
       MLA_TRY(cudaGetLastError());
     }
-    dim3 g((k.hidden + 255) / 256, (k.n_heads + 1) * kQK);
-    build_wqcat_kernel<<<g, 256, 0, st>>>(w_q, w_qr, (const __nv_bfloat16*)w->w_dkv,
-                                          (const __nv_bfloat16*)w->w_kr, w_uk, qabs_f32.p,
-                                          qr_f32.p, c->wqcat, k.hidden, k.n_heads, k.d_nope);
+    dim3 g((k.hidden + 255) / 256, (unsigned)c->wq_rows);
+    if (c->two_step) {
+      build_wq2_kernel<<<g, 256, 0, st>>>(w_q, w_qr, (const __nv_bfloat16*)w->w_dkv,
+                                          (const __nv_bfloat16*)w->w_kr, c->wqcat, k.hidden,
+                                          k.n_heads, c->latent_row0);
+      const int64_t n_uk = (int64_t)k.n_heads * mla::kQpNope * kLatent;
+      bf16_to_f16_kernel<<<(unsigned)((n_uk + 255) / 256), 256, 0, st>>>(
+          w_uk, c->wuk16, n_uk, c->status + mla::kStatusRangeWord);
+    } else {
+      build_wqcat_kernel<<<g, 256, 0, st>>>(w_q, w_qr, (const __nv_bfloat16*)w->w_dkv,
+                                            (const __nv_bfloat16*)w->w_kr, w_uk, qabs_f32.p,
+                                            qr_f32.p, c->wqcat, k.hidden, k.n_heads, k.d_nope);
+    }
     MLA_TRY(cudaGetLastError());
     dim3 g2((k.n_heads * kLatent + 255) / 256, k.hidden);
     build_wov_kernel<<<g2, 256, 0, st>>>((const __nv_bfloat16*)w->w_o,
@@ -1251,18 +1325,22 @@ mla_status mla_cache_create(const mla_config* cfg, const mla_weights* w, void* s
                       qd_cols * k.hidden * 2, 64, kOutBN, CU_TENSOR_MAP_SWIZZLE_128B)) != MLA_OK)
       return cleanup(s);
   }
-  s = make_map(&c->map_wqcat, c->wqcat, 2 * (uint64_t)k.hidden, (uint64_t)(k.n_heads + 1) * kQK, 1,
-               (uint64_t)k.hidden * 4, (uint64_t)(k.n_heads + 1) * kQK * k.hidden * 4, 64, kQK,
-               CU_TENSOR_MAP_SWIZZLE_128B);
-  if (s != MLA_OK) return cleanup(s);
-  s = make_map(&c->map_wqcat160, c->wqcat, 2 * (uint64_t)k.hidden, (uint64_t)(k.n_heads + 1) * kQK, 1,
-               (uint64_t)k.hidden * 4, (uint64_t)(k.n_heads + 1) * kQK * k.hidden * 4, 64, 160,
-               CU_TENSOR_MAP_SWIZZLE_128B);
-  if (s != MLA_OK) return cleanup(s);
-  s = make_map(&c->map_wqcat32, c->wqcat, 2 * (uint64_t)k.hidden, (uint64_t)(k.n_heads + 1) * kQK, 1,
-               (uint64_t)k.hidden * 4, (uint64_t)(k.n_heads + 1) * kQK * k.hidden * 4, 64, 32,
-               CU_TENSOR_MAP_SWIZZLE_128B);
-  if (s != MLA_OK) return cleanup(s);
+  {
+    const uint64_t wr = (uint64_t)c->wq_rows, wc = (uint64_t)c->wq_cols;
+    if ((s = make_map(&c->map_wqcat, c->wqcat, wc, wr, 1, wc * 2, wr * wc * 2, 64, kQK,
+                      CU_TENSOR_MAP_SWIZZLE_128B)) != MLA_OK ||
+        (s = make_map(&c->map_wqcat160, c->wqcat, wc, wr, 1, wc * 2, wr * wc * 2, 64, 160,
+                      CU_TENSOR_MAP_SWIZZLE_128B)) != MLA_OK ||
+        (s = make_map(&c->map_wqcat32, c->wqcat, wc, wr, 1, wc * 2, wr * wc * 2, 64, 32,
+                      CU_TENSOR_MAP_SWIZZLE_128B)) != MLA_OK)
+      return cleanup(s);
+    if (c->two_step) {
+      const uint64_t ur = (uint64_t)k.n_heads * mla::kQpNope;
+      if ((s = make_map(&c->map_wuk16, c->wuk16, kLatent, ur, 1, kLatent * 2, ur * kLatent * 2, 64,
+                        mla::kQpNope, CU_TENSOR_MAP_SWIZZLE_128B, true)) != MLA_OK)
+        return cleanup(s);
+    }
+  }
   s = make_map(&c->map_wov, c->wov, (uint64_t)k.n_heads * kLatent, k.hidden, 1,
                (uint64_t)k.n_heads * kLatent * 2, (uint64_t)k.hidden * k.n_heads * kLatent * 2,
                64, kOutBN, CU_TENSOR_MAP_SWIZZLE_128B, true);
@@ -1296,6 +1374,8 @@ mla_status mla_cache_create(const mla_config* cfg, const mla_weights* w, void* s
                    mla::GemmSmem<kOutBN, kOutAStages, kOutBStages>::kBytes);
     if (r == MLA_OK)
       r = set_smem(mla::dense_attn_kernel<kDenseStages>, mla::DenseSmem<kDenseStages>::kBytes);
+    if (r == MLA_OK)
+      r = set_smem(mla::query_proj_kernel, mla::QpSmem::kBytes);
     if (r == MLA_OK)
       r = set_smem(mla::window_attn_kernel<kAttnStages>,
                    mla::AttnSmem<kAttnStages>::kBytes);
@@ -1810,7 +1890,7 @@ mla_status mla_cache_copy_buffer(const mla_cache* c, mla_buffer which, void* hos
   switch (which) {
     case MLA_BUFFER_QP: src = c->qp; total = q_rows * kQK * 2; break;
     case MLA_BUFFER_O_LAT: src = c->o_lat; total = q_rows * kLatent * 2; break;
-    case MLA_BUFFER_W_QCAT: src = c->wqcat; total = (size_t)(k.n_heads + 1) * kQK * k.hidden * 4; break;
+    case MLA_BUFFER_W_QCAT: src = c->wqcat; total = (size_t)c->wq_rows * c->wq_cols * 2; break;
     case MLA_BUFFER_W_OV: src = c->wov; total = (size_t)k.hidden * k.n_heads * kLatent * 2; break;
     default: return fail(MLA_ERR_INVALID_ARGUMENT, "unknown buffer %d", (int)which);
   }

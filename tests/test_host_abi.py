@@ -139,9 +139,14 @@ def test_ring_bytes_reproduce_printed_accounting():
     assert B.mla_cache_device_bytes(cfg(d_latent=128)) == 0
     # The paper's 96 + 32 split enables the reconstruct-then-dense call, whose per-head weights
     # (W_Qd and W_O: 1536 x 1536 bf16 each, W_UV: 1536 x 192 and W_UK: 1152 x 192 fp16) come on top.
+    # Its query weights are the absorbed bf16 pairs (13 x 224 rows of 2 x 1536 bf16), while the
+    # full-rank d_nope = 128 query keeps the caller's rows (12 x 160 rows, padded to 2016, then
+    # 224 latent rows, of 1536 bf16) and W_UK (1536 x 192 fp16).
     wan = B.mla_cache_device_bytes(cfg(d_nope=128))
     paper = B.mla_cache_device_bytes(cfg(d_nope=96))
-    assert paper - wan == 2 * 1536 * 1536 * 2 + 1536 * 192 * 2 + 1152 * 192 * 2
+    pair = 13 * 224 * 2 * 1536 * 2
+    two_step = (2016 + 224) * 1536 * 2 + 1536 * 192 * 2
+    assert paper - wan == 2 * 1536 * 1536 * 2 + 1536 * 192 * 2 + 1152 * 192 * 2 + pair - two_step
     # A sink frame adds its padded region (1560 -> 1664 rows) to the planes.
     assert B.mla_cache_device_bytes(cfg(sink_frames=1)) - B.mla_cache_device_bytes(cfg()) == 1664 * 224 * 2
 
