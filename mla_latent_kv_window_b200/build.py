@@ -15,7 +15,7 @@ ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libmla.so")
 LIB_DEBUG = os.path.join(HERE, "libmla_debug.so")
 SOURCES = [os.path.join(HERE, "csrc", "mla_api.cu")]
-DEPS = SOURCES + [os.path.join(HERE, "csrc", f) for f in ("ptx.cuh", "gemm_tc.cuh", "window_attn.cuh", "dense_attn.cuh")] + \
+DEPS = SOURCES + [os.path.join(HERE, "csrc", f) for f in ("ptx.cuh", "gemm_tc.cuh", "query_proj.cuh", "window_attn.cuh", "dense_attn.cuh")] + \
     [os.path.join(ROOT, "include", "mla.h")]
 
 

@@ -47,3 +47,19 @@ def test_random_shapes_and_sequences(case):
                     o.append(x[b])
                 check_ring(p, f"fuzz {case}: after commit of {n}")
     p.gpu.close()
+
+
+@pytest.mark.parametrize("heads", [3, 5])
+def test_odd_head_counts(heads):
+    # Odd head counts: the query launch's column blocks (n_h heads + two latent blocks) and
+    # the output projection's 3 n_h k-blocks come out odd; every element against the oracle.
+    dims = dict(mla_synth.DIMS_WAN13B, hidden=128 * heads, n_heads=heads)
+    w = mla_synth.Workload(f"odd{heads}", frame_h=3, frame_w=7, window_frames=2, fill_frames=0,
+                           query_frames=2, batch=2, seed=7100 + heads, stream_scale=True,
+                           dims=tuple(sorted(dims.items())))
+    p = Pair(w, max_chunk_frames=2)
+    p.append(p.hidden(3, 91000 + heads))
+    check_ring(p, f"{heads} heads: after append")
+    full_check(p, p.hidden(2, 91100 + heads), f"{heads} heads: 2-frame chunk")
+    full_check(p, p.hidden(1, 91200 + heads), f"{heads} heads: 1-frame chunk")
+    p.gpu.close()
