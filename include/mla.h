@@ -133,15 +133,20 @@ size_t mla_ring_bytes(const mla_config* cfg);
  * 0 for an invalid config. */
 size_t mla_cache_device_bytes(const mla_config* cfg);
 
-/* Create a cache on the current device.  Derives and owns the absorbed weights
- *   W_Qabs[h] = W_UK[h]^T W_Q[h]   (hidden -> d_latent per head, queries; with a low-rank
- *                                   query W_UK[h]^T W_Q[h] W_DQ, and W_QR W_DQ for the RoPE part)
- *   W_OV[h]   = W_O[:, h] W_UV[h]  (d_latent per head -> hidden, outputs)
- * ([VideoMLA] §3.3 reconstructs per-head K/V from the latent through W_UK/W_UV; folding them
- * into the query and output projections is the standard MLA absorption), the RoPE tables and
- * a zeroed ring.  Synchronises `stream` once before returning, so the caller may free the
+/* Create a cache on the current device.  Owns the projection weights in the form the kernels
+ * multiply, the RoPE tables and a zeroed ring ([VideoMLA] §3.3 reconstructs per-head K/V from
+ * the latent through W_UK/W_UV; folding them into the query and output projections is the
+ * standard MLA absorption):
+ *   queries, full-rank W_Q with d_nope = 128: the caller's W_Q, W_QR, W_DKV, W_KR (bf16) and
+ *             W_UK (fp16); a query projection forms q = W_Q[h] x and then W_UK[h]^T q, so the
+ *             product W_UK[h]^T W_Q[h] is never rounded;
+ *   queries, other head splits or a low-rank query: W_Qabs[h] = W_UK[h]^T W_Q[h] (with a
+ *             low-rank query W_UK[h]^T W_Q[h] W_DQ, and W_QR W_DQ for the RoPE part) composed
+ *             in fp32 and kept as a bf16 pair hi + lo;
+ *   outputs:  W_OV[h] = W_O[:, h] W_UV[h] (d_latent per head -> hidden), fp16.
+ * Synchronises `stream` once before returning, so the caller may free the
  * weights afterwards.  *out receives the handle (NULL on failure).  MLA_ERR_RANGE (and no
- * cache) when an fp16 weight - W_OV, or the dense form's W_UK / W_UV - exceeds +-65504. */
+ * cache) when an fp16 weight - W_OV, W_UK, or the dense form's W_UK / W_UV - exceeds +-65504. */
 mla_status mla_cache_create(const mla_config* cfg, const mla_weights* w, void* stream,
                             mla_cache** out);
 
@@ -326,8 +331,12 @@ typedef struct {
   void* qp;           /* fp16 [batch][max_chunk*F*n_heads][d_latent + d_rope]: absorbed,
                          rotated queries of the last attention call, times scale * log2(e)   */
   void* o_lat;        /* fp16 [batch][max_chunk*F][n_heads*d_latent]: normalised P . c_kv     */
-  void* w_qcat;       /* bf16 [(n_heads+1)*(d_latent+d_rope)][hidden]: per head W_Qabs|W_QR,
-                         then W_DKV|W_KR                                                     */
+  void* w_qcat;       /* bf16 query and latent projection weights.  Full-rank W_Q with
+                         d_nope = 128: [L + d_latent + d_rope][hidden], per head W_Q[h] (128
+                         rows) and W_QR[h] (d_rope rows), zero rows up to L = n_heads * 160
+                         rounded up to a multiple of 224, then W_DKV and W_KR.  Otherwise
+                         [(n_heads+1)*(d_latent+d_rope)][2*hidden]: per head W_Qabs|W_QR,
+                         then W_DKV|W_KR, each row [hi | lo]                                 */
   void* w_ov;         /* fp16 [hidden][n_heads*d_latent]                                     */
   int64_t rows_per_stream;
 } mla_debug_buffers;
@@ -338,7 +347,7 @@ mla_status mla_cache_debug_buffers(const mla_cache* c, mla_debug_buffers* out);
 typedef enum {
   MLA_BUFFER_QP = 0,     /* Qp of the last attention call (fp16)   */
   MLA_BUFFER_O_LAT = 1,  /* o_lat of the last attention call (fp16) */
-  MLA_BUFFER_W_QCAT = 2, /* absorbed query + latent weights, rows [hi | lo] of 2 x hidden bf16 */
+  MLA_BUFFER_W_QCAT = 2, /* query + latent weights, bf16 (layout: w_qcat above)             */
   MLA_BUFFER_W_OV = 3    /* absorbed output weights (fp16)          */
 } mla_buffer;
 mla_status mla_cache_copy_buffer(const mla_cache* c, mla_buffer which, void* host_dst, size_t bytes,
@@ -349,7 +358,7 @@ mla_status mla_cache_copy_buffer(const mla_cache* c, mla_buffer which, void* hos
  * since the last read and clears them. */
 typedef enum {
   MLA_KERNEL_APPEND = 0,     /* fused down-projection + RoPE + ring write              */
-  MLA_KERNEL_QPROJ = 1,      /* absorbed query projection + RoPE + chunk latents       */
+  MLA_KERNEL_QPROJ = 1,      /* query projection (absorbed W_UK) + RoPE + chunk latents */
   MLA_KERNEL_ATTENTION = 2,  /* latent-window attention (scores, softmax, P . c_kv)    */
   MLA_KERNEL_OPROJ = 3,      /* absorbed output projection                             */
   MLA_KERNEL_COUNT = 4

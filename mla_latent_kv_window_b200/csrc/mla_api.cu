@@ -2,8 +2,11 @@
 // cache state, absorbed-weight derivation, tensor maps and kernel launches.
 //
 // Path of one attention call (VideoMLA paper page, §3.1-§3.3, App. D.4):
-//   1. tc_gemm<kEpiLatent>   x_chunk x [W_Qabs|W_QR per head ; W_DKV|W_KR]^T (tile shape per
-//                            launch from TileShape: 256 x 160 tiles for a one-frame chunk)
+//   1. query_proj_kernel     (full-rank W_Q, d_nope = 128) x_chunk x [W_Q|W_QR per head ;
+//                            W_DKV|W_KR]^T, then W_UK[h]^T q for each head in the same launch;
+//      or tc_gemm<kEpiLatent> (other head splits, low-rank query) x_chunk x [W_Qabs|W_QR per
+//                            head ; W_DKV|W_KR]^T with W_Qabs as a bf16 pair (tile shape per
+//                            launch from TileShape)
 //        heads  -> Qp[(q,h)] = [W_UK[h]^T q_nope | RoPE3D(q_rope)] * scale * log2 e
 //        latent -> chunk tail rows (c_kv, RoPE3D k_rope)
 //   2. window_attn_kernel     o_lat[(q,h)] = softmax(Qp . [c_kv|k_rope]^T) c_kv
@@ -605,8 +608,8 @@ std::vector<float2> make_rope_hw(const mla_config& cfg) {
   return tab;
 }
 
-// Launch the latent (and, with queries, the absorbed-query) projection GEMM over `rows` rows
-// of x per stream.  The latent rows land at cache rows [dst_row0, dst_row0 + rows) of every
+// Launch the latent (and, with queries, the query) projection over `rows` rows of x per
+// stream: query_proj_kernel for a full-rank query with d_nope = 128, else the absorbed-pair GEMM.  The latent rows land at cache rows [dst_row0, dst_row0 + rows) of every
 // stream; query rows go to qp ([batch][qp_tokens][n_heads * 224]).  The tile shape is the
 // TileShape candidate with the least estimated time: with queries 128 x 224, 256 x 160 or
 // 256 x 224 tiles; latent only 128 x 32 (seven column blocks, so that a one-frame append

@@ -63,14 +63,16 @@ def _f16(a):
     return np.asarray(a).astype(np.float16).astype(np.float64)
 
 
-def _rounding_model(dims, W, x_fill, xq, wq="pair"):
+def _rounding_model(dims, W, x_fill, xq, wq="two_step"):
     """The absorbed path in float64 with a 16-bit rounding exactly where the library stores 16-bit
-    values: the absorbed query weight W_UK[h]^T W_Q[h] (it multiplies the bf16 hidden states, so
-    it is bf16: wq="pair" carries it as hi + lo, two bf16 numbers, as the library does; "single"
-    rounds it to one bf16; "exact" keeps it in float64), the absorbed queries and the cache
-    planes (fp16), P and o_lat (fp16), W_OV (fp16) and the output (bf16).  Keys and queries are
-    rotated at absolute frame indices.  A model of where precision is lost at large input
-    scales."""
+    values.  The query's latent part W_UK[h]^T W_Q[h] x is formed in one of four ways:
+    wq="two_step" (the library's form for a full-rank query with d_nope = 128): q = W_Q[h] x in
+    fp32, carried as an fp16 pair hi + lo into the product with W_UK[h] (fp16); "pair": the
+    absorbed weight as a bf16 pair hi + lo (the library's form for other head splits);
+    "single": the absorbed weight rounded to one bf16; "exact": float64.  Then the absorbed
+    queries and the cache planes (fp16), P and o_lat (fp16), W_OV (fp16) and the output (bf16).
+    Keys and queries are rotated at absolute frame indices.  A model of where precision is lost
+    at large input scales."""
     nh, dn, dr, dv = dims["n_heads"], dims["d_nope"], dims["d_rope"], dims["d_head"]
     F, fw = dims["frame_h"] * dims["frame_w"], dims["frame_w"]
     rope = lambda v, t, h, w: rope3d(v, t, h, w, dims["rope_t"], dims["rope_h"], dims["rope_w"], dims["rope_base"])
@@ -88,14 +90,21 @@ def _rounding_model(dims, W, x_fill, xq, wq="pair"):
     scale = 1.0 / np.sqrt(dn + dr) / np.log(2.0)
     out = np.zeros((nq, dims["hidden"]))
     for h in range(nh):
-        wq_abs = Wd["w_uk"][h * dn:(h + 1) * dn].T @ Wd["w_q"][h * dn:(h + 1) * dn]
-        if wq == "single":
-            wq_abs = _bf16(wq_abs)
-        elif wq == "pair":
-            hi = _bf16(wq_abs)
-            wq_abs = hi + _bf16(wq_abs - hi)
+        w_uk = Wd["w_uk"][h * dn:(h + 1) * dn]
+        if wq == "two_step":
+            q = xqd @ Wd["w_q"][h * dn:(h + 1) * dn].T
+            q_hi = _f16(q)
+            q_nope = (q_hi + _f16(q - q_hi)) @ _f16(w_uk)
+        else:
+            wq_abs = w_uk.T @ Wd["w_q"][h * dn:(h + 1) * dn]
+            if wq == "single":
+                wq_abs = _bf16(wq_abs)
+            elif wq == "pair":
+                hi = _bf16(wq_abs)
+                wq_abs = hi + _bf16(wq_abs - hi)
+            q_nope = xqd @ wq_abs.T
         q_r = rope(xqd @ Wd["w_qr"][h * dr:(h + 1) * dr].T, t[-nq:], hh[-nq:], ww[-nq:])
-        qp = _f16(np.concatenate([xqd @ wq_abs.T, q_r], axis=1) * scale)
+        qp = _f16(np.concatenate([q_nope, q_r], axis=1) * scale)
         sc = qp @ keys.T
         P = np.exp2(sc - sc.max(axis=1, keepdims=True))
         o_lat = _f16((_f16(P) @ c) / P.sum(axis=1, keepdims=True))
@@ -110,8 +119,9 @@ def test_large_hidden_scales_stay_in_range_and_in_parity(scale):
     # range flag must stay clear.  Scores grow with scale^2; a softmax that sharp turns every
     # perturbation of the scores into an output error, and the absorbed query weight rounded to
     # a single bf16 (8 significant bits) would miss the bar at scales 8 and 32 (the rounding
-    # model prints by how much).  The library carries that weight as a bf16 pair, so the GPU
-    # must meet the bar against the oracle at every scale, and match its own rounding model.
+    # model prints by how much).  The library never rounds that product: it multiplies W_Q and
+    # then W_UK with q carried as an fp16 pair, so the GPU must meet the bar against the oracle
+    # at every scale, and match its own rounding model.
     import mla_latent_kv_window_b200 as M
     w = small(window=2, fill=2, q=1, seed=42)
     p = Pair(w)
