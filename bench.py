@@ -4,8 +4,10 @@
 One step = one rollout step of one attention layer at the Wan-1.3B geometry (hidden 1536,
 12 heads, latent 192 + RoPE 32, 30 x 52 = 1560 tokens per latent frame, 21-frame window):
 the 1560-token query frame attends to the window plus itself through the C ABI
-(mla_window_attention: query projection, window attention, output projection), then the frame
-is appended to the window (mla_cache_append: fused down-projection + RoPE + ring write).
+(mla_window_attention: query projection with the frame's own latents, window attention, output
+projection), then the frame joins the window (mla_cache_commit: its latents, which the query
+projection already computed, move into their ring slot).  The same step with the frame's
+latents recomputed by mla_cache_append is timed beside it.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -480,6 +482,7 @@ def run_ours(args, rank, local, world):
                 "algorithmic": f"{FLOP_PER_QHK} flop per (query, head, key) x {R} rows x {n_keys} keys "
                                f"= {attn_flop / 1e9:.1f} GFLOP per launch",
             },
+            "projection_rooflines": projection_rooflines(prof, dims, nq, tf_peak, peak_kind),
             "append_roofline": {
                 "kernel": "tc_gemm_kernel<224,latent> (21-frame fill; 20 back-to-back launches alternating two 100 MB inputs)",
                 "bound": "hbm", "status_ok": fill_ok,
@@ -509,6 +512,32 @@ def run_ours(args, rank, local, world):
             line["cpu_baseline"] = cpu
         print(json.dumps(line), flush=True)
     replicas.shutdown()
+
+
+def projection_rooflines(prof, dims, nq, tf_peak, peak_kind):
+    """The two projections of a step against the tensor peak, from the profiled pass's per-launch
+    CUDA-event times (each including its kernel boundary).  Algorithmic FLOPs are the absorbed
+    form's: the query launch 2 n_q hidden (n_h (d_latent + d_rope) + d_latent + d_rope) (the
+    queries and the chunk latents), the output launch 2 n_q hidden n_h d_latent; the query
+    launch's executed FLOPs (W_Q, W_QR, W_DKV, W_KR, then the W_UK product on an fp16 pair) are
+    given beside them."""
+    hid, nh, dc, dr, dn = dims["hidden"], dims["n_heads"], dims["d_latent"], dims["d_rope"], dims["d_nope"]
+    q_alg = 2.0 * nq * hid * (nh * (dc + dr) + dc + dr)
+    q_exec = 2.0 * nq * hid * (nh * (dn + dr) + dc + dr) + 2.0 * nq * nh * (2 * dn) * dc
+    o_alg = 2.0 * nq * hid * nh * dc
+    out = {}
+    for name, kern, flop, extra in (("query", "qproj", q_alg, {"executed_gflop": round(q_exec / 1e9, 2)}),
+                                    ("output", "oproj", o_alg, {})):
+        t, n = prof.get(kern, (0.0, 0))
+        if not n:
+            continue
+        ms = t / n
+        tf = flop / (ms / 1e3) / 1e12
+        out[name] = dict({"ms_per_launch": round(ms, 5), "gflop": round(flop / 1e9, 2),
+                          "achieved": round(tf, 1), "peak": tf_peak, "unit": "TFLOP/s",
+                          "frac": round(tf / tf_peak, 4), "bound": "tensor"}, **extra)
+    out["peak_source"] = f"{peak_kind} bf16 (burst)"
+    return out
 
 
 def _profiled_attention_ms(B, caches, fn, warm=1, reps=3):
