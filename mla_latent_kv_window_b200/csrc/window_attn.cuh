@@ -309,16 +309,26 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         rescale = true;
         l_sum *= alpha;
       }
-      float ps[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      // Exponentials of the keys in pairs: the subtraction of the running max and the row-sum
+      // additions run as packed fp32 pairs (4 partial sums of pairs).
+      const uint64_t m2 = f32x2_pack(m_used, m_used);
+      uint64_t ps[4] = {0ull, 0ull, 0ull, 0ull};
       uint32_t pk[kTileKeys / 2];
 #pragma unroll
       for (int i = 0; i < kTileKeys / 2; ++i) {
-        const float p0 = ex2_approx(s[2 * i] - m_used);
-        const float p1 = ex2_approx(s[2 * i + 1] - m_used);
+        float d0, d1;
+        f32x2_unpack(f32x2_sub(f32x2_pack(s[2 * i], s[2 * i + 1]), m2), d0, d1);
+        const float p0 = ex2_approx(d0);
+        const float p1 = ex2_approx(d1);
         pk[i] = pack_f16x2(p0, p1);
-        ps[i & 7] += p0 + p1;
+        ps[i & 3] = f32x2_add(ps[i & 3], f32x2_pack(p0, p1));
       }
-      l_sum += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
+      {
+        float a0, a1, b0, b1;
+        f32x2_unpack(f32x2_add(ps[0], ps[1]), a0, a1);
+        f32x2_unpack(f32x2_add(ps[2], ps[3]), b0, b1);
+        l_sum += (a0 + a1) + (b0 + b1);
+      }
 
       // P buffer and O become free once PV_{j-1} has completed.
       if (j >= 1 && !mbar_wait(pv_done, (uint32_t)(j - 1) & 1u, status)) { ok = false; break; }
