@@ -183,7 +183,8 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 }
 
 // ------------------------------------------------------------------------------ kernels
-// Create-time derivation of the absorbed weights (fp32 accumulation), stored as bf16 pairs:
+// Create-time derivation of the absorbed weights for the low-rank query and head splits other
+// than d_nope = 128 (fp32 accumulation), stored as bf16 pairs:
 // row r of Wqcat is [hi | lo] (2 * hidden columns), hi = bf16(w), lo = bf16(w - hi).  Rows,
 // per head h: [h*224, h*224+192) = W_UK[h]^T W_Q[h], [h*224+192, h*224+224) = W_QR[h];
 // then [n_h*224, n_h*224+192) = W_DKV and [n_h*224+192, (n_h+1)*224) = W_KR.  The absorbed
@@ -609,11 +610,12 @@ std::vector<float2> make_rope_hw(const mla_config& cfg) {
 }
 
 // Launch the latent (and, with queries, the query) projection over `rows` rows of x per
-// stream: query_proj_kernel for a full-rank query with d_nope = 128, else the absorbed-pair GEMM.  The latent rows land at cache rows [dst_row0, dst_row0 + rows) of every
-// stream; query rows go to qp ([batch][qp_tokens][n_heads * 224]).  The tile shape is the
-// TileShape candidate with the least estimated time: with queries 128 x 224, 256 x 160 or
-// 256 x 224 tiles; latent only 128 x 32 (seven column blocks, so that a one-frame append
-// spreads over 91 SMs instead of 13), 128 x 224 or 256 x 224.
+// stream: query_proj_kernel for a full-rank query with d_nope = 128, else the absorbed-pair
+// GEMM.  The latent rows land at cache rows [dst_row0, dst_row0 + rows) of every stream; query
+// rows go to qp ([batch][qp_tokens][n_heads * 224]).  The GEMM's tile shape is the TileShape
+// candidate with the least estimated time: with queries 128 x 224, 256 x 160 or 256 x 224
+// tiles; latent only 128 x 32 (seven column blocks, so that a one-frame append spreads over
+// 91 SMs instead of 13), 128 x 224 or 256 x 224.
 mla_status launch_latent_gemm(mla_cache* c, const void* x, int64_t rows, int64_t x_batch_rows,
                               bool with_queries, int64_t t0, int64_t dst_row0, cudaStream_t st,
                               __half* qp = nullptr, int64_t qp_tokens = 0) {
