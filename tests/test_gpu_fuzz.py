@@ -63,3 +63,20 @@ def test_odd_head_counts(heads):
     full_check(p, p.hidden(2, 91100 + heads), f"{heads} heads: 2-frame chunk")
     full_check(p, p.hidden(1, 91200 + heads), f"{heads} heads: 1-frame chunk")
     p.gpu.close()
+
+
+@pytest.mark.parametrize("d_nope", [96, 64])
+def test_full_rank_query_other_head_splits(d_nope):
+    # A full-rank query whose content part is not 128 wide keeps the absorbed query weight
+    # W_UK[h]^T W_Q[h] as a bf16 pair (the GEMM whose A column wraps), not the two-step query
+    # kernel; every element against the oracle, with stream scales and a ragged frame.
+    dims = dict(mla_synth.DIMS_WAN13B, d_nope=d_nope)
+    w = mla_synth.Workload(f"split{d_nope}", frame_h=3, frame_w=5, window_frames=2, fill_frames=0,
+                           query_frames=2, batch=2, seed=7200 + d_nope, stream_scale=True,
+                           dims=tuple(sorted(dims.items())))
+    p = Pair(w, max_chunk_frames=2)
+    p.append(p.hidden(3, 92000 + d_nope))
+    check_ring(p, f"d_nope {d_nope}: after append")
+    full_check(p, p.hidden(2, 92100 + d_nope), f"d_nope {d_nope}: 2-frame chunk")
+    full_check(p, p.hidden(1, 92200 + d_nope), f"d_nope {d_nope}: 1-frame chunk")
+    p.gpu.close()
