@@ -127,6 +127,13 @@ mla_status mla_ring_slot(const mla_config* cfg, int64_t frame, int32_t token, in
  * (16-bit cache). */
 size_t mla_ring_bytes(const mla_config* cfg);
 
+/* The same two host-only functions under the names of a cache: mla_cache_slot is mla_ring_slot
+ * for the configuration c was created with (MLA_ERR_INVALID_ARGUMENT for a NULL c or slot, and
+ * as mla_ring_slot otherwise); mla_cache_bytes is mla_ring_bytes (the ring footprint; 0 for a
+ * NULL or invalid config). */
+mla_status mla_cache_slot(const mla_cache* c, int64_t frame, int32_t token, int64_t* slot);
+size_t mla_cache_bytes(const mla_config* cfg);
+
 /* Bytes of device memory mla_cache_create allocates for this configuration (ring with its
  * chunk tail, absorbed weights, per-call scratch, status word, RoPE tables, and the per-head
  * weights of mla_window_attention_reconstruct when the configuration allows that call).

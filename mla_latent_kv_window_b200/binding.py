@@ -28,7 +28,8 @@ MLA_KERNEL_APPEND, MLA_KERNEL_QPROJ, MLA_KERNEL_ATTENTION, MLA_KERNEL_OPROJ = ra
 KERNEL_NAMES = ("append", "qproj", "attention", "oproj")
 
 EXPORTED = (
-    "mla_config_check", "mla_ring_slot", "mla_ring_bytes", "mla_cache_device_bytes",
+    "mla_config_check", "mla_ring_slot", "mla_ring_bytes", "mla_cache_slot", "mla_cache_bytes",
+    "mla_cache_device_bytes",
     "mla_cache_create", "mla_cache_append", "mla_cache_commit", "mla_commit_plan", "mla_window_attention",
     "mla_window_attention_noalloc",
     "mla_window_attention_reconstruct", "mla_cache_selftest_timeout", "mla_cache_selftest_bounds",
@@ -91,6 +92,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "mla_config_check": (I32, [P(mla_config)]),
         "mla_ring_slot": (I32, [P(mla_config), I64, I32, P(I64)]),
         "mla_ring_bytes": (ctypes.c_size_t, [P(mla_config)]),
+        "mla_cache_slot": (I32, [VP, I64, I32, P(I64)]),
+        "mla_cache_bytes": (ctypes.c_size_t, [P(mla_config)]),
         "mla_cache_device_bytes": (ctypes.c_size_t, [P(mla_config)]),
         "mla_cache_create": (I32, [P(mla_config), P(mla_weights), VP, P(VP)]),
         "mla_cache_append": (I32, [VP, VP, I32, VP]),
@@ -173,6 +176,17 @@ def mla_ring_slot(cfg: mla_config, frame: int, token: int) -> int:
 
 def mla_ring_bytes(cfg: mla_config) -> int:
     return int(load_library().mla_ring_bytes(ctypes.byref(cfg)))
+
+
+def mla_cache_slot(handle, frame: int, token: int) -> int:
+    """mla_ring_slot for the configuration the cache was created with."""
+    out = ctypes.c_int64()
+    _check(load_library().mla_cache_slot(handle, frame, token, ctypes.byref(out)), "mla_cache_slot")
+    return out.value
+
+
+def mla_cache_bytes(cfg: mla_config) -> int:
+    return int(load_library().mla_cache_bytes(ctypes.byref(cfg)))
 
 
 def mla_cache_device_bytes(cfg: mla_config) -> int:

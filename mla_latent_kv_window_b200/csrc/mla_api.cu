@@ -1076,6 +1076,11 @@ mla_status mla_ring_slot(const mla_config* cfg, int64_t frame, int32_t token, in
   return MLA_OK;
 }
 
+mla_status mla_cache_slot(const mla_cache* c, int64_t frame, int32_t token, int64_t* slot) {
+  if (!c) return fail(MLA_ERR_INVALID_ARGUMENT, "NULL cache");
+  return mla_ring_slot(&c->cfg, frame, token, slot);
+}
+
 mla_status mla_commit_plan(const mla_config* cfg, int64_t frames_appended, int32_t n_frames,
                            mla_row_move* moves, int32_t max_moves, int32_t* n_moves) {
   if (!cfg || !n_moves || (max_moves > 0 && !moves))
@@ -1115,6 +1120,8 @@ size_t mla_ring_bytes(const mla_config* cfg) {
   return (size_t)cfg->batch * (size_t)(cfg->sink_frames + cfg->window_frames) * cfg->frame_h *
          cfg->frame_w * (size_t)(cfg->d_latent + cfg->d_rope) * 2;
 }
+
+size_t mla_cache_bytes(const mla_config* cfg) { return mla_ring_bytes(cfg); }
 
 size_t mla_cache_device_bytes(const mla_config* cfg) {
   if (mla_config_check(cfg) != MLA_OK) return 0;

@@ -66,3 +66,18 @@ def test_commit_refuses_without_a_matching_chunk():
     assert p.gpu.state() == (4, 2)
     p.gpu.sync()
     p.gpu.close()
+
+
+@pytest.mark.parametrize("sink", [0, 1])
+def test_cache_slot_names_the_configs_rows(sink):
+    # mla_cache_slot reads the configuration the cache holds; it must name the rows that
+    # mla_ring_slot names for that configuration, sink region included.
+    import mla_latent_kv_window_b200 as M
+    w = small(3, 2, 1, seed=72 + sink, sink=sink)
+    p = Pair(w)
+    for f in (0, 1, 2, 3, 7, 10**6 + 1):
+        for k in (0, w.F - 1):
+            assert M.mla_cache_slot(p.gpu.handle, f, k) == M.mla_ring_slot(p.gpu.cfg, f, k)
+    with pytest.raises(M.MLAError):
+        M.mla_cache_slot(p.gpu.handle, -1, 0)
+    p.gpu.close()

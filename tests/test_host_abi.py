@@ -98,6 +98,18 @@ def test_ring_slot_matches_oracle_exactly():
         B.mla_ring_slot(cfg(), 0, 1560)
 
 
+def test_cache_named_slot_and_bytes():
+    # The boundary's cache-named forms: mla_cache_bytes is the ring footprint; mla_cache_slot
+    # reads the configuration of a cache, so without a GPU only its argument checks run.
+    for over in ({}, dict(batch=4), dict(sink_frames=1), dict(window_frames=63)):
+        assert B.mla_cache_bytes(cfg(**over)) == B.mla_ring_bytes(cfg(**over))
+    assert B.mla_cache_bytes(cfg(d_latent=0)) == 0
+    lib = B.load_library()
+    out = ctypes.c_int64(-5)
+    assert lib.mla_cache_slot(None, 0, 0, ctypes.byref(out)) == B.MLA_ERR_INVALID_ARGUMENT
+    assert out.value == -5
+
+
 def test_ring_slot_with_sink_matches_fifo_simulation():
     # Sink frames keep their own buffer for good (rows f*F of a sink region rounded up to whole
     # 128-row key tiles); the other frames cycle through W window buffers like a FIFO.  The
