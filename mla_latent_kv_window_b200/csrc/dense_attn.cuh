@@ -27,6 +27,13 @@ namespace mla {
 constexpr int kDenseThreads = 192;
 constexpr float kDenseRescaleLog2 = 8.0f;  // lazy O rescale when the max grows by > 2^8
 
+// a * b + c on packed fp32 pairs (one sm_100 instruction for both).
+__device__ __forceinline__ uint64_t dense_fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+
 template <int KV_STAGES>
 struct DenseSmem {
   static constexpr int kAtom = 128 * 128;                 // 128 rows x 64 bf16 (SW128)
@@ -225,17 +232,26 @@ __global__ void __launch_bounds__(kDenseThreads, 1)
         rescale = true;
         l_sum *= alpha;
       }
+      // Scaled, shifted scores and the row sums as packed fp32 pairs (4 partial sums of pairs).
       const float mc = m_used * c;
-      float ps[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      const uint64_t c2 = f32x2_pack(c, c), nmc2 = f32x2_pack(-mc, -mc);
+      uint64_t ps[4] = {0ull, 0ull, 0ull, 0ull};
       uint32_t pk[64];
 #pragma unroll
       for (int i = 0; i < 64; ++i) {
-        const float p0 = ex2_approx(fmaf(s[2 * i], c, -mc));
-        const float p1 = ex2_approx(fmaf(s[2 * i + 1], c, -mc));
+        float d0, d1;
+        f32x2_unpack(dense_fma2(f32x2_pack(s[2 * i], s[2 * i + 1]), c2, nmc2), d0, d1);
+        const float p0 = ex2_approx(d0);
+        const float p1 = ex2_approx(d1);
         pk[i] = pack_bf16x2(p0, p1);
-        ps[i & 7] += p0 + p1;
+        ps[i & 3] = f32x2_add(ps[i & 3], f32x2_pack(p0, p1));
       }
-      l_sum += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
+      {
+        float a0, a1, b0, b1;
+        f32x2_unpack(f32x2_add(ps[0], ps[1]), a0, a1);
+        f32x2_unpack(f32x2_add(ps[2], ps[3]), b0, b1);
+        l_sum += (a0 + a1) + (b0 + b1);
+      }
       if (j >= 1 && !mbar_wait(pv_done, (uint32_t)(j - 1) & 1u, status)) { ok = false; break; }
       tc_fence_after();
       if (__any_sync(0xffffffffu, rescale)) {
