@@ -9,7 +9,8 @@
 // Here both products multiply the caller's weights as given, and q enters the second product
 // as an fp16 pair hi + lo (hi = fp16(q), lo = fp16(q - hi); about 22 significant bits), so q
 // is carried essentially exactly.  The two products also cost less than the absorbed one:
-// 1536 x (128 + 32) then 128 x 192 multiply-adds per (token, head) instead of 1536 x 224.
+// 1536 x (128 + 32) then 2 x 128 x 192 (the pair) multiply-adds per (token, head), against
+// 1536 x 224 for one absorbed weight and twice that for it as a bf16 pair.
 //
 // Tiles: 256 rows (two M=128 halves sharing every weight k-block) x one column block of 160 B
 // rows.  B = [W_Q[0]; W_QR[0]; ...; W_Q[n_h-1]; W_QR[n_h-1]; zero rows; W_DKV; W_KR] (bf16,
