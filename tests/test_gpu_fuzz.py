@@ -80,3 +80,23 @@ def test_full_rank_query_other_head_splits(d_nope):
     full_check(p, p.hidden(2, 92100 + d_nope), f"d_nope {d_nope}: 2-frame chunk")
     full_check(p, p.hidden(1, 92200 + d_nope), f"d_nope {d_nope}: 1-frame chunk")
     p.gpu.close()
+
+
+def test_multi_tile_query_kernel_and_multi_wave_attention_every_element():
+    # 3 streams x a 2-frame chunk of 20 x 32 tokens: the query launch has 3 x 5 row tiles x 14
+    # column blocks = 210 tiles, so 62 of its 148 CTAs run two tiles (the accumulator reuse and
+    # phase bookkeeping across tiles), and the attention grid has 3 x 120 CTAs (more than two
+    # waves).  Every element of Qp and of the output against the oracle.
+    w = mla_synth.Workload("multitile", frame_h=20, frame_w=32, window_frames=2, fill_frames=0,
+                           query_frames=2, batch=3, seed=7300, stream_scale=True)
+    p = Pair(w, max_chunk_frames=2)
+    p.append(p.hidden(3, 93000))
+    check_ring(p, "multi-tile: after append")
+    x = p.hidden(2, 93100)
+    full_check(p, x, "multi-tile: 2-frame chunk")
+    p.gpu.commit(2)
+    for b, o in enumerate(p.oracles):
+        o.append(x[b])
+    check_ring(p, "multi-tile: after commit")
+    full_check(p, p.hidden(1, 93200), "multi-tile: 1-frame chunk after the commit")
+    p.gpu.close()
